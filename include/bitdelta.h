@@ -1,0 +1,207 @@
+/*
+ * bitdelta.h — C ABI of the B200 (sm_100a) BitDelta library (libbitdelta.so).
+ *
+ * Two halves of one method:
+ *   compress : Delta = W_fine - W_base, optional k-sigma clip, abs-mean scales, sign bits
+ *              ("bitdelta" page, "How BitDelta Works" 1-4 and "Safety Benefits:
+ *              1. Outlier Clipping"; "Per-Axis Weight Deltas", "Key Contributions" 1).
+ *   apply    : y_t = W_base x_t + Delta_hat_{u(t)} x_t for a batch whose tokens belong to
+ *              different tenants u ("BitDelta Guide: 1-Bit Delta Quantization for LLM
+ *              Serving", "Systems Mechanics: 1. Decoupled Forward Pass").
+ *
+ * Conventions for every entry point
+ *   - Pointers are DEVICE pointers unless the argument says "host". The caller owns and
+ *     allocates every buffer (workspace included); the library never allocates device
+ *     memory and never frees a caller's buffer.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*; NULL = the
+ *     legacy default stream). Nothing synchronises the host except bd_get_status and
+ *     bd_profile_collect, which say so.
+ *   - Argument errors that the host can see are returned before anything is launched and
+ *     leave outputs untouched. Errors only the device can see (a tenant id out of range,
+ *     a wait that ran out) set bits in a status word inside the workspace; no kernel
+ *     traps. Read it with bd_get_status.
+ *   - Matrices are [d_out][d_in] row-major (the [Out, In] layout of an nn.Linear weight).
+ *   - Sign words: uint32 signs[d_out][d_in/32], packed along the input axis; column
+ *     32*w + j of a row is bit j of its word w (least significant bit first). Bit 1 means
+ *     +1 and bit 0 means -1; sign(0) = +1 (-0.0 included), i.e. bit = !(delta_c < 0).
+ *   - Alignment: every pointer to a matrix, sign array or scale array must be 16-byte
+ *     aligned (128-bit loads and bulk copies), else BD_ERR_ALIGN.
+ *   - Shapes: d_out >= 1, d_in >= 32 and d_in % 32 == 0, else BD_ERR_SHAPE.
+ *
+ * The float arithmetic (fp32 accumulation) and what each result is compared with are
+ * described per call below.
+ */
+#ifndef BITDELTA_H
+#define BITDELTA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---------------------------------------------------------------------------------- */
+/* status, types                                                                       */
+/* ---------------------------------------------------------------------------------- */
+typedef enum {
+  BD_OK = 0,
+  BD_ERR_NULL = 1,          /* a required pointer is NULL                              */
+  BD_ERR_SHAPE = 2,         /* sizes out of range or not divisible as required        */
+  BD_ERR_DTYPE = 3,         /* a dtype code the call does not accept                   */
+  BD_ERR_ALIGN = 4,         /* a pointer is not 16-byte aligned                        */
+  BD_ERR_CONFIG = 5,        /* bad compress config / scale mode / group size           */
+  BD_ERR_CUDA = 6,          /* a CUDA runtime call failed (launch error etc.)          */
+  BD_ERR_TENANT_RANGE = 7,  /* device status: a tenant id outside [-1, n_tenants)      */
+  BD_ERR_TIMEOUT = 8,       /* device status: a bounded wait gave up                   */
+  BD_ERR_WORKSPACE = 9,     /* workspace NULL or smaller than the *_workspace_size     */
+  BD_ERR_TENANT_RECORD = 10 /* device status: a bd_tenant record is invalid            */
+} bd_status;
+
+typedef enum { BD_F32 = 0, BD_BF16 = 1, BD_F16 = 2 } bd_dtype;
+
+/* Scale granularity.
+ *  GROUP : one scale per contiguous run of group_size entries along d_in,
+ *          scales[d_out][d_in/group_size] ("2. Group Quantization", default 128).
+ *  ROW   : one scale per output row, scales[d_out]  (the 1 x d_out vector of
+ *          "Per-Axis Weight Deltas").
+ *  COL   : one scale per input column, scales[d_in] (the d_in x 1 vector).
+ *  TENSOR: one scalar alpha for the whole matrix, scales[1] ("BitDelta Guide",
+ *          "2. Optimal L2 Norm Initialization").
+ * Every scale is the abs-mean of its slice of the clipped delta, the L2-optimal
+ * value for fixed signs. */
+typedef enum { BD_SCALE_GROUP = 0, BD_SCALE_ROW = 1, BD_SCALE_COL = 2, BD_SCALE_TENSOR = 3 } bd_scale_mode;
+
+/* Device status bits (bd_get_status). */
+#define BD_DEV_TENANT_RANGE 0x1u  /* some token had a tenant id outside [-1, n_tenants) */
+#define BD_DEV_TIMEOUT      0x2u  /* a bounded wait inside a kernel gave up              */
+#define BD_DEV_TENANT_RECORD 0x4u /* a bd_tenant record had a bad mode, group size or
+                                     NULL / misaligned pointer; its tokens got the base
+                                     product only                                      */
+
+/* ---------------------------------------------------------------------------------- */
+/* compress                                                                            */
+/* ---------------------------------------------------------------------------------- */
+typedef struct {
+  int32_t group_size; /* GROUP mode: power of two, 32 <= G, G divides d_in. Ignored otherwise. */
+  int32_t mode;       /* bd_scale_mode                                                    */
+  int32_t clip;       /* 0: no clip; 1: clamp delta to [mean - k*std, mean + k*std]       */
+  float clip_k;       /* k of the clip (the pages use 3; 2 for "aggressive")            */
+} bd_compress_cfg;
+
+/* Bytes of workspace bd_compress needs for this shape and config (0 is possible). */
+size_t bd_compress_workspace_size(int64_t d_out, int64_t d_in, const bd_compress_cfg* cfg /* host */);
+
+/* bd_compress — the compress half: Delta = W_fine - W_base (computed in fp32 from the
+ * stored values), optional whole-matrix k-sigma clip with the unbiased (N-1) standard
+ * deviation accumulated in fp64, abs-mean scales over the clipped delta (fp32 sums in a
+ * fixed tree order, so results are deterministic), and sign bits of the clipped delta.
+ * Follows "bitdelta" page, "1. Delta Computation", "2. Group Quantization",
+ * "3. 1-bit Quantization", "Outlier Clipping", and the per-axis vectors of "Per-Axis
+ * Weight Deltas".
+ *
+ *   w_base, w_fine : [d_out][d_in], dtype BD_F32 or BD_BF16.
+ *   cfg            : host pointer; see bd_compress_cfg.
+ *   signs_out      : uint32[d_out][d_in/32], fully overwritten.
+ *   scales_out     : fp32, [d_out][d_in/G] (GROUP), [d_out] (ROW), [d_in] (COL), [1] (TENSOR).
+ *   stats_out      : optional (may be NULL) fp64[4] = {mean, std, lo, hi} of the delta;
+ *                    written only when cfg->clip is set.
+ *   workspace      : device scratch of bd_compress_workspace_size() bytes (16-byte aligned);
+ *                    may be NULL only when that size is 0.
+ * Signs are bit-exact with the fp64 definition (the sign of an fp32 difference is the
+ * sign of the exact difference); scales agree with it to ~1e-6 relative.
+ * Returns BD_OK or a host-detected error; nothing is written on error. */
+bd_status bd_compress(const void* w_base, const void* w_fine, int32_t dtype, int64_t d_out,
+                      int64_t d_in, const bd_compress_cfg* cfg, uint32_t* signs_out,
+                      float* scales_out, double* stats_out, void* workspace, size_t ws_bytes,
+                      void* stream);
+
+/* ---------------------------------------------------------------------------------- */
+/* reconstruct                                                                         */
+/* ---------------------------------------------------------------------------------- */
+/* bd_reconstruct — Delta_hat = sign * scale ("4. Reconstruction"); with w_base given,
+ * the personalised weight W_base + Delta_hat ("5. Serving").
+ *   signs      : uint32[d_out][d_in/32].
+ *   scales     : per `mode` as in bd_compress, dtype scale_dtype (BD_F32 or BD_F16).
+ *   w_base     : optional [d_out][d_in] of w_dtype (BD_F32 or BD_BF16), or NULL.
+ *   out        : [d_out][d_in] of out_dtype (BD_F32 or BD_BF16; bf16 is rounded to nearest
+ *                even from the fp32 value).
+ * The fp32 result is exact for fp16/fp32 scales when w_base is NULL. */
+bd_status bd_reconstruct(const uint32_t* signs, const void* scales, int32_t scale_dtype,
+                         int32_t mode, int32_t group_size, int64_t d_out, int64_t d_in,
+                         const void* w_base, int32_t w_dtype, void* out, int32_t out_dtype,
+                         void* stream);
+
+/* ---------------------------------------------------------------------------------- */
+/* multi-tenant apply                                                                  */
+/* ---------------------------------------------------------------------------------- */
+/* One resident tenant variant of one projection. An array of these lives in DEVICE
+ * memory and is read by the kernels (the host never dereferences it). */
+typedef struct {
+  const uint32_t* signs;  /* device, uint32[d_out][d_in/32], 16-byte aligned           */
+  const void* scales;     /* device, per `mode`, dtype = the call's scale_dtype          */
+  int32_t mode;           /* bd_scale_mode                                               */
+  int32_t group_size;     /* GROUP mode: power of two, 32 <= G, G divides d_in           */
+} bd_tenant;
+
+/* Bytes of workspace bd_apply_multi needs. */
+size_t bd_apply_workspace_size(int64_t d_out, int64_t d_in, int64_t batch, int32_t n_tenants);
+
+/* bd_apply_multi — decomposed multi-tenant forward of one linear projection:
+ *     y[t] = W_base x[t] + Delta_hat_{u(t)} x[t],   u(t) = tenant_ids[t]
+ * ("BitDelta Guide", "Systems Mechanics: 1. Decoupled Forward Pass", and "2. Fused
+ * Dequantization": sign bits stay packed in memory and are unpacked on chip).
+ * The base product W_base X is computed once for the whole batch; the tokens are
+ * grouped by tenant on the device (no host synchronisation) and each tenant's packed
+ * signs and scales are streamed once per group of its tokens.
+ *
+ *   w_base      : [d_out][d_in], w_dtype BD_BF16 (tensor-core path) or BD_F32.
+ *   tenants     : device array of n_tenants bd_tenant records (n_tenants >= 0).
+ *   scale_dtype : BD_F16 or BD_F32, for every tenant's scales.
+ *   tenant_ids  : device int32[batch]; -1 = base model only. Ids outside [-1, n_tenants)
+ *                 set BD_DEV_TENANT_RANGE and that token gets the base product only.
+ *                 A tenant record that is invalid (mode, group size, NULL or unaligned
+ *                 pointer) sets BD_DEV_TENANT_RECORD and its tokens get the base only.
+ *   x           : [batch][d_in], same dtype as w_base.
+ *   y           : [batch][d_out], y_dtype BD_BF16 (round to nearest even) or BD_F32.
+ *   workspace   : bd_apply_workspace_size() bytes, 16-byte aligned. Its status word is
+ *                 reset by this call, so bd_get_status reports the latest call.
+ * Products are accumulated in fp32. batch may be 0 (nothing is launched).
+ * Returns BD_OK or a host-detected error. */
+bd_status bd_apply_multi(const void* w_base, int32_t w_dtype, int64_t d_out, int64_t d_in,
+                         const bd_tenant* tenants, int32_t n_tenants, int32_t scale_dtype,
+                         const int32_t* tenant_ids, const void* x, int64_t batch, void* y,
+                         int32_t y_dtype, void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------- */
+/* status, diagnostics                                                                 */
+/* ---------------------------------------------------------------------------------- */
+/* Copies the device status word of a workspace (compress or apply) to *flags (host)
+ * and SYNCHRONISES `stream`. Returns BD_ERR_TIMEOUT, BD_ERR_TENANT_RECORD or
+ * BD_ERR_TENANT_RANGE (in that order of precedence) when the corresponding bit is set,
+ * BD_OK when none is. */
+bd_status bd_get_status(const void* workspace, uint32_t* flags /* host, may be NULL */,
+                        void* stream);
+
+/* Static description of a status code. */
+const char* bd_status_string(int32_t status);
+
+/* Kernel launch accounting: the number of kernels this library has launched since it
+ * was loaded (all calls, all streams). */
+int64_t bd_launch_count(void);
+
+/* Optional per-kernel timing. While enabled, every kernel the library launches is
+ * bracketed by two CUDA events recorded on its launch stream (at most `capacity`
+ * launches are recorded; later ones are counted but not timed). bd_profile_collect
+ * SYNCHRONISES on the recorded events, writes per kernel kind the number of timed
+ * launches and their summed duration in milliseconds, clears the records and returns
+ * the number of kernel kinds (array length written, <= max_kinds). */
+bd_status bd_profile_enable(int32_t on, int32_t capacity);
+int32_t bd_profile_collect(int64_t* launches /* host */, double* total_ms /* host */,
+                           int32_t max_kinds);
+const char* bd_kernel_name(int32_t kind);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BITDELTA_H */

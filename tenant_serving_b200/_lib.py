@@ -1,0 +1,272 @@
+"""ctypes binding of libbitdelta.so: argument marshalling only.
+
+Every function here forwards to the C entry point of the same name. PyTorch provides
+device memory (``torch.empty`` on the GPU) and the current CUDA stream; all arithmetic of
+the method runs in the library's kernels. There is no CPU path: if the library or a GPU
+is missing, the calls raise.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import c_double, c_float, c_int32, c_int64, c_size_t, c_uint32, c_void_p, POINTER
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libbitdelta.so")
+
+# status codes (include/bitdelta.h)
+BD_OK = 0
+BD_ERR_NULL = 1
+BD_ERR_SHAPE = 2
+BD_ERR_DTYPE = 3
+BD_ERR_ALIGN = 4
+BD_ERR_CONFIG = 5
+BD_ERR_CUDA = 6
+BD_ERR_TENANT_RANGE = 7
+BD_ERR_TIMEOUT = 8
+BD_ERR_WORKSPACE = 9
+BD_ERR_TENANT_RECORD = 10
+
+BD_F32, BD_BF16, BD_F16 = 0, 1, 2
+BD_SCALE_GROUP, BD_SCALE_ROW, BD_SCALE_COL, BD_SCALE_TENSOR = 0, 1, 2, 3
+BD_DEV_TENANT_RANGE, BD_DEV_TIMEOUT, BD_DEV_TENANT_RECORD = 0x1, 0x2, 0x4
+
+EXPORTS = (
+    "bd_compress", "bd_compress_workspace_size", "bd_reconstruct", "bd_apply_multi",
+    "bd_apply_workspace_size", "bd_get_status", "bd_status_string", "bd_launch_count",
+    "bd_profile_enable", "bd_profile_collect", "bd_kernel_name",
+)
+
+
+class bd_compress_cfg(ctypes.Structure):
+    _fields_ = [("group_size", c_int32), ("mode", c_int32), ("clip", c_int32), ("clip_k", c_float)]
+
+
+class bd_tenant(ctypes.Structure):
+    _fields_ = [("signs", c_void_p), ("scales", c_void_p), ("mode", c_int32), ("group_size", c_int32)]
+
+
+class BitDeltaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)} (status {code})")
+
+
+_LIB = None
+
+
+def lib():
+    """Load (once) and return the shared library; raise if it is not built."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"libbitdelta.so is not built ({LIB_PATH}); run "
+                           "`python -m tenant_serving_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    L.bd_compress.argtypes = [c_void_p, c_void_p, c_int32, c_int64, c_int64,
+                              POINTER(bd_compress_cfg), c_void_p, c_void_p, c_void_p, c_void_p,
+                              c_size_t, c_void_p]
+    L.bd_compress.restype = c_int32
+    L.bd_compress_workspace_size.argtypes = [c_int64, c_int64, POINTER(bd_compress_cfg)]
+    L.bd_compress_workspace_size.restype = c_size_t
+    L.bd_reconstruct.argtypes = [c_void_p, c_void_p, c_int32, c_int32, c_int32, c_int64, c_int64,
+                                 c_void_p, c_int32, c_void_p, c_int32, c_void_p]
+    L.bd_reconstruct.restype = c_int32
+    L.bd_apply_multi.argtypes = [c_void_p, c_int32, c_int64, c_int64, c_void_p, c_int32, c_int32,
+                                 c_void_p, c_void_p, c_int64, c_void_p, c_int32, c_void_p,
+                                 c_size_t, c_void_p]
+    L.bd_apply_multi.restype = c_int32
+    L.bd_apply_workspace_size.argtypes = [c_int64, c_int64, c_int64, c_int32]
+    L.bd_apply_workspace_size.restype = c_size_t
+    L.bd_get_status.argtypes = [c_void_p, POINTER(c_uint32), c_void_p]
+    L.bd_get_status.restype = c_int32
+    L.bd_status_string.argtypes = [c_int32]
+    L.bd_status_string.restype = ctypes.c_char_p
+    L.bd_launch_count.argtypes = []
+    L.bd_launch_count.restype = c_int64
+    L.bd_profile_enable.argtypes = [c_int32, c_int32]
+    L.bd_profile_enable.restype = c_int32
+    L.bd_profile_collect.argtypes = [POINTER(c_int64), POINTER(c_double), c_int32]
+    L.bd_profile_collect.restype = c_int32
+    L.bd_kernel_name.argtypes = [c_int32]
+    L.bd_kernel_name.restype = ctypes.c_char_p
+    _LIB = L
+    return L
+
+
+def status_string(code: int) -> str:
+    try:
+        return lib().bd_status_string(int(code)).decode()
+    except Exception:
+        return "unknown"
+
+
+def check(code: int, where: str):
+    if code != BD_OK:
+        raise BitDeltaError(code, where)
+
+
+# ----------------------------------------------------------------------------------
+# torch marshalling
+# ----------------------------------------------------------------------------------
+def _torch():
+    import torch
+    return torch
+
+
+def dtype_code(t) -> int:
+    torch = _torch()
+    m = {torch.float32: BD_F32, torch.bfloat16: BD_BF16, torch.float16: BD_F16}
+    if t.dtype not in m:
+        raise TypeError(f"unsupported dtype {t.dtype}")
+    return m[t.dtype]
+
+
+def _ptr(t):
+    return None if t is None else c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return c_void_p(s.cuda_stream)
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("tensors passed to the library must live on the GPU")
+
+
+def compress_cfg(mode=BD_SCALE_GROUP, group_size=128, clip=False, clip_k=3.0) -> bd_compress_cfg:
+    return bd_compress_cfg(int(group_size), int(mode), 1 if clip else 0, float(clip_k))
+
+
+def scales_shape(mode, d_out, d_in, group_size):
+    if mode == BD_SCALE_GROUP:
+        return (d_out, d_in // group_size)
+    if mode == BD_SCALE_ROW:
+        return (d_out,)
+    if mode == BD_SCALE_COL:
+        return (d_in,)
+    return (1,)
+
+
+def bd_compress_workspace_size(d_out, d_in, cfg: bd_compress_cfg) -> int:
+    return int(lib().bd_compress_workspace_size(int(d_out), int(d_in), ctypes.byref(cfg)))
+
+
+def bd_compress(w_base, w_fine, cfg: bd_compress_cfg, signs=None, scales=None, stats=None,
+                workspace=None, stream=None):
+    """Wrap ``bd_compress``. Allocates missing outputs with torch on the inputs' device.
+    Returns ``(signs int32[d_out, d_in//32] holding the uint32 words, scales fp32,
+    stats fp64[4] or None)``."""
+    torch = _torch()
+    _require_cuda(w_base, w_fine)
+    d_out, d_in = w_base.shape
+    dev = w_base.device
+    if signs is None:
+        signs = torch.empty((d_out, d_in // 32), dtype=torch.int32, device=dev)
+    if scales is None:
+        scales = torch.empty(scales_shape(cfg.mode, d_out, d_in, cfg.group_size),
+                             dtype=torch.float32, device=dev)
+    if stats is None and cfg.clip:
+        stats = torch.zeros(4, dtype=torch.float64, device=dev)
+    ws = bd_compress_workspace_size(d_out, d_in, cfg)
+    if workspace is None:
+        workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=dev)
+    rc = lib().bd_compress(_ptr(w_base), _ptr(w_fine), dtype_code(w_base), d_out, d_in,
+                           ctypes.byref(cfg), _ptr(signs), _ptr(scales), _ptr(stats),
+                           _ptr(workspace), workspace.numel(), _stream(stream))
+    check(rc, "bd_compress")
+    return signs, scales, stats
+
+
+def bd_reconstruct(signs, scales, mode, group_size, d_out, d_in, w_base=None, out=None,
+                   out_dtype=None, stream=None):
+    torch = _torch()
+    _require_cuda(signs, scales, w_base)
+    if out is None:
+        out = torch.empty((d_out, d_in), dtype=out_dtype or torch.float32, device=signs.device)
+    rc = lib().bd_reconstruct(_ptr(signs), _ptr(scales), dtype_code(scales), int(mode),
+                              int(group_size), int(d_out), int(d_in), _ptr(w_base),
+                              dtype_code(w_base) if w_base is not None else BD_F32, _ptr(out),
+                              dtype_code(out), _stream(stream))
+    check(rc, "bd_reconstruct")
+    return out
+
+
+class TenantTable:
+    """A device array of ``bd_tenant`` records for one projection. Keeps references to
+    the tensors it points at so they stay alive as long as the table does."""
+
+    def __init__(self, tenants, device):
+        torch = _torch()
+        self._keep = []
+        n = len(tenants)
+        arr = (bd_tenant * max(n, 1))()
+        for i, (signs, scales, mode, group_size) in enumerate(tenants):
+            _require_cuda(signs, scales)
+            arr[i] = bd_tenant(signs.data_ptr(), scales.data_ptr(), int(mode), int(group_size))
+            self._keep.append((signs, scales))
+        raw = bytes(arr)
+        self.n = n
+        self.scale_dtype = dtype_code(tenants[0][1]) if n else BD_F16
+        host = torch.frombuffer(bytearray(raw), dtype=torch.uint8)
+        self.dev = host.to(device)
+
+    def ptr(self):
+        return c_void_p(self.dev.data_ptr())
+
+
+def bd_apply_workspace_size(d_out, d_in, batch, n_tenants) -> int:
+    return int(lib().bd_apply_workspace_size(int(d_out), int(d_in), int(batch), int(n_tenants)))
+
+
+def bd_apply_multi(w_base, table: TenantTable, tenant_ids, x, y=None, y_dtype=None,
+                   workspace=None, stream=None):
+    """Wrap ``bd_apply_multi``: y[t] = W_base x[t] + Delta_hat_{ids[t]} x[t]."""
+    torch = _torch()
+    _require_cuda(w_base, tenant_ids, x)
+    d_out, d_in = w_base.shape
+    batch = x.shape[0]
+    if y is None:
+        y = torch.empty((batch, d_out), dtype=y_dtype or torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(max(bd_apply_workspace_size(d_out, d_in, batch, table.n), 16),
+                                dtype=torch.uint8, device=x.device)
+    rc = lib().bd_apply_multi(_ptr(w_base), dtype_code(w_base), d_out, d_in, table.ptr(), table.n,
+                              table.scale_dtype, _ptr(tenant_ids), _ptr(x), batch, _ptr(y),
+                              dtype_code(y), _ptr(workspace), workspace.numel(), _stream(stream))
+    check(rc, "bd_apply_multi")
+    return y, workspace
+
+
+def bd_get_status(workspace, stream=None):
+    """Returns (status code, flags). Synchronises the stream."""
+    f = c_uint32(0)
+    rc = lib().bd_get_status(_ptr(workspace), ctypes.byref(f), _stream(stream))
+    return int(rc), int(f.value)
+
+
+def bd_launch_count() -> int:
+    return int(lib().bd_launch_count())
+
+
+def bd_profile_enable(on: bool, capacity: int = 65536):
+    check(lib().bd_profile_enable(1 if on else 0, int(capacity)), "bd_profile_enable")
+
+
+def bd_profile_collect():
+    """{kernel name: (timed launches, total ms)} for kernels launched while enabled."""
+    n = 32
+    la = (c_int64 * n)()
+    ms = (c_double * n)()
+    k = lib().bd_profile_collect(la, ms, n)
+    out = {}
+    for i in range(k):
+        if la[i]:
+            out[lib().bd_kernel_name(i).decode()] = (int(la[i]), float(ms[i]))
+    return out

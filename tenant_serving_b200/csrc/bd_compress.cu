@@ -1,0 +1,578 @@
+// bd_compress: the compress half of BitDelta on sm_100a.
+//
+// Method ("bitdelta" page, "How BitDelta Works" 1-3 and "Safety Benefits: 1. Outlier
+// Clipping"; per-axis vectors from "Per-Axis Weight Deltas", "Key Contributions" 1):
+//   delta = W_fine - W_base; optional clamp to [mean - k std, mean + k std] over the whole
+//   matrix; scale = mean |delta_c| over each group / row / column / the whole matrix;
+//   sign bit = !(delta_c < 0), packed LSB-first along d_in into uint32 words.
+//
+// Kernels (all HBM-bound streams; 16-byte coalesced loads of both inputs):
+//   k_delta_stats      pass 1 when clipping: shifted fp32 sums per 16-byte vector,
+//                      accumulated in fp64 per thread, one (S1, S2) pair per block.
+//   k_stats_final      one block merges the block pairs in a fixed order -> mean, std,
+//                      lo, hi and the fp32 thresholds the main pass compares with.
+//   k_scale_signpack   main pass for GROUP / ROW / TENSOR: a warp streams a segment of
+//                      one row, 16 bytes per lane per input; signs are packed with two
+//                      (bf16) or three (fp32) xor-shuffles of per-lane bit masks; group
+//                      sums are xor-shuffle trees; row / tensor sums go to fp64 partials.
+//   k_col_scale_signpack  COL mode: a warp walks a tile of rows of one column chunk,
+//                      keeping fp64 column sums in registers; fp64 partials per tile.
+//   k_scale_final      fixed-order reduction of the partials into row / column / tensor
+//                      scales (deterministic, no atomics).
+#include "bd_internal.cuh"
+
+#include <math.h>
+
+namespace bd {
+
+struct ClipParams {
+  double mean, stddev, lo, hi;
+  float lo_up;   // smallest float >= lo:  x < lo  <=>  x < lo_up   (x a float)
+  float hi_dn;   // largest float <= hi:   x > hi  <=>  x > hi_dn
+  float lo_val;  // value a clamped-low entry takes (lo rounded, sign kept)
+  float hi_val;  // value a clamped-high entry takes
+};
+
+// ------------------------------------------------------------------------------------
+// element access: 16 bytes of W_base and W_fine -> VEC deltas in fp32
+// ------------------------------------------------------------------------------------
+template <bool BF16>
+struct Vec;
+template <>
+struct Vec<true> {  // 8 bf16 per 16 bytes
+  static constexpr int N = 8;
+  __device__ __forceinline__ static void delta(const uint4& b, const uint4& f, float* d) {
+    const uint32_t bb[4] = {b.x, b.y, b.z, b.w};
+    const uint32_t ff[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      d[2 * k] = bf16lo(ff[k]) - bf16lo(bb[k]);
+      d[2 * k + 1] = bf16hi(ff[k]) - bf16hi(bb[k]);
+    }
+  }
+};
+template <>
+struct Vec<false> {  // 4 fp32 per 16 bytes
+  static constexpr int N = 4;
+  __device__ __forceinline__ static void delta(const uint4& b, const uint4& f, float* d) {
+    d[0] = __uint_as_float(f.x) - __uint_as_float(b.x);
+    d[1] = __uint_as_float(f.y) - __uint_as_float(b.y);
+    d[2] = __uint_as_float(f.z) - __uint_as_float(b.z);
+    d[3] = __uint_as_float(f.w) - __uint_as_float(b.w);
+  }
+};
+
+__device__ __forceinline__ float clamp_delta(float d, const ClipParams& c) {
+  // Comparisons against the float thresholds are exactly the comparisons of the float
+  // delta with the fp64 bounds; the replacement keeps the sign of the fp64 bound.
+  return d < c.lo_up ? c.lo_val : (d > c.hi_dn ? c.hi_val : d);
+}
+
+// ------------------------------------------------------------------------------------
+// pass 1: shifted sums for mean / std
+// ------------------------------------------------------------------------------------
+template <bool BF16>
+__global__ void __launch_bounds__(256) k_delta_stats(const uint4* __restrict__ wb,
+                                                     const uint4* __restrict__ wf,
+                                                     int64_t nvec, double* __restrict__ partials) {
+  using V = Vec<BF16>;
+  // shift: delta of element 0 (every thread computes the same value)
+  float shift;
+  {
+    float d0[V::N];
+    V::delta(wb[0], wf[0], d0);
+    shift = d0[0];
+  }
+  double s1 = 0.0, s2 = 0.0;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  for (; i + 3 * stride < nvec; i += 4 * stride) {
+    uint4 b[4], f[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      b[u] = ldg_stream(wb + i + u * stride);
+      f[u] = ldg_stream(wf + i + u * stride);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      float d[V::N];
+      V::delta(b[u], f[u], d);
+      float a1 = 0.f, a2 = 0.f;
+#pragma unroll
+      for (int k = 0; k < V::N; ++k) {
+        const float t = d[k] - shift;
+        a1 += t;
+        a2 = fmaf(t, t, a2);
+      }
+      s1 += (double)a1;
+      s2 += (double)a2;
+    }
+  }
+  for (; i < nvec; i += stride) {
+    float d[V::N];
+    V::delta(ldg_stream(wb + i), ldg_stream(wf + i), d);
+    float a1 = 0.f, a2 = 0.f;
+#pragma unroll
+    for (int k = 0; k < V::N; ++k) {
+      const float t = d[k] - shift;
+      a1 += t;
+      a2 = fmaf(t, t, a2);
+    }
+    s1 += (double)a1;
+    s2 += (double)a2;
+  }
+  s1 = warp_sum_d(s1);
+  s2 = warp_sum_d(s2);
+  __shared__ double sh[2][8];
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  if (l == 0) {
+    sh[0][w] = s1;
+    sh[1][w] = s2;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t1 = 0.0, t2 = 0.0;
+    for (int k = 0; k < (int)(blockDim.x >> 5); ++k) {
+      t1 += sh[0][k];
+      t2 += sh[1][k];
+    }
+    partials[2 * blockIdx.x] = t1;
+    partials[2 * blockIdx.x + 1] = t2;
+  }
+}
+
+template <bool BF16>
+__global__ void k_stats_final(const uint4* __restrict__ wb, const uint4* __restrict__ wf,
+                              const double* __restrict__ partials, int nparts, int64_t n,
+                              double k, ClipParams* __restrict__ out, double* __restrict__ stats_out) {
+  // one block of 256 threads: strided per-thread sums, then a fixed tree
+  __shared__ double sh1[256], sh2[256];
+  double t1 = 0.0, t2 = 0.0;
+  for (int p = threadIdx.x; p < nparts; p += blockDim.x) {
+    t1 += partials[2 * p];
+    t2 += partials[2 * p + 1];
+  }
+  sh1[threadIdx.x] = t1;
+  sh2[threadIdx.x] = t2;
+  __syncthreads();
+  for (int s = 128; s > 0; s >>= 1) {
+    if ((int)threadIdx.x < s) {
+      sh1[threadIdx.x] += sh1[threadIdx.x + s];
+      sh2[threadIdx.x] += sh2[threadIdx.x + s];
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    using V = Vec<BF16>;
+    float d0[V::N];
+    V::delta(wb[0], wf[0], d0);
+    const double shift = (double)d0[0];
+    const double S1 = sh1[0], S2 = sh2[0];
+    const double dn = (double)n;
+    const double mean = shift + S1 / dn;
+    double sd = 0.0;
+    if (n > 1) {
+      double var = (S2 - S1 * (S1 / dn)) / (dn - 1.0);
+      sd = var > 0.0 ? sqrt(var) : 0.0;
+    }
+    const double lo = mean - k * sd, hi = mean + k * sd;
+    ClipParams c;
+    c.mean = mean;
+    c.stddev = sd;
+    c.lo = lo;
+    c.hi = hi;
+    c.lo_up = __double2float_ru(lo);
+    c.hi_dn = __double2float_rd(hi);
+    float lv = __double2float_rn(lo), hv = __double2float_rn(hi);
+    // keep the sign of the fp64 bound if rounding flushed it to zero
+    if (lo < 0.0 && lv == 0.0f) lv = -1.401298464e-45f;
+    if (hi < 0.0 && hv == 0.0f) hv = -1.401298464e-45f;
+    if (lo >= 0.0 && lv == 0.0f) lv = 0.0f;
+    if (hi >= 0.0 && hv == 0.0f) hv = 0.0f;
+    c.lo_val = lv;
+    c.hi_val = hv;
+    *out = c;
+    if (stats_out) {
+      stats_out[0] = mean;
+      stats_out[1] = sd;
+      stats_out[2] = lo;
+      stats_out[3] = hi;
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------
+// main pass for GROUP / ROW / TENSOR
+// ------------------------------------------------------------------------------------
+// A task is (row, segment of seg_chunks chunks); a chunk is 32 lanes x 16 bytes.
+template <bool BF16, int SEGC>
+__global__ void __launch_bounds__(256) k_scale_signpack(
+    const uint8_t* __restrict__ wb, const uint8_t* __restrict__ wf, int64_t d_out, int64_t d_in,
+    int mode, int group, int seg_chunks, int nseg, const ClipParams* __restrict__ clipp,
+    uint32_t* __restrict__ signs, float* __restrict__ scales, double* __restrict__ partials) {
+  using V = Vec<BF16>;
+  constexpr int VEC = V::N;
+  constexpr int CHUNK = 32 * VEC;             // columns per chunk
+  constexpr int LPW = 32 / VEC;               // lanes per 32-bit sign word
+  constexpr int ESZ = BF16 ? 2 : 4;
+  const int lane = threadIdx.x & 31;
+  const int64_t task = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (task >= d_out * (int64_t)nseg) return;
+  const int64_t row = task / nseg;
+  const int seg = (int)(task % nseg);
+
+  ClipParams cp;
+  const bool do_clip = clipp != nullptr;
+  if (do_clip) cp = *clipp;
+
+  const uint8_t* rb = wb + row * d_in * ESZ;
+  const uint8_t* rf = wf + row * d_in * ESZ;
+  const int64_t words_per_row = d_in >> 5;
+  uint32_t* srow = signs + row * words_per_row;
+  const int64_t col_seg0 = (int64_t)seg * seg_chunks * CHUNK;
+
+  double acc_row = 0.0;   // ROW / TENSOR: this lane's share of the segment sum
+  double acc_grp = 0.0;   // GROUP with G > CHUNK: running group sum (all lanes equal)
+
+  for (int c0 = 0; c0 < seg_chunks; c0 += SEGC) {
+    uint4 b[SEGC], f[SEGC];
+    bool valid[SEGC];
+#pragma unroll
+    for (int u = 0; u < SEGC; ++u) {
+      const int64_t col = col_seg0 + (int64_t)(c0 + u) * CHUNK + lane * VEC;
+      valid[u] = (c0 + u < seg_chunks) && col < d_in;
+      if (valid[u]) {
+        b[u] = ldg_stream(rb + col * ESZ);
+        f[u] = ldg_stream(rf + col * ESZ);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < SEGC; ++u) {
+      const int64_t chunk_col0 = col_seg0 + (int64_t)(c0 + u) * CHUNK;
+      if (c0 + u >= seg_chunks || chunk_col0 >= d_in) break;  // warp-uniform
+      float d[VEC];
+      uint32_t m = 0;
+      float a = 0.f;
+      if (valid[u]) {
+        V::delta(b[u], f[u], d);
+#pragma unroll
+        for (int k = 0; k < VEC; ++k) {
+          float dc = do_clip ? clamp_delta(d[k], cp) : d[k];
+          m |= (dc < 0.f ? 0u : 1u) << k;
+          a += fabsf(dc);
+        }
+      }
+      // pack: LPW lanes x VEC bits -> one word, lane order = column order (LSB first)
+      uint32_t v = m << (VEC * (lane % LPW));
+#pragma unroll
+      for (int o = 1; o < LPW; o <<= 1) v |= __shfl_xor_sync(0xffffffffu, v, o);
+      if (valid[u] && (lane % LPW) == 0) srow[(chunk_col0 + lane * VEC) >> 5] = v;
+
+      if (mode == BD_SCALE_GROUP) {
+        if (group <= CHUNK) {
+          const int lpg = group / VEC;  // lanes per group (power of two, >= 4 / >= 8)
+          float s = a;
+          for (int o = 1; o < lpg; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+          if (valid[u] && (lane % lpg) == 0) {
+            const int64_t col = chunk_col0 + lane * VEC;
+            scales[row * (d_in / group) + col / group] = s / (float)group;
+          }
+        } else {
+          float s = warp_sum_f(a);
+          acc_grp += (double)s;
+          if (((chunk_col0 + CHUNK) % group) == 0 || chunk_col0 + CHUNK >= d_in) {
+            if (lane == 0) scales[row * (d_in / group) + chunk_col0 / group] = (float)(acc_grp / (double)group);
+            acc_grp = 0.0;
+          }
+        }
+      } else {
+        acc_row += (double)a;
+      }
+    }
+  }
+  if (mode != BD_SCALE_GROUP) {
+    acc_row = warp_sum_d(acc_row);
+    if (lane == 0) partials[row * nseg + seg] = acc_row;
+  }
+}
+
+// ------------------------------------------------------------------------------------
+// COL mode: per-column sums over row tiles
+// ------------------------------------------------------------------------------------
+template <bool BF16>
+__global__ void __launch_bounds__(256) k_col_scale_signpack(
+    const uint8_t* __restrict__ wb, const uint8_t* __restrict__ wf, int64_t d_out, int64_t d_in,
+    int tile_rows, int64_t nchunks, const ClipParams* __restrict__ clipp,
+    uint32_t* __restrict__ signs, double* __restrict__ colpart) {
+  using V = Vec<BF16>;
+  constexpr int VEC = V::N;
+  constexpr int CHUNK = 32 * VEC;
+  constexpr int LPW = 32 / VEC;
+  constexpr int ESZ = BF16 ? 2 : 4;
+  constexpr int UR = 4;  // rows in flight per warp
+  const int lane = threadIdx.x & 31;
+  const int64_t task = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t ntile = (d_out + tile_rows - 1) / tile_rows;
+  if (task >= ntile * nchunks) return;
+  const int64_t tile = task / nchunks;
+  const int64_t chunk = task % nchunks;
+  const int64_t col = chunk * CHUNK + lane * VEC;
+  const bool valid = col < d_in;
+  ClipParams cp;
+  const bool do_clip = clipp != nullptr;
+  if (do_clip) cp = *clipp;
+  double acc[VEC];
+#pragma unroll
+  for (int k = 0; k < VEC; ++k) acc[k] = 0.0;
+  const int64_t r0 = tile * tile_rows;
+  const int64_t r1 = min(d_out, r0 + tile_rows);
+  const int64_t words_per_row = d_in >> 5;
+  for (int64_t r = r0; r < r1; r += UR) {
+    uint4 b[UR], f[UR];
+#pragma unroll
+    for (int u = 0; u < UR; ++u) {
+      if (valid && r + u < r1) {
+        b[u] = ldg_stream(wb + ((r + u) * d_in + col) * ESZ);
+        f[u] = ldg_stream(wf + ((r + u) * d_in + col) * ESZ);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < UR; ++u) {
+      if (r + u >= r1) break;  // warp-uniform
+      uint32_t m = 0;
+      if (valid) {
+        float d[VEC];
+        V::delta(b[u], f[u], d);
+#pragma unroll
+        for (int k = 0; k < VEC; ++k) {
+          float dc = do_clip ? clamp_delta(d[k], cp) : d[k];
+          m |= (dc < 0.f ? 0u : 1u) << k;
+          acc[k] += (double)fabsf(dc);
+        }
+      }
+      uint32_t v = m << (VEC * (lane % LPW));
+#pragma unroll
+      for (int o = 1; o < LPW; o <<= 1) v |= __shfl_xor_sync(0xffffffffu, v, o);
+      if (valid && (lane % LPW) == 0) signs[(r + u) * words_per_row + (col >> 5)] = v;
+    }
+  }
+  if (valid) {
+#pragma unroll
+    for (int k = 0; k < VEC; ++k) colpart[tile * d_in + col + k] = acc[k];
+  }
+}
+
+// ------------------------------------------------------------------------------------
+// fixed-order reductions of the partial sums
+// ------------------------------------------------------------------------------------
+// ROW: scales[r] = sum_s partials[r][s] / d_in (one thread per row)
+__global__ void k_row_final(const double* __restrict__ partials, int nseg, int64_t d_out,
+                            int64_t d_in, float* __restrict__ scales) {
+  const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= d_out) return;
+  double s = 0.0;
+  for (int k = 0; k < nseg; ++k) s += partials[r * nseg + k];
+  scales[r] = (float)(s / (double)d_in);
+}
+
+// COL: scales[i] = sum_t colpart[t][i] / d_out (one thread per column)
+__global__ void k_col_final(const double* __restrict__ colpart, int64_t ntile, int64_t d_out,
+                            int64_t d_in, float* __restrict__ scales) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= d_in) return;
+  double s = 0.0;
+  for (int64_t t = 0; t < ntile; ++t) s += colpart[t * d_in + i];
+  scales[i] = (float)(s / (double)d_out);
+}
+
+// TENSOR: one block; strided per-thread sums then a fixed tree
+__global__ void k_tensor_final(const double* __restrict__ partials, int64_t n, double count,
+                               float* __restrict__ scales) {
+  __shared__ double sh[256];
+  double s = 0.0;
+  for (int64_t k = threadIdx.x; k < n; k += blockDim.x) s += partials[k];
+  sh[threadIdx.x] = s;
+  __syncthreads();
+  for (int st = 128; st > 0; st >>= 1) {
+    if ((int)threadIdx.x < st) sh[threadIdx.x] += sh[threadIdx.x + st];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) scales[0] = (float)(sh[0] / count);
+}
+
+// ------------------------------------------------------------------------------------
+// host side
+// ------------------------------------------------------------------------------------
+namespace {
+
+struct CompressPlan {
+  bool bf16;
+  int chunk;          // columns per warp chunk
+  int seg_chunks;     // chunks per task (GROUP / ROW / TENSOR)
+  int nseg;           // tasks per row
+  int stats_blocks;   // blocks of the stats pass
+  int col_tile;       // rows per tile (COL)
+  int64_t nchunks;    // chunks per row
+  int64_t ntile;      // row tiles (COL)
+  size_t off_clip, off_stats, off_part, total;
+};
+
+bd_status plan_compress(int32_t dtype, int64_t d_out, int64_t d_in, const bd_compress_cfg* cfg,
+                        CompressPlan* p) {
+  if (!cfg) return BD_ERR_NULL;
+  if (dtype != BD_F32 && dtype != BD_BF16) return BD_ERR_DTYPE;
+  if (d_out < 1 || d_in < 32 || (d_in % 32) != 0) return BD_ERR_SHAPE;
+  if (cfg->mode < BD_SCALE_GROUP || cfg->mode > BD_SCALE_TENSOR) return BD_ERR_CONFIG;
+  if (cfg->clip != 0 && cfg->clip != 1) return BD_ERR_CONFIG;
+  if (cfg->clip && !(cfg->clip_k >= 0.0f)) return BD_ERR_CONFIG;
+  const int64_t G = cfg->group_size;
+  if (cfg->mode == BD_SCALE_GROUP) {
+    if (G < 32 || !is_pow2(G) || (d_in % G) != 0) return BD_ERR_CONFIG;
+  }
+  p->bf16 = dtype == BD_BF16;
+  p->chunk = p->bf16 ? 256 : 128;
+  p->nchunks = (d_in + p->chunk - 1) / p->chunk;
+  const int sms = sm_count();
+  const int64_t target_tasks = (int64_t)sms * 64;  // warps in flight we want
+  int segc = 4;
+  while (segc > 1 && d_out * ((p->nchunks + segc - 1) / segc) < target_tasks) segc >>= 1;
+  if (cfg->mode == BD_SCALE_GROUP && G > p->chunk) {
+    const int need = (int)(G / p->chunk);
+    segc = ((segc + need - 1) / need) * need;
+  }
+  p->seg_chunks = segc;
+  p->nseg = (int)((p->nchunks + segc - 1) / segc);
+  p->stats_blocks = sms * 4;
+  // COL tiles: enough tasks for the GPU, tiles of 32..256 rows
+  int tile = 256;
+  while (tile > 32 && ((d_out + tile - 1) / tile) * p->nchunks < target_tasks) tile >>= 1;
+  p->col_tile = tile;
+  p->ntile = (d_out + tile - 1) / tile;
+  size_t off = kStatusBytes;
+  p->off_clip = off;
+  off = align_up(off + sizeof(ClipParams), 256);
+  p->off_stats = off;
+  off = align_up(off + (size_t)p->stats_blocks * 2 * sizeof(double), 256);
+  p->off_part = off;
+  size_t part = 0;
+  if (cfg->mode == BD_SCALE_ROW || cfg->mode == BD_SCALE_TENSOR)
+    part = (size_t)d_out * p->nseg * sizeof(double);
+  else if (cfg->mode == BD_SCALE_COL)
+    part = (size_t)p->ntile * d_in * sizeof(double);
+  off = align_up(off + part, 256);
+  p->total = off;
+  return BD_OK;
+}
+
+template <bool BF16>
+bd_status launch_compress(const CompressPlan& p, const void* w_base, const void* w_fine,
+                          int64_t d_out, int64_t d_in, const bd_compress_cfg* cfg,
+                          uint32_t* signs, float* scales, double* stats_out, uint8_t* ws,
+                          cudaStream_t s) {
+  ClipParams* clipp = nullptr;
+  const int64_t nvec = d_out * d_in * (BF16 ? 2 : 4) / 16;
+  if (cfg->clip) {
+    clipp = reinterpret_cast<ClipParams*>(ws + p.off_clip);
+    double* parts = reinterpret_cast<double*>(ws + p.off_stats);
+    launch_begin(K_DELTA_STATS, s);
+    k_delta_stats<BF16><<<p.stats_blocks, 256, 0, s>>>((const uint4*)w_base, (const uint4*)w_fine,
+                                                       nvec, parts);
+    launch_end(K_DELTA_STATS, s);
+    BD_LAUNCH_CHECK();
+    launch_begin(K_STATS_FINAL, s);
+    k_stats_final<BF16><<<1, 256, 0, s>>>((const uint4*)w_base, (const uint4*)w_fine, parts,
+                                          p.stats_blocks, d_out * d_in, (double)cfg->clip_k,
+                                          clipp, stats_out);
+    launch_end(K_STATS_FINAL, s);
+    BD_LAUNCH_CHECK();
+  }
+  double* part = reinterpret_cast<double*>(ws + p.off_part);
+  if (cfg->mode == BD_SCALE_COL) {
+    const int64_t tasks = p.ntile * p.nchunks;
+    const int64_t blocks = (tasks + 7) / 8;
+    launch_begin(K_COL_SCALE_SIGNPACK, s);
+    k_col_scale_signpack<BF16><<<(unsigned)blocks, 256, 0, s>>>(
+        (const uint8_t*)w_base, (const uint8_t*)w_fine, d_out, d_in, p.col_tile, p.nchunks,
+        clipp, signs, part);
+    launch_end(K_COL_SCALE_SIGNPACK, s);
+    BD_LAUNCH_CHECK();
+    launch_begin(K_SCALE_FINAL, s);
+    k_col_final<<<(unsigned)((d_in + 255) / 256), 256, 0, s>>>(part, p.ntile, d_out, d_in, scales);
+    launch_end(K_SCALE_FINAL, s);
+    BD_LAUNCH_CHECK();
+    return BD_OK;
+  }
+  const int64_t tasks = d_out * (int64_t)p.nseg;
+  const int64_t blocks = (tasks + 7) / 8;
+  const int G = cfg->mode == BD_SCALE_GROUP ? cfg->group_size : 0;
+  launch_begin(K_SCALE_SIGNPACK, s);
+  if (p.seg_chunks >= 4) {
+    k_scale_signpack<BF16, 4><<<(unsigned)blocks, 256, 0, s>>>(
+        (const uint8_t*)w_base, (const uint8_t*)w_fine, d_out, d_in, cfg->mode, G, p.seg_chunks,
+        p.nseg, clipp, signs, scales, part);
+  } else {
+    k_scale_signpack<BF16, 2><<<(unsigned)blocks, 256, 0, s>>>(
+        (const uint8_t*)w_base, (const uint8_t*)w_fine, d_out, d_in, cfg->mode, G, p.seg_chunks,
+        p.nseg, clipp, signs, scales, part);
+  }
+  launch_end(K_SCALE_SIGNPACK, s);
+  BD_LAUNCH_CHECK();
+  if (cfg->mode == BD_SCALE_ROW) {
+    launch_begin(K_SCALE_FINAL, s);
+    k_row_final<<<(unsigned)((d_out + 255) / 256), 256, 0, s>>>(part, p.nseg, d_out, d_in, scales);
+    launch_end(K_SCALE_FINAL, s);
+    BD_LAUNCH_CHECK();
+  } else if (cfg->mode == BD_SCALE_TENSOR) {
+    launch_begin(K_SCALE_FINAL, s);
+    k_tensor_final<<<1, 256, 0, s>>>(part, d_out * (int64_t)p.nseg, (double)d_out * (double)d_in,
+                                     scales);
+    launch_end(K_SCALE_FINAL, s);
+    BD_LAUNCH_CHECK();
+  }
+  return BD_OK;
+}
+
+}  // namespace
+
+bd_status compress_impl(const void* w_base, const void* w_fine, int32_t dtype, int64_t d_out,
+                        int64_t d_in, const bd_compress_cfg* cfg, uint32_t* signs_out,
+                        float* scales_out, double* stats_out, void* workspace, size_t ws_bytes,
+                        cudaStream_t s) {
+  CompressPlan p;
+  bd_status st = plan_compress(dtype, d_out, d_in, cfg, &p);
+  if (st != BD_OK) return st;
+  if (!w_base || !w_fine || !signs_out || !scales_out) return BD_ERR_NULL;
+  if (!aligned16(w_base) || !aligned16(w_fine) || !aligned16(signs_out) || !aligned16(scales_out))
+    return BD_ERR_ALIGN;
+  if (!workspace || ws_bytes < p.total) return BD_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return BD_ERR_ALIGN;
+  if (stats_out && (reinterpret_cast<uintptr_t>(stats_out) & 7u)) return BD_ERR_ALIGN;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (p.bf16)
+    return launch_compress<true>(p, w_base, w_fine, d_out, d_in, cfg, signs_out, scales_out,
+                                 stats_out, ws, s);
+  return launch_compress<false>(p, w_base, w_fine, d_out, d_in, cfg, signs_out, scales_out,
+                                stats_out, ws, s);
+}
+
+size_t compress_workspace_size(int64_t d_out, int64_t d_in, const bd_compress_cfg* cfg) {
+  CompressPlan p;
+  if (plan_compress(BD_BF16, d_out, d_in, cfg, &p) != BD_OK) return 0;
+  CompressPlan q;
+  plan_compress(BD_F32, d_out, d_in, cfg, &q);
+  return p.total > q.total ? p.total : q.total;
+}
+
+}  // namespace bd
+
+extern "C" bd_status bd_compress(const void* w_base, const void* w_fine, int32_t dtype,
+                                 int64_t d_out, int64_t d_in, const bd_compress_cfg* cfg,
+                                 uint32_t* signs_out, float* scales_out, double* stats_out,
+                                 void* workspace, size_t ws_bytes, void* stream) {
+  return bd::compress_impl(w_base, w_fine, dtype, d_out, d_in, cfg, signs_out, scales_out,
+                           stats_out, workspace, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" size_t bd_compress_workspace_size(int64_t d_out, int64_t d_in, const bd_compress_cfg* cfg) {
+  return bd::compress_workspace_size(d_out, d_in, cfg);
+}

@@ -1,0 +1,96 @@
+// Internal helpers shared by the library's translation units (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "../../include/bitdelta.h"
+
+namespace bd {
+
+// ------------------------------------------------------------------------------------
+// kernel kinds (for launch accounting and per-kernel timing)
+// ------------------------------------------------------------------------------------
+enum KernelKind : int32_t {
+  K_DELTA_STATS = 0,     // fused delta + whole-matrix shifted sums for the clip
+  K_STATS_FINAL,         // fixed-order merge of the partial sums -> mean, std, lo, hi
+  K_SCALE_SIGNPACK,      // clip + abs-mean (group / row / tensor partials) + sign pack
+  K_COL_SCALE_SIGNPACK,  // clip + per-column partial abs sums + sign pack
+  K_SCALE_FINAL,         // fixed-order row / column / tensor scale reduction
+  K_RECONSTRUCT,         // signs * scales (+ W_base)
+  K_TENANT_BUCKET,       // counting sort of tenant ids -> segments
+  K_BASE_GEMV,           // CUDA-core base product for small batches / fp32
+  K_BASE_TC,             // tcgen05 base product (bf16, fp32 accumulation in TMEM)
+  K_DELTA_LUT,           // per-tenant sign-LUT delta product + combine
+  K_SELECT_FIXUP,        // compress: re-read of groups touched by the clip
+  K_KIND_COUNT
+};
+
+const char* kernel_name(int32_t kind);
+
+// Called around every kernel launch of the library (bd_abi.cu).
+void launch_begin(int32_t kind, cudaStream_t s);
+void launch_end(int32_t kind, cudaStream_t s);
+
+int sm_count();  // multiprocessors of the current device (cached per device)
+
+// Device status word, the first 16 bytes of every workspace.
+struct DevStatus {
+  uint32_t flags;
+  uint32_t pad[3];
+};
+constexpr size_t kStatusBytes = 256;  // keeps what follows 256-byte aligned
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool is_pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
+
+#define BD_CUDA_TRY(expr)                           \
+  do {                                              \
+    cudaError_t _e = (expr);                        \
+    if (_e != cudaSuccess) {                        \
+      (void)cudaGetLastError();                     \
+      return BD_ERR_CUDA;                           \
+    }                                               \
+  } while (0)
+
+#define BD_LAUNCH_CHECK()                           \
+  do {                                              \
+    cudaError_t _e = cudaGetLastError();            \
+    if (_e != cudaSuccess) return BD_ERR_CUDA;      \
+  } while (0)
+
+// ------------------------------------------------------------------------------------
+// device helpers
+// ------------------------------------------------------------------------------------
+__device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+// round-to-nearest-even float -> bf16 bits (finite inputs)
+__device__ __forceinline__ uint32_t f2bf_bits(float f) {
+  return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+
+__device__ __forceinline__ float warp_sum_f(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ uint4 ldg_stream(const void* p) {
+  // 16-byte global load that is not kept in L1 (each byte is read once)
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+}  // namespace bd

@@ -1,0 +1,230 @@
+"""GPU parity of bd_apply_multi against the fp64 oracle, through the C ABI.
+
+Tolerance (apply outputs, bf16 inputs, fp32 accumulation):
+    |y - y_ref| <= 1e-2 * (|y_ref| + rms(y_ref))
+checked on the full output, plus cases where W_base = 0 so that the same bound applies
+to the delta product alone, and fp32-output cases held to a much tighter bound."""
+
+import numpy as np
+import pytest
+
+import oracle as O
+from helpers import APPLY_TOL, assert_apply_close, dev, host
+from workloads import (LLAMA3_8B_PROJECTIONS, activations, bf16_bits, random_tenant, tiny_config,
+                       weight_pair, zipf_ids)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def bd():
+    from tenant_serving_b200 import build
+    build.build()
+    import tenant_serving_b200 as m
+    return m
+
+
+def _table(bd, tenants):
+    return bd.TenantTable([(dev(t["signs"]), dev(t["scales"]), t["mode"], t["group_size"])
+                           for t in tenants], "cuda")
+
+
+def _run(bd, wb, tenants, ids, x, y_dtype="bf16", w_dtype="bf16"):
+    import torch
+    table = _table(bd, tenants)
+    y, ws = bd.bd_apply_multi(dev(wb, w_dtype), table, dev(ids), dev(x, w_dtype),
+                              y_dtype=torch.bfloat16 if y_dtype == "bf16" else torch.float32)
+    rc, flags = bd.bd_get_status(ws)
+    yh = host(y)
+    yv = O.decode(yh, "bf16") if y_dtype == "bf16" else yh.astype(np.float64)
+    return yv, rc, flags
+
+
+def _problem(seed, d_out, d_in, B, T, modes=(0,), G=128, zero_base=False, ids=None):
+    rng = np.random.default_rng(seed)
+    wb = bf16_bits(rng.normal(0, 0.02, size=(d_out, d_in)))
+    if zero_base:
+        wb[:] = 0
+    tenants = [random_tenant(rng, d_out, d_in, modes[u % len(modes)], G) for u in range(T)]
+    x = activations(rng, B, d_in)
+    if ids is None:
+        ids = rng.integers(0, T, size=B).astype(np.int32)
+    return wb, tenants, np.asarray(ids, dtype=np.int32), x
+
+
+# -----------------------------------------------------------------------------------
+def test_tiny_config_end_to_end(bd):
+    """Compress both tenants on the GPU and in the oracle, then apply the 4 fp32 tokens
+    (ids [0, 1, 0, 1]); each side uses only its own compress results."""
+    import torch
+    cfg = tiny_config()
+    wb = cfg["w_base"]
+    ref_t, gpu_t = [], []
+    for wf in cfg["w_fine"]:
+        r = O.compress(wb, wf, "f32", O.MODE_GROUP, 128, True, 3.0)
+        ref_t.append({"signs": r["signs"], "scales": r["scales"].astype(np.float32),
+                      "scale_dtype": "f32", "mode": 0, "group_size": 128})
+        c = bd.compress_cfg(mode=0, group_size=128, clip=True, clip_k=3.0)
+        s, sc, _ = bd.bd_compress(dev(wb), dev(wf), c)
+        gpu_t.append((s, sc, 0, 128))
+    y_ref = O.apply_multi(wb, "f32", ref_t, cfg["tenant_ids"], cfg["x"], "f32")
+    table = bd.TenantTable(gpu_t, "cuda")
+    y, ws = bd.bd_apply_multi(dev(wb), table, dev(cfg["tenant_ids"]), dev(cfg["x"]),
+                              y_dtype=torch.float32)
+    assert bd.bd_get_status(ws)[0] == bd.BD_OK
+    assert_apply_close(host(y), y_ref)
+    assert_apply_close(host(y), y_ref, tol=1e-5, what="y (fp32 path, tight)")
+
+
+@pytest.mark.parametrize("B", [1, 4, 16, 63, 200, 300])
+@pytest.mark.parametrize("mode", [0, 1, 2, 3])
+def test_random_batches(bd, B, mode):
+    d_out, d_in = 384 + 8, 1024
+    wb, tenants, ids, x = _problem(B * 10 + mode, d_out, d_in, B, 5, (mode,))
+    ids[0] = -1  # base only
+    y, rc, _ = _run(bd, wb, tenants, ids, x)
+    assert rc == bd.BD_OK
+    y_ref = O.apply_multi(wb, "bf16", tenants, ids, x, "bf16")
+    assert_apply_close(y, y_ref)
+
+
+@pytest.mark.parametrize("mode", [0, 1, 2, 3])
+@pytest.mark.parametrize("d_out,d_in", [(1100, 544), (64, 4096), (2050, 256), (130, 96)])
+def test_delta_only_tight(bd, mode, d_out, d_in):
+    """W_base = 0: the bound now constrains the delta product by itself; with fp32
+    outputs it must also hold at 1e-5."""
+    G = 32 if d_in % 128 else 128
+    wb, tenants, ids, x = _problem(d_out + d_in + mode, d_out, d_in, 9, 3, (mode,), G=G,
+                                   zero_base=True)
+    y_ref = O.apply_multi(wb, "bf16", tenants, ids, x, "bf16")
+    y, rc, _ = _run(bd, wb, tenants, ids, x, y_dtype="f32")
+    assert rc == bd.BD_OK
+    assert_apply_close(y, y_ref)
+    assert_apply_close(y, y_ref, tol=1e-5, what="delta only (fp32 out)")
+
+
+def test_mixed_modes_and_group_sizes(bd):
+    rng = np.random.default_rng(12)
+    d_out, d_in = 520, 2048
+    wb = bf16_bits(rng.normal(0, 0.02, size=(d_out, d_in)))
+    tenants = [random_tenant(rng, d_out, d_in, 0, g) for g in (32, 64, 128, 256, 512, 2048)]
+    tenants += [random_tenant(rng, d_out, d_in, m) for m in (1, 2, 3)]
+    B = 40
+    x = activations(rng, B, d_in)
+    ids = rng.integers(-1, len(tenants), size=B).astype(np.int32)
+    y, rc, _ = _run(bd, wb, tenants, ids, x, y_dtype="f32")
+    assert rc == bd.BD_OK
+    assert_apply_close(y, O.apply_multi(wb, "bf16", tenants, ids, x, "bf16"), tol=1e-5)
+
+
+def test_single_tenant_equals_merged_weight(bd):
+    """All tokens of one tenant: y = (W_base + Delta_hat) X, a plain matmul."""
+    wb, tenants, _, x = _problem(3, 640, 1024, 48, 1, (0,))
+    ids = np.zeros(48, dtype=np.int32)
+    y, rc, _ = _run(bd, wb, tenants, ids, x, y_dtype="f32")
+    t = tenants[0]
+    W = O.reconstruct(t["signs"], O.decode(t["scales"], "f16"), 0, 128, 640, 1024,
+                      w_base=O.decode(wb, "bf16"))
+    assert_apply_close(y, O.decode(x, "bf16") @ W.T, tol=1e-5)
+
+
+def test_zero_input_and_permutation(bd):
+    wb, tenants, ids, x = _problem(5, 256, 512, 24, 4, (0, 1, 2))
+    y0, _, _ = _run(bd, wb, tenants, ids, np.zeros_like(x), y_dtype="f32")
+    assert np.all(y0 == 0)
+    y, _, _ = _run(bd, wb, tenants, ids, x, y_dtype="f32")
+    p = np.random.default_rng(1).permutation(len(ids))
+    yp, _, _ = _run(bd, wb, tenants, ids[p], x[p], y_dtype="f32")
+    np.testing.assert_array_equal(yp, y[p])  # per-token results do not depend on order
+
+
+def test_out_of_range_ids_flag_and_base_only(bd):
+    wb, tenants, ids, x = _problem(6, 256, 512, 10, 3, (0,))
+    ids[2] = 3
+    ids[5] = -7
+    y, rc, flags = _run(bd, wb, tenants, ids, x, y_dtype="f32")
+    assert rc == bd.BD_ERR_TENANT_RANGE and flags & bd.BD_DEV_TENANT_RANGE
+    fixed = ids.copy()
+    fixed[2] = -1
+    fixed[5] = -1
+    assert_apply_close(y, O.apply_multi(wb, "bf16", tenants, fixed, x, "bf16"), tol=1e-5)
+    # the next good call clears the status word
+    _, rc2, flags2 = _run(bd, wb, tenants, fixed, x, y_dtype="f32")
+    assert rc2 == bd.BD_OK and flags2 == 0
+
+
+def test_bad_tenant_record_flag(bd):
+    import torch
+    wb, tenants, ids, x = _problem(8, 256, 512, 6, 2, (0,))
+    ids[:] = [0, 1, 0, 1, 0, 1]
+    t0 = tenants[0]
+    good = (dev(t0["signs"]), dev(t0["scales"]), 0, 128)
+    bad = (dev(tenants[1]["signs"]), dev(tenants[1]["scales"]), 0, 96)  # 96 is not a power of 2
+    table = bd.TenantTable([good, bad], "cuda")
+    y, ws = bd.bd_apply_multi(dev(wb), table, dev(ids), dev(x), y_dtype=torch.float32)
+    rc, flags = bd.bd_get_status(ws)
+    assert rc == bd.BD_ERR_TENANT_RECORD and flags & bd.BD_DEV_TENANT_RECORD
+    fixed = np.where(ids == 1, -1, ids).astype(np.int32)
+    assert_apply_close(host(y), O.apply_multi(wb, "bf16", tenants, fixed, x, "bf16"), tol=1e-5)
+
+
+def test_tenant_without_tokens_and_many_tenants(bd):
+    wb, tenants, _, x = _problem(10, 300, 768, 33, 40, (0, 1, 2, 3))
+    ids = np.array([39] * 20 + list(range(13)), dtype=np.int32)  # tenants 13..38 idle
+    y, rc, _ = _run(bd, wb, tenants, ids, x)
+    assert rc == bd.BD_OK
+    assert_apply_close(y, O.apply_multi(wb, "bf16", tenants, ids, x, "bf16"))
+
+
+def _sampled_rows_check(bd, d_out, d_in, tenants, ids, x, wb, rows, y):
+    sub = []
+    for t in tenants:
+        s = t["scales"]
+        if t["mode"] == 0:
+            s = s[rows]
+        elif t["mode"] == 1:
+            s = s[rows]
+        sub.append(dict(t, signs=t["signs"][rows], scales=s))
+    y_ref = O.apply_multi(wb[rows], "bf16", sub, ids, x, "bf16")
+    assert_apply_close(y[:, rows], y_ref)
+
+
+def test_decode_config_up_proj(bd):
+    """Decode GEMV at full size: up_proj 14336 x 4096 bf16 base, 64 resident tenants with
+    group-128 fp16 scales, 64 tokens, one per tenant (a seeded permutation). Checked on
+    256 sampled output rows plus full-tensor properties."""
+    rng = np.random.default_rng(2000)
+    d_out, d_in, T = 14336, 4096, 64
+    wb = bf16_bits(rng.normal(0, 0.02, size=(d_out, d_in)))
+    tenants = [random_tenant(rng, d_out, d_in, 0, 128) for _ in range(T)]
+    ids = rng.permutation(T).astype(np.int32)
+    x = activations(rng, T, d_in)
+    y, rc, _ = _run(bd, wb, tenants, ids, x)
+    assert rc == bd.BD_OK
+    rows = np.sort(rng.choice(d_out, 256, replace=False))
+    _sampled_rows_check(bd, d_out, d_in, tenants, ids, x, wb, rows, y)
+    assert np.isfinite(y).all()
+
+
+def test_mixed_config_layer(bd):
+    """One Llama-3-8B-shaped layer (7 projections), 32 tenants with per-axis fp16 scales
+    (row or column per (tenant, projection) by seed), 256 tokens with Zipf(1.1) ids.
+    Sampled rows per projection."""
+    rng = np.random.default_rng(3000)
+    B, T = 256, 32
+    ids = zipf_ids(rng, B, T, 1.1)
+    for name, d_out, d_in in LLAMA3_8B_PROJECTIONS:
+        wb = bf16_bits(rng.normal(0, 0.02, size=(d_out, d_in)))
+        tenants = [random_tenant(rng, d_out, d_in, int(rng.integers(1, 3))) for _ in range(T)]
+        x = activations(rng, B, d_in)
+        y, rc, _ = _run(bd, wb, tenants, ids, x)
+        assert rc == bd.BD_OK, name
+        rows = np.sort(rng.choice(d_out, 64, replace=False))
+        _sampled_rows_check(bd, d_out, d_in, tenants, ids, x, wb, rows, y)
+
+
+def test_launches_are_counted(bd):
+    n0 = bd.bd_launch_count()
+    wb, tenants, ids, x = _problem(1, 128, 256, 4, 2, (0,))
+    _run(bd, wb, tenants, ids, x)
+    assert bd.bd_launch_count() - n0 == 3  # bucket, base product, delta
