@@ -7,8 +7,8 @@
 //   sign bit = !(delta_c < 0), packed LSB-first along d_in into uint32 words.
 //
 // Kernels (all HBM-bound streams; 16-byte coalesced loads of both inputs):
-//   k_delta_stats      pass 1 when clipping: shifted fp32 sums per 16-byte vector,
-//                      accumulated in fp64 per thread, one (S1, S2) pair per block.
+//   k_delta_stats      pass 1 when clipping: sums of the shifted delta and of its square,
+//                      in fp64 per element, one (S1, S2) pair per block.
 //   k_stats_final      one block merges the block pairs in a fixed order -> mean, std,
 //                      lo, hi and the fp32 thresholds the main pass compares with.
 //   k_scale_signpack   main pass for GROUP / ROW / TENSOR: a warp streams a segment of
@@ -50,6 +50,16 @@ struct Vec<true> {  // 8 bf16 per 16 bytes
       d[2 * k + 1] = bf16hi(ff[k]) - bf16hi(bb[k]);
     }
   }
+  // exact differences in fp64
+  __device__ __forceinline__ static void delta64(const uint4& b, const uint4& f, double* d) {
+    const uint32_t bb[4] = {b.x, b.y, b.z, b.w};
+    const uint32_t ff[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      d[2 * k] = (double)bf16lo(ff[k]) - (double)bf16lo(bb[k]);
+      d[2 * k + 1] = (double)bf16hi(ff[k]) - (double)bf16hi(bb[k]);
+    }
+  }
 };
 template <>
 struct Vec<false> {  // 4 fp32 per 16 bytes
@@ -59,6 +69,12 @@ struct Vec<false> {  // 4 fp32 per 16 bytes
     d[1] = __uint_as_float(f.y) - __uint_as_float(b.y);
     d[2] = __uint_as_float(f.z) - __uint_as_float(b.z);
     d[3] = __uint_as_float(f.w) - __uint_as_float(b.w);
+  }
+  __device__ __forceinline__ static void delta64(const uint4& b, const uint4& f, double* d) {
+    d[0] = (double)__uint_as_float(f.x) - (double)__uint_as_float(b.x);
+    d[1] = (double)__uint_as_float(f.y) - (double)__uint_as_float(b.y);
+    d[2] = (double)__uint_as_float(f.z) - (double)__uint_as_float(b.z);
+    d[3] = (double)__uint_as_float(f.w) - (double)__uint_as_float(b.w);
   }
 };
 
@@ -76,11 +92,12 @@ __global__ void __launch_bounds__(256) k_delta_stats(const uint4* __restrict__ w
                                                      const uint4* __restrict__ wf,
                                                      int64_t nvec, double* __restrict__ partials) {
   using V = Vec<BF16>;
-  // shift: delta of element 0 (every thread computes the same value)
-  float shift;
+  // shift: delta of element 0 (every thread computes the same value); sums of the
+  // shifted deltas are accumulated in fp64 per element
+  double shift;
   {
-    float d0[V::N];
-    V::delta(wb[0], wf[0], d0);
+    double d0[V::N];
+    V::delta64(wb[0], wf[0], d0);
     shift = d0[0];
   }
   double s1 = 0.0, s2 = 0.0;
@@ -95,31 +112,25 @@ __global__ void __launch_bounds__(256) k_delta_stats(const uint4* __restrict__ w
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      float d[V::N];
-      V::delta(b[u], f[u], d);
-      float a1 = 0.f, a2 = 0.f;
+      double d[V::N];
+      V::delta64(b[u], f[u], d);  // exact difference of the stored values
 #pragma unroll
       for (int k = 0; k < V::N; ++k) {
-        const float t = d[k] - shift;
-        a1 += t;
-        a2 = fmaf(t, t, a2);
+        const double t = d[k] - shift;
+        s1 += t;
+        s2 = fma(t, t, s2);
       }
-      s1 += (double)a1;
-      s2 += (double)a2;
     }
   }
   for (; i < nvec; i += stride) {
-    float d[V::N];
-    V::delta(ldg_stream(wb + i), ldg_stream(wf + i), d);
-    float a1 = 0.f, a2 = 0.f;
+    double d[V::N];
+    V::delta64(ldg_stream(wb + i), ldg_stream(wf + i), d);
 #pragma unroll
     for (int k = 0; k < V::N; ++k) {
-      const float t = d[k] - shift;
-      a1 += t;
-      a2 = fmaf(t, t, a2);
+      const double t = d[k] - shift;
+      s1 += t;
+      s2 = fma(t, t, s2);
     }
-    s1 += (double)a1;
-    s2 += (double)a2;
   }
   s1 = warp_sum_d(s1);
   s2 = warp_sum_d(s2);
@@ -164,9 +175,9 @@ __global__ void k_stats_final(const uint4* __restrict__ wb, const uint4* __restr
   }
   if (threadIdx.x == 0) {
     using V = Vec<BF16>;
-    float d0[V::N];
-    V::delta(wb[0], wf[0], d0);
-    const double shift = (double)d0[0];
+    double d0[V::N];
+    V::delta64(wb[0], wf[0], d0);
+    const double shift = d0[0];
     const double S1 = sh1[0], S2 = sh2[0];
     const double dn = (double)n;
     const double mean = shift + S1 / dn;
