@@ -116,6 +116,31 @@ bd_status bd_compress(const void* w_base, const void* w_fine, int32_t dtype, int
                       float* scales_out, double* stats_out, void* workspace, size_t ws_bytes,
                       void* stream);
 
+/* bd_compress_noalloc — the same computation, arguments and results as bd_compress,
+ * but with no workspace argument and no device allocation anywhere on its path.
+ * There is no counterpart on the method's source pages; this entry point exists for
+ * callers that cannot allocate device memory themselves: code embedded in a host
+ * runtime that owns all device memory and forbids raw cudaMalloc, or a latency-critical
+ * loop where an allocation (which may synchronise the device) is not acceptable.
+ * Its scratch is one fixed array of BD_NOALLOC_SCRATCH_BYTES in the library's device
+ * image; every GPU that loads the library holds it until the process exits.
+ *   - Shapes and configs whose scratch need (bd_compress_workspace_size) exceeds
+ *     BD_NOALLOC_SCRATCH_BYTES are rejected with BD_ERR_WORKSPACE before any launch.
+ *     GROUP mode needs about 10 KB at any size; ROW / TENSOR need 8 bytes per row per
+ *     column segment (every Llama-3-8B projection fits); COL needs 8 bytes per column
+ *     per tile of rows, so large COL problems do not fit.
+ *   - The first call on each device looks up the array's device address (with that
+ *     device current) and caches it; make that first call before any stream capture.
+ *   - Every call shares the one array and it keeps the last call's contents; nothing in
+ *     it has to start at zero. Calls whose execution overlaps on the GPU (other streams,
+ *     other host threads) race on it: serialise them.
+ * The caller still passes inputs and outputs, as for bd_compress. */
+#define BD_NOALLOC_SCRATCH_BYTES ((size_t)1 << 20)
+bd_status bd_compress_noalloc(const void* w_base, const void* w_fine, int32_t dtype,
+                              int64_t d_out, int64_t d_in, const bd_compress_cfg* cfg,
+                              uint32_t* signs_out, float* scales_out, double* stats_out,
+                              void* stream);
+
 /* ---------------------------------------------------------------------------------- */
 /* reconstruct                                                                         */
 /* ---------------------------------------------------------------------------------- */

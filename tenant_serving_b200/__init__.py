@@ -13,7 +13,7 @@ from ._lib import (  # noqa: F401
     BD_DEV_TENANT_RANGE, BD_DEV_TIMEOUT, BD_DEV_TENANT_RECORD,
     EXPORTS, LIB_PATH, BitDeltaError, TenantTable, bd_compress_cfg, bd_tenant,
     lib, check, status_string, compress_cfg, scales_shape,
-    bd_compress, bd_compress_workspace_size, bd_reconstruct, bd_apply_multi,
+    bd_compress, bd_compress_noalloc, bd_compress_workspace_size, bd_reconstruct, bd_apply_multi,
     bd_apply_workspace_size, bd_get_status, bd_launch_count, bd_profile_enable,
     bd_profile_collect,
 )

@@ -33,7 +33,8 @@ BD_SCALE_GROUP, BD_SCALE_ROW, BD_SCALE_COL, BD_SCALE_TENSOR = 0, 1, 2, 3
 BD_DEV_TENANT_RANGE, BD_DEV_TIMEOUT, BD_DEV_TENANT_RECORD = 0x1, 0x2, 0x4
 
 EXPORTS = (
-    "bd_compress", "bd_compress_workspace_size", "bd_reconstruct", "bd_apply_multi",
+    "bd_compress", "bd_compress_noalloc", "bd_compress_workspace_size", "bd_reconstruct",
+    "bd_apply_multi",
     "bd_apply_workspace_size", "bd_get_status", "bd_status_string", "bd_launch_count",
     "bd_profile_enable", "bd_profile_collect", "bd_kernel_name",
 )
@@ -69,6 +70,10 @@ def lib():
                               POINTER(bd_compress_cfg), c_void_p, c_void_p, c_void_p, c_void_p,
                               c_size_t, c_void_p]
     L.bd_compress.restype = c_int32
+    L.bd_compress_noalloc.argtypes = [c_void_p, c_void_p, c_int32, c_int64, c_int64,
+                                      POINTER(bd_compress_cfg), c_void_p, c_void_p, c_void_p,
+                                      c_void_p]
+    L.bd_compress_noalloc.restype = c_int32
     L.bd_compress_workspace_size.argtypes = [c_int64, c_int64, POINTER(bd_compress_cfg)]
     L.bd_compress_workspace_size.restype = c_size_t
     L.bd_reconstruct.argtypes = [c_void_p, c_void_p, c_int32, c_int32, c_int32, c_int64, c_int64,
@@ -181,6 +186,28 @@ def bd_compress(w_base, w_fine, cfg: bd_compress_cfg, signs=None, scales=None, s
                            ctypes.byref(cfg), _ptr(signs), _ptr(scales), _ptr(stats),
                            _ptr(workspace), workspace.numel(), _stream(stream))
     check(rc, "bd_compress")
+    return signs, scales, stats
+
+
+def bd_compress_noalloc(w_base, w_fine, cfg: bd_compress_cfg, signs=None, scales=None,
+                        stats=None, stream=None):
+    """Wrap ``bd_compress_noalloc``: the library allocates nothing and uses its fixed
+    device scratch array (outputs missing here are still allocated by torch)."""
+    torch = _torch()
+    _require_cuda(w_base, w_fine)
+    d_out, d_in = w_base.shape
+    dev = w_base.device
+    if signs is None:
+        signs = torch.empty((d_out, d_in // 32), dtype=torch.int32, device=dev)
+    if scales is None:
+        scales = torch.empty(scales_shape(cfg.mode, d_out, d_in, cfg.group_size),
+                             dtype=torch.float32, device=dev)
+    if stats is None and cfg.clip:
+        stats = torch.zeros(4, dtype=torch.float64, device=dev)
+    rc = lib().bd_compress_noalloc(_ptr(w_base), _ptr(w_fine), dtype_code(w_base), d_out, d_in,
+                                   ctypes.byref(cfg), _ptr(signs), _ptr(scales), _ptr(stats),
+                                   _stream(stream))
+    check(rc, "bd_compress_noalloc")
     return signs, scales, stats
 
 

@@ -587,3 +587,56 @@ extern "C" bd_status bd_compress(const void* w_base, const void* w_fine, int32_t
 extern "C" size_t bd_compress_workspace_size(int64_t d_out, int64_t d_in, const bd_compress_cfg* cfg) {
   return bd::compress_workspace_size(d_out, d_in, cfg);
 }
+
+// ------------------------------------------------------------------------------------
+// bd_compress_noalloc: bd_compress for callers that cannot allocate device memory.
+// Its scratch is a fixed array in this library's device image instead of a caller
+// workspace. Every GPU that loads the library holds the array until the process exits.
+// ------------------------------------------------------------------------------------
+#include <mutex>
+
+namespace bd {
+
+constexpr size_t kNoAllocScratchBytes = (size_t)1 << 20;  // BD_NOALLOC_SCRATCH_BYTES
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch on the current device. In host code the array's
+// name is only a host-side stand-in, so the address is looked up once per device (with
+// that device current) and cached.
+static bd_status noalloc_scratch(void** out) {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    (void)cudaGetLastError();
+    return BD_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      (void)cudaGetLastError();
+      return BD_ERR_CUDA;
+    }
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return BD_OK;
+}
+
+}  // namespace bd
+
+extern "C" bd_status bd_compress_noalloc(const void* w_base, const void* w_fine, int32_t dtype,
+                                         int64_t d_out, int64_t d_in, const bd_compress_cfg* cfg,
+                                         uint32_t* signs_out, float* scales_out,
+                                         double* stats_out, void* stream) {
+  void* scratch = nullptr;
+  bd_status st = bd::noalloc_scratch(&scratch);
+  if (st != BD_OK) return st;
+  // bd_compress checks the arguments first and answers BD_ERR_WORKSPACE when this shape
+  // and config need more scratch than the fixed array holds.
+  return bd::compress_impl(w_base, w_fine, dtype, d_out, d_in, cfg, signs_out, scales_out,
+                           stats_out, scratch, bd::kNoAllocScratchBytes,
+                           static_cast<cudaStream_t>(stream));
+}
