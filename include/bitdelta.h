@@ -55,7 +55,8 @@ typedef enum {
   BD_ERR_TENANT_RANGE = 7,  /* device status: a tenant id outside [-1, n_tenants)      */
   BD_ERR_TIMEOUT = 8,       /* device status: a bounded wait gave up                   */
   BD_ERR_WORKSPACE = 9,     /* workspace NULL or smaller than the *_workspace_size     */
-  BD_ERR_TENANT_RECORD = 10 /* device status: a bd_tenant record is invalid            */
+  BD_ERR_TENANT_RECORD = 10,/* device status: a bd_tenant record is invalid            */
+  BD_ERR_INTERNAL = 11      /* device status: a kernel's layout self-check failed       */
 } bd_status;
 
 typedef enum { BD_F32 = 0, BD_BF16 = 1, BD_F16 = 2 } bd_dtype;
@@ -78,6 +79,8 @@ typedef enum { BD_SCALE_GROUP = 0, BD_SCALE_ROW = 1, BD_SCALE_COL = 2, BD_SCALE_
 #define BD_DEV_TENANT_RECORD 0x4u /* a bd_tenant record had a bad mode, group size or
                                      NULL / misaligned pointer; its tokens got the base
                                      product only                                      */
+#define BD_DEV_INTERNAL     0x8u  /* a kernel's shared-memory layout self-check failed and
+                                     it returned without writing its outputs            */
 
 /* ---------------------------------------------------------------------------------- */
 /* compress                                                                            */
@@ -160,14 +163,46 @@ bd_status bd_reconstruct(const uint32_t* signs, const void* scales, int32_t scal
 /* ---------------------------------------------------------------------------------- */
 /* multi-tenant apply                                                                  */
 /* ---------------------------------------------------------------------------------- */
+/* Storage layouts of a tenant's sign words (and group-128 scales) for bd_apply_multi.
+ *  ROWMAJOR : signs uint32[d_out][d_in/32] exactly as bd_compress writes them; scales as
+ *             bd_compress writes them (converted to the call's scale_dtype).
+ *  TILED    : the serving layout written by bd_prepare_tenant. The matrix is cut into
+ *             tiles of 512 rows x 256 columns (8 sign words); tile (rb, w) is 4096
+ *             consecutive words [row 0..511][word 0..7] at word offset
+ *             (rb * ceil(d_in/256) + w) * 4096, rows past d_out and words past d_in/32
+ *             zero. For GROUP scales with group_size 128 the scales are tiled the same
+ *             way: tile (rb, w) holds [row 0..511][2 scales] at element offset
+ *             (rb * ceil(d_in/256) + w) * 1024. Other scale modes keep their plain layout.
+ *  The same bits in either layout give the same result; TILED lets every 512-row stage
+ *  of the apply kernel arrive as one contiguous 16 KB block. */
+#define BD_LAYOUT_ROWMAJOR 0
+#define BD_LAYOUT_TILED 1
+
 /* One resident tenant variant of one projection. An array of these lives in DEVICE
  * memory and is read by the kernels (the host never dereferences it). */
 typedef struct {
-  const uint32_t* signs;  /* device, uint32[d_out][d_in/32], 16-byte aligned           */
-  const void* scales;     /* device, per `mode`, dtype = the call's scale_dtype          */
+  const uint32_t* signs;  /* device, per `layout`, 16-byte aligned                       */
+  const void* scales;     /* device, per `mode` and `layout`, dtype = the call's scale_dtype */
   int32_t mode;           /* bd_scale_mode                                               */
   int32_t group_size;     /* GROUP mode: power of two, 32 <= G, G divides d_in           */
+  int32_t layout;         /* BD_LAYOUT_ROWMAJOR or BD_LAYOUT_TILED                        */
+  int32_t reserved;       /* must be 0                                                   */
 } bd_tenant;
+
+/* Bytes of the TILED sign words and scales of one tenant (bd_prepare_tenant outputs). */
+size_t bd_prepared_signs_bytes(int64_t d_out, int64_t d_in);
+size_t bd_prepared_scales_bytes(int64_t d_out, int64_t d_in, int32_t mode, int32_t group_size,
+                                int32_t scale_dtype);
+
+/* bd_prepare_tenant — rewrite one tenant's sign words (uint32[d_out][d_in/32], as
+ * bd_compress writes them) and scales (dtype scale_dtype, BD_F16 or BD_F32) into the
+ * TILED serving layout described above: a pure re-ordering, no value changes. Scales of
+ * modes other than GROUP-128 are copied unchanged. Outputs must not overlap the inputs;
+ * sizes are bd_prepared_signs_bytes / bd_prepared_scales_bytes. Done once when a tenant
+ * is loaded, not per batch. */
+bd_status bd_prepare_tenant(const uint32_t* signs, const void* scales, int32_t scale_dtype,
+                            int32_t mode, int32_t group_size, int64_t d_out, int64_t d_in,
+                            uint32_t* signs_out, void* scales_out, void* stream);
 
 /* Bytes of workspace bd_apply_multi needs. */
 size_t bd_apply_workspace_size(int64_t d_out, int64_t d_in, int64_t batch, int32_t n_tenants);
@@ -202,9 +237,9 @@ bd_status bd_apply_multi(const void* w_base, int32_t w_dtype, int64_t d_out, int
 /* status, diagnostics                                                                 */
 /* ---------------------------------------------------------------------------------- */
 /* Copies the device status word of a workspace (compress or apply) to *flags (host)
- * and SYNCHRONISES `stream`. Returns BD_ERR_TIMEOUT, BD_ERR_TENANT_RECORD or
- * BD_ERR_TENANT_RANGE (in that order of precedence) when the corresponding bit is set,
- * BD_OK when none is. */
+ * and SYNCHRONISES `stream`. Returns BD_ERR_INTERNAL, BD_ERR_TIMEOUT,
+ * BD_ERR_TENANT_RECORD or BD_ERR_TENANT_RANGE (in that order of precedence) when the
+ * corresponding bit is set, BD_OK when none is. */
 bd_status bd_get_status(const void* workspace, uint32_t* flags /* host, may be NULL */,
                         void* stream);
 

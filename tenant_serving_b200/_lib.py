@@ -27,14 +27,16 @@ BD_ERR_TENANT_RANGE = 7
 BD_ERR_TIMEOUT = 8
 BD_ERR_WORKSPACE = 9
 BD_ERR_TENANT_RECORD = 10
+BD_ERR_INTERNAL = 11
 
 BD_F32, BD_BF16, BD_F16 = 0, 1, 2
 BD_SCALE_GROUP, BD_SCALE_ROW, BD_SCALE_COL, BD_SCALE_TENSOR = 0, 1, 2, 3
-BD_DEV_TENANT_RANGE, BD_DEV_TIMEOUT, BD_DEV_TENANT_RECORD = 0x1, 0x2, 0x4
+BD_DEV_TENANT_RANGE, BD_DEV_TIMEOUT, BD_DEV_TENANT_RECORD, BD_DEV_INTERNAL = 0x1, 0x2, 0x4, 0x8
+BD_LAYOUT_ROWMAJOR, BD_LAYOUT_TILED = 0, 1
 
 EXPORTS = (
     "bd_compress", "bd_compress_noalloc", "bd_compress_workspace_size", "bd_reconstruct",
-    "bd_apply_multi",
+    "bd_apply_multi", "bd_prepared_signs_bytes", "bd_prepared_scales_bytes", "bd_prepare_tenant",
     "bd_apply_workspace_size", "bd_get_status", "bd_status_string", "bd_launch_count",
     "bd_profile_enable", "bd_profile_collect", "bd_kernel_name",
 )
@@ -45,7 +47,8 @@ class bd_compress_cfg(ctypes.Structure):
 
 
 class bd_tenant(ctypes.Structure):
-    _fields_ = [("signs", c_void_p), ("scales", c_void_p), ("mode", c_int32), ("group_size", c_int32)]
+    _fields_ = [("signs", c_void_p), ("scales", c_void_p), ("mode", c_int32),
+                ("group_size", c_int32), ("layout", c_int32), ("reserved", c_int32)]
 
 
 class BitDeltaError(RuntimeError):
@@ -83,6 +86,13 @@ def lib():
                                  c_void_p, c_void_p, c_int64, c_void_p, c_int32, c_void_p,
                                  c_size_t, c_void_p]
     L.bd_apply_multi.restype = c_int32
+    L.bd_prepared_signs_bytes.argtypes = [c_int64, c_int64]
+    L.bd_prepared_signs_bytes.restype = c_size_t
+    L.bd_prepared_scales_bytes.argtypes = [c_int64, c_int64, c_int32, c_int32, c_int32]
+    L.bd_prepared_scales_bytes.restype = c_size_t
+    L.bd_prepare_tenant.argtypes = [c_void_p, c_void_p, c_int32, c_int32, c_int32, c_int64, c_int64,
+                                    c_void_p, c_void_p, c_void_p]
+    L.bd_prepare_tenant.restype = c_int32
     L.bd_apply_workspace_size.argtypes = [c_int64, c_int64, c_int64, c_int32]
     L.bd_apply_workspace_size.restype = c_size_t
     L.bd_get_status.argtypes = [c_void_p, POINTER(c_uint32), c_void_p]
@@ -225,18 +235,40 @@ def bd_reconstruct(signs, scales, mode, group_size, d_out, d_in, w_base=None, ou
     return out
 
 
+def bd_prepare_tenant(signs, scales, mode, group_size, d_out, d_in, stream=None):
+    """Wrap ``bd_prepare_tenant``: returns (tiled sign words int32, tiled/plain scales) in
+    the serving layout, allocated with torch."""
+    torch = _torch()
+    _require_cuda(signs, scales)
+    sdt = dtype_code(scales)
+    nb = int(lib().bd_prepared_signs_bytes(int(d_out), int(d_in)))
+    ns = int(lib().bd_prepared_scales_bytes(int(d_out), int(d_in), int(mode), int(group_size), sdt))
+    if nb == 0 or ns == 0:
+        raise BitDeltaError(BD_ERR_CONFIG, "bd_prepare_tenant")
+    so = torch.empty(nb // 4, dtype=torch.int32, device=signs.device)
+    sc = torch.empty(ns // scales.element_size(), dtype=scales.dtype, device=signs.device)
+    rc = lib().bd_prepare_tenant(_ptr(signs), _ptr(scales), sdt, int(mode), int(group_size),
+                                 int(d_out), int(d_in), _ptr(so), _ptr(sc), _stream(stream))
+    check(rc, "bd_prepare_tenant")
+    return so, sc
+
+
 class TenantTable:
     """A device array of ``bd_tenant`` records for one projection. Keeps references to
-    the tensors it points at so they stay alive as long as the table does."""
+    the tensors it points at so they stay alive as long as the table does. Entries are
+    (signs, scales, mode, group_size) or (signs, scales, mode, group_size, layout)."""
 
     def __init__(self, tenants, device):
         torch = _torch()
         self._keep = []
         n = len(tenants)
         arr = (bd_tenant * max(n, 1))()
-        for i, (signs, scales, mode, group_size) in enumerate(tenants):
+        for i, rec in enumerate(tenants):
+            signs, scales, mode, group_size = rec[:4]
+            layout = rec[4] if len(rec) > 4 else BD_LAYOUT_ROWMAJOR
             _require_cuda(signs, scales)
-            arr[i] = bd_tenant(signs.data_ptr(), scales.data_ptr(), int(mode), int(group_size))
+            arr[i] = bd_tenant(signs.data_ptr(), scales.data_ptr(), int(mode), int(group_size),
+                               int(layout), 0)
             self._keep.append((signs, scales))
         raw = bytes(arr)
         self.n = n

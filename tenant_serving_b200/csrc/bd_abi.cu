@@ -10,7 +10,7 @@ namespace bd {
 static const char* const kKernelNames[K_KIND_COUNT] = {
     "delta_stats",       "stats_final",  "scale_signpack", "col_scale_signpack",
     "scale_final",       "reconstruct",  "tenant_bucket",  "base_gemv",
-    "base_tc",           "delta_lut",    "select_fixup",
+    "base_tc",           "delta_lut",    "select_fixup",   "prepare",
 };
 
 const char* kernel_name(int32_t kind) {
@@ -98,6 +98,7 @@ extern "C" const char* bd_status_string(int32_t st) {
     case BD_ERR_TIMEOUT: return "a bounded wait inside a kernel gave up";
     case BD_ERR_WORKSPACE: return "workspace missing or too small";
     case BD_ERR_TENANT_RECORD: return "a bd_tenant record is invalid";
+    case BD_ERR_INTERNAL: return "a kernel's layout self-check failed";
     default: return "unknown status";
   }
 }
@@ -109,6 +110,7 @@ extern "C" bd_status bd_get_status(const void* workspace, uint32_t* flags, void*
   BD_CUDA_TRY(cudaMemcpyAsync(&f, workspace, sizeof(uint32_t), cudaMemcpyDeviceToHost, s));
   BD_CUDA_TRY(cudaStreamSynchronize(s));
   if (flags) *flags = f;
+  if (f & BD_DEV_INTERNAL) return BD_ERR_INTERNAL;
   if (f & BD_DEV_TIMEOUT) return BD_ERR_TIMEOUT;
   if (f & BD_DEV_TENANT_RECORD) return BD_ERR_TENANT_RECORD;
   if (f & BD_DEV_TENANT_RANGE) return BD_ERR_TENANT_RANGE;

@@ -4,12 +4,15 @@
 // per-tenant delta product) and "2. Fused Dequantization ..." (sign bits stay packed in
 // HBM and are expanded on chip). The pages give no kernel for this GPU; the design here:
 //
-//   k_tenant_bucket  one CTA: counting sort of the tenant ids into segments (tenant,
-//                    start, length) and a token permutation. Invalid ids set a status
-//                    bit and join the base-only segment. No host synchronisation.
+//   k_tenant_bucket  one CTA: counting sort of the tenant ids, every tenant's tokens cut
+//                    into groups of <= 2 (tenant, start, length) plus a token
+//                    permutation. Invalid ids set a status bit and join the base-only
+//                    tokens. No host synchronisation.
 //   base product     bf16: tcgen05 tensor-core GEMM (bd_base_tc.cu), fp32: k_base_gemv.
 //                    Both write fp32 partial sums y_part[kz][t][row].
-//   k_delta_lut      one CTA per (segment, 1024-row block): streams the tenant's sign
+//   k_delta_lut      persistent CTAs split the (token group, row) space evenly; groups
+//                    of one tenant are adjacent in it, so its sign words come from HBM
+//                    once and from L2 for the other groups. A CTA streams the
 //                    words through shared memory 256 columns at a time and, per token,
 //                    turns every byte of signs into ONE table lookup: for each 8-column
 //                    chunk a 256-entry table holds sum_j (+/-) x_j for every sign
@@ -36,26 +39,31 @@ constexpr int kMaxTenants = 16384;
 constexpr int kMaxBatch = 65536;
 
 // ------------------------------------------------------------------------------------
-// segments
+// token groups
 // ------------------------------------------------------------------------------------
-struct SegTable {
-  int32_t n_seg;
-  int32_t pad[3];
-  // followed in memory by: tenant[max_seg], start[max_seg], len[max_seg], perm[batch]
-};
+// Tokens are grouped by tenant (a counting sort) and every tenant's tokens are cut into
+// groups of at most kGroupTokens; one delta CTA serves one group for one block of rows.
+// Workspace layout (int32): [0] n_groups, [1..3] pad, then grp_tenant[max_groups],
+// grp_start[max_groups], grp_len[max_groups] (offsets into perm), perm[batch].
+constexpr int kGroupTokens = 2;
+
+inline int max_groups_for(int64_t batch, int32_t n_tenants) {
+  const int64_t keys = batch < (int64_t)n_tenants + 1 ? batch : (int64_t)n_tenants + 1;
+  return (int)((batch + kGroupTokens - 1) / kGroupTokens + keys);
+}
 
 __global__ void __launch_bounds__(1024) k_tenant_bucket(const int32_t* __restrict__ ids, int batch,
-                                                        int n_tenants, int max_seg,
+                                                        int n_tenants, int max_groups,
                                                         int32_t* __restrict__ seg_base,
                                                         uint32_t* __restrict__ status) {
   extern __shared__ int32_t cnt[];  // n_tenants + 1 counters (last = base only)
-  __shared__ int32_t warp_tot[32], warp_seg[32];
+  __shared__ int32_t warp_tot[32], warp_grp[32];
   __shared__ int32_t bad;
   const int nkeys = n_tenants + 1;
-  int32_t* seg_tenant = seg_base + 4;
-  int32_t* seg_start = seg_tenant + max_seg;
-  int32_t* seg_len = seg_start + max_seg;
-  int32_t* perm = seg_len + max_seg;
+  int32_t* grp_tenant = seg_base + 4;
+  int32_t* grp_start = grp_tenant + max_groups;
+  int32_t* grp_len = grp_start + max_groups;
+  int32_t* perm = grp_len + max_groups;
   if (threadIdx.x == 0) {
     status[0] = 0;  // the status word reports this call
     bad = 0;
@@ -71,32 +79,32 @@ __global__ void __launch_bounds__(1024) k_tenant_bucket(const int32_t* __restric
     atomicAdd(&cnt[u < 0 ? n_tenants : u], 1);
   }
   __syncthreads();
-  // exclusive scan of counts and of "count > 0" (segment index), contiguous per thread
+  // exclusive scans of token counts and of group counts, contiguous keys per thread
   const int per = (nkeys + blockDim.x - 1) / blockDim.x;
   const int k0 = threadIdx.x * per, k1 = min(nkeys, k0 + per);
-  int tot = 0, nz = 0;
+  int tot = 0, ng = 0;
   for (int k = k0; k < k1; ++k) {
     tot += cnt[k];
-    nz += cnt[k] > 0;
+    ng += (cnt[k] + kGroupTokens - 1) / kGroupTokens;
   }
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  int itot = tot, inz = nz;
+  int itot = tot, ing = ng;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    int a = __shfl_up_sync(0xffffffffu, itot, o), b = __shfl_up_sync(0xffffffffu, inz, o);
+    int a = __shfl_up_sync(0xffffffffu, itot, o), b = __shfl_up_sync(0xffffffffu, ing, o);
     if (lane >= o) {
       itot += a;
-      inz += b;
+      ing += b;
     }
   }
   if (lane == 31) {
     warp_tot[w] = itot;
-    warp_seg[w] = inz;
+    warp_grp[w] = ing;
   }
   __syncthreads();
   if (w == 0) {
     const int nw = blockDim.x >> 5;
-    int a = lane < nw ? warp_tot[lane] : 0, b = lane < nw ? warp_seg[lane] : 0;
+    int a = lane < nw ? warp_tot[lane] : 0, b = lane < nw ? warp_grp[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       int c = __shfl_up_sync(0xffffffffu, a, o), d = __shfl_up_sync(0xffffffffu, b, o);
@@ -107,24 +115,24 @@ __global__ void __launch_bounds__(1024) k_tenant_bucket(const int32_t* __restric
     }
     if (lane < nw) {
       warp_tot[lane] = a;
-      warp_seg[lane] = b;
+      warp_grp[lane] = b;
     }
   }
   __syncthreads();
   int off = itot - tot + (w > 0 ? warp_tot[w - 1] : 0);
-  int sidx = inz - nz + (w > 0 ? warp_seg[w - 1] : 0);
+  int gidx = ing - ng + (w > 0 ? warp_grp[w - 1] : 0);
   for (int k = k0; k < k1; ++k) {
     const int c = cnt[k];
-    if (c > 0) {
-      seg_tenant[sidx] = (k == n_tenants) ? -1 : k;
-      seg_start[sidx] = off;
-      seg_len[sidx] = c;
-      ++sidx;
+    for (int j = 0; j < c; j += kGroupTokens) {
+      grp_tenant[gidx] = (k == n_tenants) ? -1 : k;
+      grp_start[gidx] = off + j;
+      grp_len[gidx] = min(kGroupTokens, c - j);
+      ++gidx;
     }
     cnt[k] = off;  // becomes the scatter cursor
     off += c;
   }
-  if (threadIdx.x == blockDim.x - 1) seg_base[0] = sidx;  // last thread holds the total
+  if (threadIdx.x == blockDim.x - 1) seg_base[0] = gidx;  // last thread holds the total
   __syncthreads();
   for (int t = threadIdx.x; t < batch; t += blockDim.x) {
     int u = ids[t];
@@ -171,249 +179,549 @@ __global__ void __launch_bounds__(256) k_base_gemv_f32(const float* __restrict__
 // ------------------------------------------------------------------------------------
 // delta product with per-chunk sign lookup tables
 // ------------------------------------------------------------------------------------
-constexpr int LUT_R = 1024;                 // rows per CTA
-constexpr int LUT_THREADS = 512;            // 16 warps
+// Persistent CTAs (one per SM, 32 warps) split the flattened (token group, output row)
+// space evenly; a CTA walks its share in pieces of at most 2048 rows of one group
+// (<= 2 tokens of one tenant). Groups of one tenant are adjacent in that space, so the
+// CTAs working on a tenant run at the same time and its sign words come from HBM once.
+//
+// A piece streams the tenant's sign words 256 columns (8 words) x 512 rows per stage
+// through a 6-deep cp.async ring. Per 256-column window and token, a table
+// T[v][c] = sum_j (bit j of v ? +x : -x)[8c + j] over the 8 columns of chunk c is built
+// in shared memory for every sign byte v; then one byte of signs costs one table read
+// per token.
+//   lanes: q = lane >> 1 picks one of 16 rows, wp = lane & 1 one half of the window
+//   (words 4wp..4wp+3). At step (k, j) a lane reads word 4wp + ((k + q/4) & 3) and its
+//   byte (j + q) & 3: the 32 lanes read 32 different staged words and 32 different
+//   table chunks (= 32 different banks), so neither read has bank conflicts.
+//   table page: it sits at shared address 0x10000, entry (v, token, chunk) at
+//   0x10000 + v * 256 + 4 * (32 * token + chunk). One PRMT of the sign word with the
+//   lane's slot constant (which carries the 0x1 of 0x10000 in its upper half) yields the
+//   whole 32-bit shared address of token 0's entry; token 1's is 128 bytes further, an
+//   immediate. A lookup is PRMT + ld.shared + FADD.
+//   Group-128 scales are one per lane per row (words 4wp..4wp+3 are one group) and are
+//   staged next to the sign words.
+constexpr int LUT_THREADS = 256;    // 8 warps, 64 rows each per stage
+constexpr int LUT_RG = 4;           // 16-row groups per warp per stage
 constexpr int LUT_WARPS = LUT_THREADS / 32;
-constexpr int LUT_TT = 4;                   // tokens per pass (two 64 KB table pages)
-constexpr int LUT_W = 256;                  // columns per window (8 sign words per row)
-constexpr int LUT_NQ = LUT_R / (LUT_WARPS * 4);  // row quads per warp
-constexpr int LUT_PAGE = 65536;             // bytes: 256 sign patterns x 64 slots x 4 B
-constexpr int LUT_BITS_BYTES = LUT_R * 32;  // one window of sign words for LUT_R rows
-constexpr size_t LUT_SMEM = (size_t)(LUT_TT / 2) * LUT_PAGE + 2 * LUT_BITS_BYTES + 64;
+constexpr int LUT_W = 256;          // columns per window
+constexpr int LUT_SB = 512;         // rows per stage: one 16-row slice per warp
+constexpr int LUT_NSB = 4;          // stages (sub-blocks) per window of a piece
+constexpr int LUT_PASS = LUT_SB * LUT_NSB;  // rows per piece
+constexpr int LUT_STAGES = 6;       // cp.async ring depth
+constexpr int LUT_SC = 8;           // staged scale bytes per row per window
+constexpr uint32_t LUT_BITS_STAGE = LUT_SB * 32;
+constexpr uint32_t LUT_SC_STAGE = LUT_SB * LUT_SC;
+constexpr uint32_t LUT_ADDR = 0x10000;  // shared address of the table page
+constexpr uint32_t LUT_HALF = 3 * (LUT_BITS_STAGE + LUT_SC_STAGE);  // ring stages below / above
+constexpr uint32_t LUT_LOW = LUT_ADDR - LUT_HALF;    // first ring byte; dynamic smem must start <=
+constexpr uint32_t LUT_X_STAGE = 4096;  // per ring slot: x of 2 tokens + column scales
+constexpr uint32_t LUT_XBASE = 0x20000 + LUT_HALF;   // x slots of the ring
+constexpr uint32_t LUT_PIECE = LUT_XBASE + LUT_STAGES * LUT_X_STAGE;  // piece descriptor
+constexpr size_t LUT_SMEM = LUT_PIECE + 128;  // requested from the dynamic base
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
-                   (uint32_t)__cvta_generic_to_shared(dst)),
-               "l"(src)
-               : "memory");
+__device__ __forceinline__ uint32_t sh_addr(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ float lds_f32(uint32_t a) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ float lds_f32_128(uint32_t a) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1+128];" : "=f"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ float lds_f16(uint32_t a) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+  return __half2float(__ushort_as_half(v));
+}
+__device__ __forceinline__ void sts_f32(uint32_t a, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(
-                   (uint32_t)__cvta_generic_to_shared(dst)),
-               "l"(src)
-               : "memory");
-}
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-template <bool XBF16>
-__device__ __forceinline__ void load_x8(const void* x, int64_t off, float* v) {
-  if (XBF16) {
-    const uint4 q = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(x) + off);
-    const uint32_t a[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      v[2 * k] = bf16lo(a[k]);
-      v[2 * k + 1] = bf16hi(a[k]);
-    }
-  } else {
-    const float4* p = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(x) + off);
-    const float4 a = p[0], b = p[1];
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-  }
 }
 
 __device__ __forceinline__ float ld_scale(const void* s, bool f16, int64_t i) {
   return f16 ? __half2float(reinterpret_cast<const __half*>(s)[i]) : reinterpret_cast<const float*>(s)[i];
 }
 
-template <bool XBF16>
-__global__ void __launch_bounds__(LUT_THREADS, 1) k_delta_lut(
-    const bd_tenant* __restrict__ tenants, int n_tenants, bool scale_f16,
-    const int32_t* __restrict__ seg_base, int max_seg, const void* __restrict__ x,
-    const float* __restrict__ y_part, int ksplit, int64_t d_out, int64_t d_in, int batch,
-    void* __restrict__ y, bool y_bf16, uint32_t* __restrict__ status) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  const int seg = blockIdx.y;
-  const int n_seg = seg_base[0];
-  if (seg >= n_seg) return;
-  const int32_t* seg_tenant = seg_base + 4;
-  const int32_t* seg_start = seg_tenant + max_seg;
-  const int32_t* seg_len = seg_start + max_seg;
-  const int32_t* perm = seg_len + max_seg;
-  const int u_in = seg_tenant[seg];
-  const int start = seg_start[seg], len = seg_len[seg];
-  const int64_t r0 = (int64_t)blockIdx.x * LUT_R;
-  const int rows = (int)min((int64_t)LUT_R, d_out - r0);
-
-  float* lut = reinterpret_cast<float*>(smem);
-  uint8_t* bits_s = smem + (size_t)(LUT_TT / 2) * LUT_PAGE;
-  float* out_s = lut;  // reused after the last window
-  int* tok_s = reinterpret_cast<int*>(bits_s + 2 * LUT_BITS_BYTES);
-
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int q = lane >> 3;        // row inside the warp's row quad
-  const int wd = lane & 7;        // sign word inside the 256-column window
-  const int64_t wpr = d_in >> 5;  // sign words per row
-  const int nwin = (int)((d_in + LUT_W - 1) / LUT_W);
-
+struct LutPiece {
   bd_tenant T;
-  int mode = BD_SCALE_GROUP, G = 128;
-  int u = u_in;
-  if (u >= 0) {
-    T = tenants[u];
-    mode = T.mode;
-    G = T.group_size;
-    // the table lives in device memory, so its records are checked here
-    const bool ok_mode = mode >= BD_SCALE_GROUP && mode <= BD_SCALE_TENSOR;
-    const bool ok_group = mode != BD_SCALE_GROUP ||
-                          (G >= 32 && (G & (G - 1)) == 0 && (d_in % G) == 0);
-    const bool ok_ptr = T.signs != nullptr && T.scales != nullptr &&
-                        ((reinterpret_cast<uintptr_t>(T.signs) | reinterpret_cast<uintptr_t>(T.scales)) & 15u) == 0;
-    if (!(ok_mode && ok_group && ok_ptr)) {
-      if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(status, BD_DEV_TENANT_RECORD);
-      u = -1;  // base product only
+  int u, mode, G, ntok, t0, t1, rows, sc_kind, layout, pos_step, scale_f16;
+  int64_t rb0;      // first 512-row tile of the piece
+  int64_t r0;
+  int64_t bstride;  // sign words between consecutive 512-row stages
+  int64_t half_stride;  // sign words between rows r and r + 256
+  int64_t sstride;  // staged-scale bytes between consecutive stages
+  int whole;
+};
+
+__device__ __forceinline__ uint32_t lut_bits_stage(int b) {
+  return b < 3 ? LUT_LOW + (uint32_t)b * LUT_BITS_STAGE
+               : 0x20000u + (uint32_t)(b - 3) * LUT_BITS_STAGE;
+}
+__device__ __forceinline__ uint32_t lut_sc_stage(int b) {
+  return b < 3 ? LUT_LOW + 3 * LUT_BITS_STAGE + (uint32_t)b * LUT_SC_STAGE
+               : 0x20000u + 3 * LUT_BITS_STAGE + (uint32_t)(b - 3) * LUT_SC_STAGE;
+}
+
+__device__ __forceinline__ uint32_t lut_x_stage(int b) { return LUT_XBASE + (uint32_t)b * LUT_X_STAGE; }
+
+// Issue the copies of stage (win, sb) into ring buffer b. Staged scales are 2 per row
+// (2 * ssz bytes, row stride 2 * ssz).
+__device__ __forceinline__ void lut_stage(const LutPiece& P, int win, int sb,
+                                          int b, int64_t d_in, bool scale_f16, const void* x,
+                                          bool xbf16, int nwin) {
+  const int tid = threadIdx.x;
+  const int rb = sb * LUT_SB;
+  const int ssz = scale_f16 ? 2 : 4;
+  if (P.layout == BD_LAYOUT_TILED) {
+    // one contiguous 16 KB tile of sign words and (group-128) a 2 / 4 KB tile of scales
+    const int64_t tile = (P.rb0 + sb) * nwin + win;
+    const uint32_t* src = P.T.signs + tile * 4096;
+#pragma unroll
+    for (int c = 0; c < 1024; c += LUT_THREADS)
+      cp_async16(lut_bits_stage(b) + (uint32_t)(c + tid) * 16u, src + (c + tid) * 4);
+    if (P.sc_kind == 1) {
+      const uint8_t* ssrc = reinterpret_cast<const uint8_t*>(P.T.scales) + tile * 1024 * ssz;
+      for (int c = tid; c * 16 < 1024 * ssz; c += LUT_THREADS)
+        cp_async16(lut_sc_stage(b) + (uint32_t)c * 16u, ssrc + c * 16);
+    }
+  } else {
+    if (P.whole) {
+      // two 16-byte copies per thread: rows tid/2 and tid/2 + 256 of the stage, half tid & 1
+      const int64_t wpr = d_in >> 5;
+      // 16-byte copies: copy c = row (c >> 1), half (c & 1) of the stage
+      for (int c = tid; c < 1024; c += LUT_THREADS) {
+        const int row = c >> 1;
+        if (rb + row < P.rows)
+          cp_async16(lut_bits_stage(b) + (uint32_t)c * 16u,
+                     P.T.signs + (P.r0 + rb + row) * wpr + (c & 1) * 4 + win * 8);
+      }
+    } else {
+      const int64_t wpr = d_in >> 5;
+      const int64_t w0 = (int64_t)win * (LUT_W / 32);
+      const int nr = min(LUT_SB, P.rows - rb);
+      const uint32_t* src = P.T.signs + (P.r0 + rb) * wpr + w0;
+      for (int i = tid; i < nr * 8; i += LUT_THREADS) {
+        const int rl = i >> 3, k = i & 7;
+        if (w0 + k < wpr) cp_async4(lut_bits_stage(b) + rl * 32 + k * 4, src + rl * wpr + k);
+      }
+    }
+    if (P.sc_kind == 1) {
+      const int64_t per_row = (d_in / 128) * ssz;
+      for (int r = tid; r < LUT_SB && rb + r < P.rows; r += LUT_THREADS) {
+        const uint8_t* sp = reinterpret_cast<const uint8_t*>(P.T.scales) + (P.r0 + rb + r) * per_row +
+                            win * 2 * ssz;
+        const uint32_t sd = lut_sc_stage(b) + (uint32_t)(r * 2 * ssz);
+        if (scale_f16) cp_async4(sd, sp);
+        else cp_async8(sd, sp);
+      }
     }
   }
+  // the first stage of a window also brings the window's slice of x (both tokens) and,
+  // for column scales, the window's scales: [x0 1 KB][x1 1 KB][col scales 1 KB]
+  if (sb == 0 && tid < 3 * 64) {
+    const int part = tid >> 6, k = tid & 63;  // 64 x 16 B per part (LUT_THREADS >= 192)
+    const int64_t col0 = (int64_t)win * LUT_W;
+    const int xb = xbf16 ? 2 : 4;
+    const uint32_t dst = lut_x_stage(b) + (uint32_t)(part * 1024 + k * 16);
+    if (part < 2) {
+      const int64_t col = col0 + (int64_t)k * (16 / xb);
+      if (part < P.ntok && k * 16 < LUT_W * xb && col < d_in) {
+        const int t = part == 0 ? P.t0 : P.t1;
+        cp_async16(dst, reinterpret_cast<const uint8_t*>(x) + ((int64_t)t * d_in + col) * xb);
+      }
+    } else if (P.mode == BD_SCALE_COL) {
+      const int64_t col = col0 + (int64_t)k * (16 / ssz);
+      if (k * 16 < LUT_W * ssz && col < d_in)
+        cp_async16(dst, reinterpret_cast<const uint8_t*>(P.T.scales) + col * ssz);
+    }
+  }
+}
 
-  // per-lane lookup constants: byte order rotated by q so a warp hits 32 distinct banks
-  uint32_t sel[4], slot[2][4];
+// Build the sign tables of one window for the piece's tokens from the x slice (and
+// column scales) staged in ring slot b.
+template <bool XBF16>
+__device__ __forceinline__ void lut_build(const LutPiece& P, int win, int b, int64_t d_in,
+                                          bool scale_f16) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int c = lane;  // chunk of the window
+  // this thread fills the sign patterns with high nibble h and h + 8 (h = warp, 8 warps)
+  const int64_t col = (int64_t)win * LUT_W + 8 * c;
+  const uint32_t xs = lut_x_stage(b);
+  float sc[8];
+  if (P.mode == BD_SCALE_COL) {
+    if (scale_f16) {
+      uint4 v;
+      asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                   : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(xs + 2048 + 16 * c));
+      const uint32_t a[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const __half2 hh = *reinterpret_cast<const __half2*>(&a[k]);
+        sc[2 * k] = __low2float(hh);
+        sc[2 * k + 1] = __high2float(hh);
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) sc[k] = lds_f32(xs + 2048 + 32 * c + 4 * k);
+    }
+  }
+#pragma unroll
+  for (int tt = 0; tt < 2; ++tt) {
+    if (tt < P.ntok) {
+      float xv[8];
+      if (col < d_in) {
+        if (XBF16) {
+          uint4 v;
+          asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                       : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                       : "r"(xs + 1024 * tt + 16 * c));
+          const uint32_t a[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            xv[2 * k] = bf16lo(a[k]);
+            xv[2 * k + 1] = bf16hi(a[k]);
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) xv[k] = lds_f32(xs + 1024 * tt + 32 * c + 4 * k);
+        }
+        if (P.mode == BD_SCALE_COL) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) xv[k] *= sc[k];
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) xv[k] = 0.f;
+      }
+      float p01[4], p23[4];
+#pragma unroll
+      for (int n = 0; n < 4; ++n) {
+        p01[n] = ((n & 1) ? xv[0] : -xv[0]) + ((n & 2) ? xv[1] : -xv[1]);
+        p23[n] = ((n & 1) ? xv[2] : -xv[2]) + ((n & 2) ? xv[3] : -xv[3]);
+      }
+      float lo16[16];
+#pragma unroll
+      for (int lo = 0; lo < 16; ++lo) lo16[lo] = p01[lo & 3] + p23[lo >> 2];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int h = warp + 8 * hh;
+        const float hi = (((h & 1) ? xv[4] : -xv[4]) + ((h & 2) ? xv[5] : -xv[5])) +
+                         (((h & 4) ? xv[6] : -xv[6]) + ((h & 8) ? xv[7] : -xv[7]));
+        const uint32_t base = LUT_ADDR + (uint32_t)(h << 12) + 4u * (uint32_t)(32 * tt + c);
+#pragma unroll
+        for (int lo = 0; lo < 16; ++lo) sts_f32(base + (uint32_t)lo * 256u, lo16[lo] + hi);
+      }
+    }
+  }
+}
+
+// Generic path: group sizes other than 128 (one scale per word from global memory) and
+// windows that run past d_in. Recomputes the lane constants itself (slow path).
+template <int NT>
+__device__ __forceinline__ float2 lut_rows_generic(uint32_t wrow, uint32_t srow, const LutPiece& P,
+                                                int sb, int i, int win, int64_t d_in,
+                                                bool scale_f16) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int q = lane >> 1, wp = lane & 1;
+  const int rl = sb * LUT_SB + warp * (16 * LUT_RG) + i * 16 + q;  // row inside the piece
+  float a0 = 0.f, a1 = 0.f;
+  if (rl >= P.rows) return make_float2(0.f, 0.f);
+#pragma unroll 1
+  for (int k = 0; k < 4; ++k) {
+    const int wi = 4 * wp + ((k + (q >> 2)) & 3);
+    const int64_t col = (int64_t)win * LUT_W + 32 * wi;
+    if (col >= d_in) continue;
+    const uint32_t word = lds_u32(wrow + 4u * (uint32_t)wi);
+    float p0 = 0.f, p1 = 0.f;
+    for (int j = 0; j < 4; ++j) {
+      const int b = (j + q) & 3;
+      const uint32_t idx = LUT_ADDR + (((word >> (8 * b)) & 0xFFu) << 8) + 4u * (uint32_t)(4 * wi + b);
+      p0 += lds_f32(idx);
+      if (NT == 2) p1 += lds_f32_128(idx);
+    }
+    float sw = 1.f;
+    if (P.sc_kind == 1) {  // staged group-128 scales: group (wi >> 2) of the window
+      const uint32_t a = srow + (uint32_t)((wi >> 2) * (scale_f16 ? 2 : 4));
+      sw = scale_f16 ? lds_f16(a) : lds_f32(a);
+    } else if (P.sc_kind == 2) {
+      sw = ld_scale(P.T.scales, scale_f16, (P.r0 + rl) * (d_in / P.G) + col / P.G);
+    }
+    a0 = fmaf(sw, p0, a0);
+    if (NT == 2) a1 = fmaf(sw, p1, a1);
+  }
+  return make_float2(a0, a1);
+}
+
+// The stage loop of one piece. SC: 0 = no per-word scale (row / col / tensor modes, or
+// the generic path, which handles scales itself), 1 = staged fp16 group-128 scales,
+// 2 = staged fp32 group-128 scales. GENERIC: group sizes other than 128 or a last window
+// that runs past d_in.
+template <bool XBF16, int NT, int SC, bool GENERIC>
+__device__ __forceinline__ void lut_piece(const LutPiece& P, float (&acc)[LUT_NSB][LUT_RG][2], int nwin,
+                                          int64_t d_in, const void* x, const uint32_t (&sel)[4],
+                                          const uint32_t (&slot2)[4][2], const uint32_t (&wofs)[4],
+                                          int warp, int q, int wp) {
+  const bool f16s = P.scale_f16 != 0;
+  const int ssz = GENERIC ? (f16s ? 2 : 4) : (SC == 2 ? 4 : 2);
+  const int rows = P.rows;
+  const int nsb = (rows + LUT_SB - 1) / LUT_SB;  // 1..4
+  int pw = 0, ps = 0;
+#pragma unroll
+  for (int i = 0; i < LUT_STAGES - 1; ++i) {
+    if (pw < nwin) {
+      lut_stage(P, pw, ps, i, d_in, P.scale_f16 != 0, x, XBF16, nwin);
+      if (++ps == nsb) { ps = 0; ++pw; }
+    }
+    cp_async_commit();
+  }
+  int bcur = 0, bnext = LUT_STAGES - 1;
+  for (int win = 0; win < nwin; ++win) {
+#pragma unroll
+    for (int sb = 0; sb < LUT_NSB; ++sb) {
+      if (sb < nsb) {
+        if (pw < nwin) {
+          lut_stage(P, pw, ps, bnext, d_in, P.scale_f16 != 0, x, XBF16, nwin);
+          if (++ps == nsb) { ps = 0; ++pw; }
+        }
+        cp_async_commit();
+        cp_async_wait<LUT_STAGES - 1>();
+        __syncthreads();
+        if (sb == 0) {  // new window: build its tables from the staged x slice
+          lut_build<XBF16>(P, win, bcur, d_in, P.scale_f16 != 0);
+          __syncthreads();
+        }
+#pragma unroll
+        for (int i = 0; i < LUT_RG; ++i) {  // the warp's 16-row groups of this stage
+          const int rs = warp * (16 * LUT_RG) + i * 16;  // first row of the group in the stage
+          const uint32_t wrow = lut_bits_stage(bcur) + (uint32_t)((rs + q) * 32);
+          // the fast path runs every row group unconditionally (no branch, so the groups'
+          // loads interleave); rows past the piece read stale staging data and their
+          // results are never written out
+          if (!GENERIC || sb * LUT_SB + rs < rows) {
+            if (!GENERIC) {
+              float s_ = 1.f;
+              if (SC != 0) {
+                const uint32_t sa = lut_sc_stage(bcur) + (uint32_t)((rs + q) * 2 * ssz + wp * ssz);
+                s_ = SC == 1 ? lds_f16(sa) : lds_f32(sa);
+              }
+              // 16 independent table reads per token, summed as a tree (depth 4)
+              uint32_t wd[4];
+#pragma unroll
+              for (int k = 0; k < 4; ++k) wd[k] = lds_u32(wrow + wofs[k]);
+              float w0[4], w1[4];
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                float v0[4], v1[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  const uint32_t idx = __byte_perm(wd[k], slot2[k][j >> 1], sel[j]);
+                  v0[j] = lds_f32(idx);
+                  if (NT == 2) v1[j] = lds_f32_128(idx);
+                }
+                w0[k] = (v0[0] + v0[1]) + (v0[2] + v0[3]);
+                if (NT == 2) w1[k] = (v1[0] + v1[1]) + (v1[2] + v1[3]);
+              }
+              acc[sb][i][0] = fmaf(s_, (w0[0] + w0[1]) + (w0[2] + w0[3]), acc[sb][i][0]);
+              if (NT == 2) acc[sb][i][1] = fmaf(s_, (w1[0] + w1[1]) + (w1[2] + w1[3]), acc[sb][i][1]);
+            } else {
+              const uint32_t srow = lut_sc_stage(bcur) + (uint32_t)((rs + q) * 2 * ssz);
+              const float2 r = lut_rows_generic<NT>(wrow, srow, P, sb, i, win, d_in, f16s);
+              acc[sb][i][0] += r.x;
+              acc[sb][i][1] += r.y;
+            }
+          }
+        }
+        __syncthreads();
+        bcur = bcur + 1 == LUT_STAGES ? 0 : bcur + 1;
+        bnext = bnext + 1 == LUT_STAGES ? 0 : bnext + 1;
+      }
+    }
+  }
+}
+
+// Per-lane lookup constants (see the comment above k_delta_lut's lookup loop).
+__device__ __forceinline__ void lut_lane_constants(int q, int wp, uint32_t (&sel)[4],
+                                                   uint32_t (&slot2)[4][2], uint32_t (&wofs)[4]) {
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const int b = (j + q) & 3;
-    sel[j] = 0x7604u | ((uint32_t)b << 4);
-    slot[0][j] = 4u * (uint32_t)(4 * wd + b);
-    slot[1][j] = 4u * (uint32_t)(32 + 4 * wd + b);
+    sel[j] = 0x7600u | ((uint32_t)b << 4) | (uint32_t)(4 + (j & 1));
   }
-
-  for (int tg = 0; tg < len; tg += LUT_TT) {
-    const int ntok = min(LUT_TT, len - tg);
-    if (tid < LUT_TT) tok_s[tid] = tid < ntok ? perm[start + tg + tid] : -1;
-    float acc[LUT_NQ][LUT_TT];
 #pragma unroll
-    for (int i = 0; i < LUT_NQ; ++i)
+  for (int k = 0; k < 4; ++k) {
+    const int wi = 4 * wp + ((k + (q >> 2)) & 3);
+    wofs[k] = 4u * (uint32_t)wi;
 #pragma unroll
-      for (int t = 0; t < LUT_TT; ++t) acc[i][t] = 0.f;
-    __syncthreads();
-
-    if (u >= 0) {
-      // stage window 0 of sign words
-      // 16-byte copies when every row starts 16-byte aligned and windows are whole
-      // (d_in % 256 == 0), else one 4-byte copy per sign word.
-      const bool whole = (d_in % LUT_W) == 0;
-      auto stage = [&](int win, int buf) {
-        uint8_t* dst = bits_s + (size_t)buf * LUT_BITS_BYTES;
-        const int64_t w0 = (int64_t)win * (LUT_W / 32);
-        if (whole) {
-          for (int i = tid; i < LUT_R * 2; i += LUT_THREADS) {
-            const int rl = i >> 1, half = i & 1;
-            if (rl < rows) cp_async16(dst + rl * 32 + half * 16, T.signs + (r0 + rl) * wpr + w0 + half * 4);
-          }
-        } else {
-          for (int i = tid; i < LUT_R * 8; i += LUT_THREADS) {
-            const int rl = i >> 3, k = i & 7;
-            if (rl < rows && w0 + k < wpr) cp_async4(dst + rl * 32 + k * 4, T.signs + (r0 + rl) * wpr + w0 + k);
-          }
-        }
-      };
-      stage(0, 0);
-      cp_async_commit();
-      for (int win = 0; win < nwin; ++win) {
-        if (win + 1 < nwin) stage(win + 1, (win + 1) & 1);
-        cp_async_commit();
-        // ---- build the tables of this window: T[v][slot], slot = 32*(tt&1) + chunk
-        {
-          const int c = lane;      // chunk (8 columns) of the window
-          const int h = warp;      // high nibble of the sign byte this thread fills
-          const int64_t col = (int64_t)win * LUT_W + 8 * c;
-#pragma unroll
-          for (int tt = 0; tt < LUT_TT; ++tt) {
-            if (tt < ntok) {
-              const int t = tok_s[tt];
-              float xv[8];
-              if (col < d_in) {
-                load_x8<XBF16>(x, (int64_t)t * d_in + col, xv);
-                if (mode == BD_SCALE_COL) {
-#pragma unroll
-                  for (int k = 0; k < 8; ++k) xv[k] *= ld_scale(T.scales, scale_f16, col + k);
-                }
-              } else {
-#pragma unroll
-                for (int k = 0; k < 8; ++k) xv[k] = 0.f;
-              }
-              float p01[4], p23[4];
-#pragma unroll
-              for (int n = 0; n < 4; ++n) {
-                p01[n] = ((n & 1) ? xv[0] : -xv[0]) + ((n & 2) ? xv[1] : -xv[1]);
-                p23[n] = ((n & 1) ? xv[2] : -xv[2]) + ((n & 2) ? xv[3] : -xv[3]);
-              }
-              const float hi = (((h & 1) ? xv[4] : -xv[4]) + ((h & 2) ? xv[5] : -xv[5])) +
-                               (((h & 4) ? xv[6] : -xv[6]) + ((h & 8) ? xv[7] : -xv[7]));
-              float* page = lut + (size_t)(tt >> 1) * (LUT_PAGE / 4);
-              const int sl = 32 * (tt & 1) + c;
-#pragma unroll
-              for (int n = 0; n < 16; ++n) {
-                const float lo = p01[n & 3] + p23[n >> 2];
-                page[((h << 4) | n) * 64 + sl] = lo + hi;
-              }
-            }
-          }
-        }
-        if (win + 1 < nwin) cp_async_wait<1>();
-        else cp_async_wait<0>();
-        __syncthreads();
-        // ---- lookups
-        const uint32_t* wbuf = reinterpret_cast<const uint32_t*>(bits_s + (size_t)(win & 1) * LUT_BITS_BYTES);
-        const int64_t wcol = (int64_t)win * LUT_W + 32 * wd;
-        const bool wvalid = wcol < d_in;
-#pragma unroll
-        for (int iq = 0; iq < LUT_NQ; ++iq) {
-          const int rl = (warp * LUT_NQ + iq) * 4 + q;
-          if (rl < rows && wvalid) {
-            const uint32_t word = wbuf[rl * 8 + wd];
-            float s = 1.f;
-            if (mode == BD_SCALE_GROUP)
-              s = ld_scale(T.scales, scale_f16, (r0 + rl) * (d_in / G) + wcol / G);
-#pragma unroll
-            for (int tt = 0; tt < LUT_TT; ++tt) {
-              const uint8_t* page = reinterpret_cast<const uint8_t*>(lut) + (size_t)(tt >> 1) * LUT_PAGE;
-              float p = 0.f;
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const uint32_t idx = __byte_perm(word, slot[tt & 1][j], sel[j]);
-                p += *reinterpret_cast<const float*>(page + idx);
-              }
-              acc[iq][tt] = fmaf(s, p, acc[iq][tt]);
-            }
-          }
-        }
-        __syncthreads();
-      }
+    for (int hh = 0; hh < 2; ++hh) {
+      const uint32_t s0 = 4u * (uint32_t)(4 * wi + ((2 * hh + q) & 3));
+      const uint32_t s1 = 4u * (uint32_t)(4 * wi + ((2 * hh + 1 + q) & 3));
+      slot2[k][hh] = s0 | (s1 << 8) | (LUT_ADDR & 0xFFFF0000u);
     }
-    // ---- reduce the 8 lanes of each row and stage per-token results
-#pragma unroll
-    for (int iq = 0; iq < LUT_NQ; ++iq) {
-#pragma unroll
-      for (int tt = 0; tt < LUT_TT; ++tt) {
-        float v = acc[iq][tt];
-        v += __shfl_xor_sync(0xffffffffu, v, 1);
-        v += __shfl_xor_sync(0xffffffffu, v, 2);
-        v += __shfl_xor_sync(0xffffffffu, v, 4);
-        const int rl = (warp * LUT_NQ + iq) * 4 + q;
-        if (wd == 0) out_s[tt * LUT_R + rl] = v;
+  }
+}
+
+template <bool XBF16>
+__global__ void __launch_bounds__(LUT_THREADS, 1) k_delta_lut(
+    const bd_tenant* __restrict__ tenants, bool scale_f16, const int32_t* __restrict__ seg_base,
+    int max_groups, const void* __restrict__ x, const float* __restrict__ y_part, int ksplit,
+    int64_t d_out, int64_t d_in, int batch, void* __restrict__ y, bool y_bf16,
+    uint32_t* __restrict__ status) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const uint32_t base = sh_addr(smem);
+  if (base > LUT_LOW) {  // the fixed layout needs the dynamic window to start low enough
+    if (threadIdx.x == 0) atomicOr(status, BD_DEV_INTERNAL);
+    return;
+  }
+  LutPiece& piece = *reinterpret_cast<LutPiece*>(smem + (LUT_PIECE - base));
+  float* out_s = reinterpret_cast<float*>(smem + (LUT_ADDR - base));  // after the last window
+
+  const int32_t* grp_tenant = seg_base + 4;
+  const int32_t* grp_start = grp_tenant + max_groups;
+  const int32_t* grp_len = grp_start + max_groups;
+  const int32_t* perm = grp_len + max_groups;
+  // the (token group, 512-row tile) space is split evenly over the CTAs; a piece is up to
+  // LUT_NSB consecutive tiles of one group
+  const int n_groups = seg_base[0];
+  const int64_t n_rt = (d_out + LUT_SB - 1) / LUT_SB;
+  const int64_t total = (int64_t)n_groups * n_rt;
+  const int64_t share = (total + gridDim.x - 1) / gridDim.x;
+  int64_t pos = (int64_t)blockIdx.x * share;
+  const int64_t end = min(total, pos + share);
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int q = lane >> 1, wp = lane & 1;
+  const int nwin = (int)((d_in + LUT_W - 1) / LUT_W);
+  // per-lane lookup constants. sel[j]: byte 0 <- slot byte (j & 1) of slot2[k][j >> 1],
+  // byte 1 <- sign byte (j + q) & 3, bytes 2-3 <- 0x0001 (the table's 0x10000).
+  uint32_t sel[4], slot2[4][2], wofs[4];
+  lut_lane_constants(q, wp, sel, slot2, wofs);
+
+  while (pos < end) {
+    if (tid == 0) {
+      LutPiece Q;
+      const int g = (int)(pos / n_rt);
+      Q.rb0 = pos - (int64_t)g * n_rt;
+      const int64_t ntiles = min((int64_t)LUT_NSB, min(n_rt - Q.rb0, end - pos));
+      Q.r0 = Q.rb0 * LUT_SB;
+      Q.rows = (int)min(ntiles * LUT_SB, d_out - Q.r0);
+      Q.pos_step = (int)ntiles;
+      Q.u = grp_tenant[g];
+      Q.ntok = grp_len[g];
+      Q.t0 = perm[grp_start[g]];
+      Q.t1 = Q.ntok > 1 ? perm[grp_start[g] + 1] : Q.t0;
+      Q.mode = BD_SCALE_GROUP;
+      Q.G = 128;
+      Q.T.signs = nullptr;
+      Q.T.scales = nullptr;
+      if (Q.u >= 0) {
+        Q.T = tenants[Q.u];
+        Q.mode = Q.T.mode;
+        Q.G = Q.T.group_size;
+        // the table lives in device memory, so its records are checked here
+        const bool ok_mode = Q.mode >= BD_SCALE_GROUP && Q.mode <= BD_SCALE_TENSOR;
+        const bool ok_group = Q.mode != BD_SCALE_GROUP ||
+                              (Q.G >= 32 && (Q.G & (Q.G - 1)) == 0 && (d_in % Q.G) == 0);
+        const bool ok_ptr = Q.T.signs != nullptr && Q.T.scales != nullptr &&
+                            ((reinterpret_cast<uintptr_t>(Q.T.signs) |
+                              reinterpret_cast<uintptr_t>(Q.T.scales)) & 15u) == 0;
+        const bool ok_layout = (Q.T.layout == BD_LAYOUT_ROWMAJOR || Q.T.layout == BD_LAYOUT_TILED) &&
+                               Q.T.reserved == 0;
+        if (!(ok_mode && ok_group && ok_ptr && ok_layout)) {
+          atomicOr(status, BD_DEV_TENANT_RECORD);
+          Q.u = -1;  // base product only
+        }
       }
+      Q.whole = (d_in % LUT_W) == 0;
+      Q.layout = Q.u >= 0 ? Q.T.layout : BD_LAYOUT_ROWMAJOR;
+      // 0: no per-word scale; 1: staged group-128 scales (tiled, or row-major with whole
+      // windows); 2: group scales read from global memory per word
+      Q.sc_kind = Q.mode != BD_SCALE_GROUP
+                      ? 0
+                      : ((Q.G == 128 && (Q.whole || Q.layout == BD_LAYOUT_TILED)) ? 1 : 2);
+      Q.scale_f16 = scale_f16 ? 1 : 0;
+      Q.bstride = (int64_t)LUT_SB * (d_in >> 5);
+      Q.half_stride = (int64_t)256 * (d_in >> 5);
+      Q.sstride = (int64_t)LUT_SB * (d_in / 128) * (scale_f16 ? 2 : 4);
+      piece = Q;
     }
     __syncthreads();
-    // ---- combine with the base product and write y in request order
+    const LutPiece& P = piece;
+    pos += P.pos_step;
+
+    float acc[LUT_NSB][LUT_RG][2];  // [sub-block][16-row group][token]
+#pragma unroll
+    for (int i = 0; i < LUT_NSB; ++i)
+#pragma unroll
+      for (int j = 0; j < LUT_RG; ++j) acc[i][j][0] = acc[i][j][1] = 0.f;
+
+    if (P.u >= 0) {
+      // one specialised stage loop per (tokens, scale kind, path), chosen once per piece
+      const bool generic = P.sc_kind == 2 || !P.whole;
+      const int ntok = P.ntok;
+#define BD_PIECE(NT, SC, GEN) \
+  lut_piece<XBF16, NT, SC, GEN>(P, acc, nwin, d_in, x, sel, slot2, wofs, warp, q, wp)
+      if (generic) {
+        if (ntok == 2) BD_PIECE(2, 0, true); else BD_PIECE(1, 0, true);
+      } else if (P.sc_kind == 1) {
+        if (scale_f16) { if (ntok == 2) BD_PIECE(2, 1, false); else BD_PIECE(1, 1, false); }
+        else { if (ntok == 2) BD_PIECE(2, 2, false); else BD_PIECE(1, 2, false); }
+      } else {
+        if (ntok == 2) BD_PIECE(2, 0, false); else BD_PIECE(1, 0, false);
+      }
+#undef BD_PIECE
+    }
+    // ---- reduce the two lanes of each row, stage per-token results
+#pragma unroll
+    for (int sb = 0; sb < LUT_NSB; ++sb) {
+#pragma unroll
+      for (int i = 0; i < LUT_RG; ++i) {
+#pragma unroll
+        for (int tt = 0; tt < 2; ++tt) {
+          const float v = acc[sb][i][tt] + __shfl_xor_sync(0xffffffffu, acc[sb][i][tt], 1);
+          const int rl = sb * LUT_SB + warp * (16 * LUT_RG) + i * 16 + q;
+          if (wp == 0) out_s[tt * LUT_PASS + rl] = v;
+        }
+      }
+    }
+    __syncthreads();
+    // ---- combine with the base product, write y in request order
     float rs = 1.f;
-    if (u >= 0 && mode == BD_SCALE_TENSOR) rs = ld_scale(T.scales, scale_f16, 0);
-    for (int tt = 0; tt < ntok; ++tt) {
-      const int t = tok_s[tt];
-      for (int rl = tid; rl < rows; rl += LUT_THREADS) {
-        const int64_t row = r0 + rl;
-        float base = 0.f;
-        for (int kz = 0; kz < ksplit; ++kz) base += y_part[((int64_t)kz * batch + t) * d_out + row];
+    if (P.u >= 0 && P.mode == BD_SCALE_TENSOR) rs = ld_scale(P.T.scales, scale_f16, 0);
+    for (int tt = 0; tt < P.ntok; ++tt) {
+      const int t = tt == 0 ? P.t0 : P.t1;
+      for (int rl = tid; rl < P.rows; rl += LUT_THREADS) {
+        const int64_t row = P.r0 + rl;
+        float bsum = 0.f;
+        for (int kz = 0; kz < ksplit; ++kz) bsum += y_part[((int64_t)kz * batch + t) * d_out + row];
         float d = 0.f;
-        if (u >= 0) {
+        if (P.u >= 0) {
           float sc = rs;
-          if (mode == BD_SCALE_ROW) sc = ld_scale(T.scales, scale_f16, row);
-          d = sc * out_s[tt * LUT_R + rl];
+          if (P.mode == BD_SCALE_ROW) sc = ld_scale(P.T.scales, scale_f16, row);
+          d = sc * out_s[tt * LUT_PASS + rl];
         }
-        const float v = base + d;
+        const float v = bsum + d;
         if (y_bf16)
           reinterpret_cast<uint16_t*>(y)[(int64_t)t * d_out + row] = (uint16_t)f2bf_bits(v);
         else
@@ -429,7 +737,7 @@ __global__ void __launch_bounds__(LUT_THREADS, 1) k_delta_lut(
 // ------------------------------------------------------------------------------------
 namespace {
 struct ApplyLayout {
-  int max_seg;
+  int max_groups;
   TcPlan tc;
   int ksplit;
   size_t off_seg, off_part, total;
@@ -437,8 +745,8 @@ struct ApplyLayout {
 
 ApplyLayout layout_apply(int64_t d_out, int64_t d_in, int64_t batch, int32_t n_tenants, bool tc) {
   ApplyLayout L;
-  L.max_seg = (int)(batch < (int64_t)n_tenants + 1 ? batch : (int64_t)n_tenants + 1);
-  if (L.max_seg < 1) L.max_seg = 1;
+  L.max_groups = max_groups_for(batch, n_tenants);
+  if (L.max_groups < 1) L.max_groups = 1;
   L.ksplit = 1;
   if (tc) {
     L.tc = plan_base_tc(d_out, d_in, batch);
@@ -446,7 +754,7 @@ ApplyLayout layout_apply(int64_t d_out, int64_t d_in, int64_t batch, int32_t n_t
   }
   size_t off = kStatusBytes;
   L.off_seg = off;
-  off = align_up(off + (16 + 3 * (size_t)L.max_seg * 4 + (size_t)batch * 4), 256);
+  off = align_up(off + (16 + 3 * (size_t)L.max_groups * 4 + (size_t)batch * 4), 256);
   L.off_part = off;
   off = align_up(off + (size_t)L.ksplit * batch * d_out * sizeof(float), 256);
   L.total = off;
@@ -485,7 +793,7 @@ bd_status apply_impl(const void* w_base, int32_t w_dtype, int64_t d_out, int64_t
   int32_t* seg = reinterpret_cast<int32_t*>(ws + L.off_seg);
   float* y_part = reinterpret_cast<float*>(ws + L.off_part);
 
-  // 1. bucket tokens by tenant
+  // 1. bucket tokens by tenant into groups
   const size_t bucket_smem = (size_t)(n_tenants + 1) * sizeof(int32_t);
   static bool bucket_attr = false;
   if (!bucket_attr) {
@@ -497,8 +805,8 @@ bd_status apply_impl(const void* w_base, int32_t w_dtype, int64_t d_out, int64_t
     bucket_attr = true;
   }
   launch_begin(K_TENANT_BUCKET, s);
-  k_tenant_bucket<<<1, 1024, bucket_smem, s>>>(tenant_ids, (int)batch, n_tenants, L.max_seg, seg,
-                                               status);
+  k_tenant_bucket<<<1, 1024, bucket_smem, s>>>(tenant_ids, (int)batch, n_tenants, L.max_groups,
+                                               seg, status);
   launch_end(K_TENANT_BUCKET, s);
   BD_LAUNCH_CHECK();
 
@@ -515,9 +823,9 @@ bd_status apply_impl(const void* w_base, int32_t w_dtype, int64_t d_out, int64_t
     BD_LAUNCH_CHECK();
   }
 
-  // 3. delta product per (segment, row block) fused with the combine
-  static bool lut_attr[2] = {false, false};
+  // 3. delta product over the (token group, row) space, fused with the combine
   auto kfn = tc ? k_delta_lut<true> : k_delta_lut<false>;
+  static bool lut_attr[2] = {false, false};
   if (!lut_attr[tc ? 1 : 0]) {
     if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LUT_SMEM) !=
         cudaSuccess) {
@@ -526,11 +834,11 @@ bd_status apply_impl(const void* w_base, int32_t w_dtype, int64_t d_out, int64_t
     }
     lut_attr[tc ? 1 : 0] = true;
   }
-  dim3 grid((unsigned)((d_out + LUT_R - 1) / LUT_R), (unsigned)L.max_seg);
   launch_begin(K_DELTA_LUT, s);
-  kfn<<<grid, LUT_THREADS, LUT_SMEM, s>>>(tenants, n_tenants, scale_dtype == BD_F16, seg, L.max_seg,
-                                          x, y_part, L.ksplit, d_out, d_in, (int)batch, y,
-                                          y_dtype == BD_BF16, status);
+  kfn<<<(unsigned)sm_count(), LUT_THREADS, LUT_SMEM, s>>>(tenants, scale_dtype == BD_F16, seg,
+                                                         L.max_groups, x, y_part, L.ksplit, d_out,
+                                                         d_in, (int)batch, y, y_dtype == BD_BF16,
+                                                         status);
   launch_end(K_DELTA_LUT, s);
   BD_LAUNCH_CHECK();
   return BD_OK;

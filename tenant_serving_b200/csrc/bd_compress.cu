@@ -78,7 +78,15 @@ struct Vec<false> {  // 4 fp32 per 16 bytes
   }
 };
 
-__device__ __forceinline__ float clamp_delta(float d, const ClipParams& c) {
+// The four fp32 values the main pass needs from ClipParams.
+struct ClipF {
+  float lo_up, hi_dn, lo_val, hi_val;
+};
+__device__ __forceinline__ ClipF load_clip(const ClipParams* c) {
+  return ClipF{c->lo_up, c->hi_dn, c->lo_val, c->hi_val};
+}
+
+__device__ __forceinline__ float clamp_delta(float d, const ClipF& c) {
   // Comparisons against the float thresholds are exactly the comparisons of the float
   // delta with the fp64 bounds; the replacement keeps the sign of the fp64 bound.
   return d < c.lo_up ? c.lo_val : (d > c.hi_dn ? c.hi_val : d);
@@ -215,11 +223,13 @@ __global__ void k_stats_final(const uint4* __restrict__ wb, const uint4* __restr
 // ------------------------------------------------------------------------------------
 // main pass for GROUP / ROW / TENSOR
 // ------------------------------------------------------------------------------------
-// A task is (row, segment of seg_chunks chunks); a chunk is 32 lanes x 16 bytes.
-template <bool BF16, int SEGC>
-__global__ void __launch_bounds__(256) k_scale_signpack(
-    const uint8_t* __restrict__ wb, const uint8_t* __restrict__ wf, int64_t d_out, int64_t d_in,
-    int mode, int group, int seg_chunks, int nseg, const ClipParams* __restrict__ clipp,
+// A task is (row, segment of seg_chunks chunks); a chunk is 32 lanes x 16 bytes. Column
+// arithmetic is 32-bit (d_in < 2^31 is checked on the host) and the group size is a power
+// of two, so group indices are shifts.
+template <bool BF16, int SEGC, bool CLIP, bool GROUP>
+__global__ void __launch_bounds__(256, 3) k_scale_signpack(
+    const uint8_t* __restrict__ wb, const uint8_t* __restrict__ wf, int64_t d_out, int d_in,
+    int lg, int seg_chunks, int nseg, const ClipParams* __restrict__ clipp,
     uint32_t* __restrict__ signs, float* __restrict__ scales, double* __restrict__ partials) {
   using V = Vec<BF16>;
   constexpr int VEC = V::N;
@@ -230,17 +240,19 @@ __global__ void __launch_bounds__(256) k_scale_signpack(
   const int64_t task = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (task >= d_out * (int64_t)nseg) return;
   const int64_t row = task / nseg;
-  const int seg = (int)(task % nseg);
+  const int seg = (int)(task - row * nseg);
 
-  ClipParams cp;
-  const bool do_clip = clipp != nullptr;
-  if (do_clip) cp = *clipp;
+  ClipF cp{0.f, 0.f, 0.f, 0.f};
+  if (CLIP) cp = load_clip(clipp);
 
-  const uint8_t* rb = wb + row * d_in * ESZ;
-  const uint8_t* rf = wf + row * d_in * ESZ;
-  const int64_t words_per_row = d_in >> 5;
-  uint32_t* srow = signs + row * words_per_row;
-  const int64_t col_seg0 = (int64_t)seg * seg_chunks * CHUNK;
+  const uint8_t* rb = wb + row * (int64_t)d_in * ESZ;
+  const uint8_t* rf = wf + row * (int64_t)d_in * ESZ;
+  uint32_t* srow = signs + row * (int64_t)(d_in >> 5);
+  const int G = 1 << lg;
+  float* srow_s = GROUP ? scales + row * (int64_t)(d_in >> lg) : nullptr;
+  const float invG = 1.0f / (float)G;  // exact: G is a power of two
+  const int lpg = G / VEC;              // lanes per group when G <= CHUNK
+  const int col_seg0 = seg * seg_chunks * CHUNK;
 
   double acc_row = 0.0;   // ROW / TENSOR: this lane's share of the segment sum
   double acc_grp = 0.0;   // GROUP with G > CHUNK: running group sum (all lanes equal)
@@ -250,49 +262,46 @@ __global__ void __launch_bounds__(256) k_scale_signpack(
     bool valid[SEGC];
 #pragma unroll
     for (int u = 0; u < SEGC; ++u) {
-      const int64_t col = col_seg0 + (int64_t)(c0 + u) * CHUNK + lane * VEC;
+      const int col = col_seg0 + (c0 + u) * CHUNK + lane * VEC;
       valid[u] = (c0 + u < seg_chunks) && col < d_in;
       if (valid[u]) {
-        b[u] = ldg_stream(rb + col * ESZ);
-        f[u] = ldg_stream(rf + col * ESZ);
+        b[u] = ldg_stream(rb + (int64_t)col * ESZ);
+        f[u] = ldg_stream(rf + (int64_t)col * ESZ);
       }
     }
 #pragma unroll
     for (int u = 0; u < SEGC; ++u) {
-      const int64_t chunk_col0 = col_seg0 + (int64_t)(c0 + u) * CHUNK;
+      const int chunk_col0 = col_seg0 + (c0 + u) * CHUNK;
       if (c0 + u >= seg_chunks || chunk_col0 >= d_in) break;  // warp-uniform
-      float d[VEC];
+      const int col = chunk_col0 + lane * VEC;
       uint32_t m = 0;
       float a = 0.f;
       if (valid[u]) {
+        float d[VEC];
         V::delta(b[u], f[u], d);
 #pragma unroll
         for (int k = 0; k < VEC; ++k) {
-          float dc = do_clip ? clamp_delta(d[k], cp) : d[k];
+          const float dc = CLIP ? clamp_delta(d[k], cp) : d[k];
           m |= (dc < 0.f ? 0u : 1u) << k;
           a += fabsf(dc);
         }
       }
       // pack: LPW lanes x VEC bits -> one word, lane order = column order (LSB first)
-      uint32_t v = m << (VEC * (lane % LPW));
+      uint32_t v = m << (VEC * (lane & (LPW - 1)));
 #pragma unroll
       for (int o = 1; o < LPW; o <<= 1) v |= __shfl_xor_sync(0xffffffffu, v, o);
-      if (valid[u] && (lane % LPW) == 0) srow[(chunk_col0 + lane * VEC) >> 5] = v;
+      if (valid[u] && (lane & (LPW - 1)) == 0) srow[col >> 5] = v;
 
-      if (mode == BD_SCALE_GROUP) {
-        if (group <= CHUNK) {
-          const int lpg = group / VEC;  // lanes per group (power of two, >= 4 / >= 8)
+      if (GROUP) {
+        if (G <= CHUNK) {
           float s = a;
           for (int o = 1; o < lpg; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-          if (valid[u] && (lane % lpg) == 0) {
-            const int64_t col = chunk_col0 + lane * VEC;
-            scales[row * (d_in / group) + col / group] = s / (float)group;
-          }
+          if (valid[u] && (lane & (lpg - 1)) == 0) srow_s[col >> lg] = s * invG;
         } else {
-          float s = warp_sum_f(a);
+          const float s = warp_sum_f(a);
           acc_grp += (double)s;
-          if (((chunk_col0 + CHUNK) % group) == 0 || chunk_col0 + CHUNK >= d_in) {
-            if (lane == 0) scales[row * (d_in / group) + chunk_col0 / group] = (float)(acc_grp / (double)group);
+          if (((chunk_col0 + CHUNK) & (G - 1)) == 0 || chunk_col0 + CHUNK >= d_in) {
+            if (lane == 0) srow_s[chunk_col0 >> lg] = (float)(acc_grp * (double)invG);
             acc_grp = 0.0;
           }
         }
@@ -301,7 +310,7 @@ __global__ void __launch_bounds__(256) k_scale_signpack(
       }
     }
   }
-  if (mode != BD_SCALE_GROUP) {
+  if (!GROUP) {
     acc_row = warp_sum_d(acc_row);
     if (lane == 0) partials[row * nseg + seg] = acc_row;
   }
@@ -329,22 +338,25 @@ __global__ void __launch_bounds__(256) k_col_scale_signpack(
   const int64_t chunk = task % nchunks;
   const int64_t col = chunk * CHUNK + lane * VEC;
   const bool valid = col < d_in;
-  ClipParams cp;
+  ClipF cp{0.f, 0.f, 0.f, 0.f};
   const bool do_clip = clipp != nullptr;
-  if (do_clip) cp = *clipp;
+  if (do_clip) cp = load_clip(clipp);
   double acc[VEC];
 #pragma unroll
   for (int k = 0; k < VEC; ++k) acc[k] = 0.0;
   const int64_t r0 = tile * tile_rows;
   const int64_t r1 = min(d_out, r0 + tile_rows);
   const int64_t words_per_row = d_in >> 5;
-  for (int64_t r = r0; r < r1; r += UR) {
+  const int64_t rstride = d_in * ESZ;
+  const uint8_t* pb = wb + (r0 * d_in + col) * ESZ;
+  const uint8_t* pf = wf + (r0 * d_in + col) * ESZ;
+  for (int64_t r = r0; r < r1; r += UR, pb += UR * rstride, pf += UR * rstride) {
     uint4 b[UR], f[UR];
 #pragma unroll
     for (int u = 0; u < UR; ++u) {
       if (valid && r + u < r1) {
-        b[u] = ldg_stream(wb + ((r + u) * d_in + col) * ESZ);
-        f[u] = ldg_stream(wf + ((r + u) * d_in + col) * ESZ);
+        b[u] = ldg_stream(pb + u * rstride);
+        f[u] = ldg_stream(pf + u * rstride);
       }
     }
 #pragma unroll
@@ -433,6 +445,7 @@ bd_status plan_compress(int32_t dtype, int64_t d_out, int64_t d_in, const bd_com
   if (!cfg) return BD_ERR_NULL;
   if (dtype != BD_F32 && dtype != BD_BF16) return BD_ERR_DTYPE;
   if (d_out < 1 || d_in < 32 || (d_in % 32) != 0) return BD_ERR_SHAPE;
+  if (d_in > ((int64_t)1 << 30) || d_out > ((int64_t)1 << 40)) return BD_ERR_SHAPE;
   if (cfg->mode < BD_SCALE_GROUP || cfg->mode > BD_SCALE_TENSOR) return BD_ERR_CONFIG;
   if (cfg->clip != 0 && cfg->clip != 1) return BD_ERR_CONFIG;
   if (cfg->clip && !(cfg->clip_k >= 0.0f)) return BD_ERR_CONFIG;
@@ -514,18 +527,26 @@ bd_status launch_compress(const CompressPlan& p, const void* w_base, const void*
     return BD_OK;
   }
   const int64_t tasks = d_out * (int64_t)p.nseg;
-  const int64_t blocks = (tasks + 7) / 8;
-  const int G = cfg->mode == BD_SCALE_GROUP ? cfg->group_size : 0;
+  const unsigned blocks = (unsigned)((tasks + 7) / 8);
+  const bool group = cfg->mode == BD_SCALE_GROUP;
+  int lg = 0;
+  if (group)
+    while ((1 << lg) < cfg->group_size) ++lg;
+  const bool clip = cfg->clip != 0;
+  const int din = (int)d_in;
+#define BD_SIGNPACK(SEGC, CLIP, GRP)                                                           \
+  k_scale_signpack<BF16, SEGC, CLIP, GRP><<<blocks, 256, 0, s>>>(                              \
+      (const uint8_t*)w_base, (const uint8_t*)w_fine, d_out, din, lg, p.seg_chunks, p.nseg,    \
+      clipp, signs, scales, part)
   launch_begin(K_SCALE_SIGNPACK, s);
   if (p.seg_chunks >= 4) {
-    k_scale_signpack<BF16, 4><<<(unsigned)blocks, 256, 0, s>>>(
-        (const uint8_t*)w_base, (const uint8_t*)w_fine, d_out, d_in, cfg->mode, G, p.seg_chunks,
-        p.nseg, clipp, signs, scales, part);
+    if (clip) { if (group) BD_SIGNPACK(4, true, true); else BD_SIGNPACK(4, true, false); }
+    else { if (group) BD_SIGNPACK(4, false, true); else BD_SIGNPACK(4, false, false); }
   } else {
-    k_scale_signpack<BF16, 2><<<(unsigned)blocks, 256, 0, s>>>(
-        (const uint8_t*)w_base, (const uint8_t*)w_fine, d_out, d_in, cfg->mode, G, p.seg_chunks,
-        p.nseg, clipp, signs, scales, part);
+    if (clip) { if (group) BD_SIGNPACK(2, true, true); else BD_SIGNPACK(2, true, false); }
+    else { if (group) BD_SIGNPACK(2, false, true); else BD_SIGNPACK(2, false, false); }
   }
+#undef BD_SIGNPACK
   launch_end(K_SCALE_SIGNPACK, s);
   BD_LAUNCH_CHECK();
   if (cfg->mode == BD_SCALE_ROW) {

@@ -25,6 +25,7 @@ enum KernelKind : int32_t {
   K_BASE_TC,             // tcgen05 base product (bf16, fp32 accumulation in TMEM)
   K_DELTA_LUT,           // per-tenant sign-LUT delta product + combine
   K_SELECT_FIXUP,        // compress: re-read of groups touched by the clip
+  K_PREPARE,             // re-tiling of a tenant into the serving layout
   K_KIND_COUNT
 };
 

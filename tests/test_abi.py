@@ -40,7 +40,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    for code in range(0, 11):
+    for code in range(0, 12):
         s = bd.status_string(code)
         assert s and s != "unknown status"
     assert bd.status_string(999) == "unknown status"

@@ -24,14 +24,22 @@ def bd():
     return m
 
 
-def _table(bd, tenants):
-    return bd.TenantTable([(dev(t["signs"]), dev(t["scales"]), t["mode"], t["group_size"])
-                           for t in tenants], "cuda")
+def _table(bd, tenants, layout=0):
+    """Device tenant table; layout 1 stores every tenant in the tiled serving layout
+    written by bd_prepare_tenant (the oracle always receives the row-major words)."""
+    recs = []
+    for t in tenants:
+        s, sc = dev(t["signs"]), dev(t["scales"])
+        if layout == 1:
+            d_out, wpr = t["signs"].shape
+            s, sc = bd.bd_prepare_tenant(s, sc, t["mode"], t["group_size"], d_out, wpr * 32)
+        recs.append((s, sc, t["mode"], t["group_size"], layout))
+    return bd.TenantTable(recs, "cuda")
 
 
-def _run(bd, wb, tenants, ids, x, y_dtype="bf16", w_dtype="bf16"):
+def _run(bd, wb, tenants, ids, x, y_dtype="bf16", w_dtype="bf16", layout=0):
     import torch
-    table = _table(bd, tenants)
+    table = _table(bd, tenants, layout)
     y, ws = bd.bd_apply_multi(dev(wb, w_dtype), table, dev(ids), dev(x, w_dtype),
                               y_dtype=torch.bfloat16 if y_dtype == "bf16" else torch.float32)
     rc, flags = bd.bd_get_status(ws)
@@ -76,34 +84,37 @@ def test_tiny_config_end_to_end(bd):
     assert_apply_close(host(y), y_ref, tol=1e-5, what="y (fp32 path, tight)")
 
 
+@pytest.mark.parametrize("layout", [0, 1])
 @pytest.mark.parametrize("B", [1, 4, 16, 63, 200, 300])
 @pytest.mark.parametrize("mode", [0, 1, 2, 3])
-def test_random_batches(bd, B, mode):
+def test_random_batches(bd, B, mode, layout):
     d_out, d_in = 384 + 8, 1024
     wb, tenants, ids, x = _problem(B * 10 + mode, d_out, d_in, B, 5, (mode,))
     ids[0] = -1  # base only
-    y, rc, _ = _run(bd, wb, tenants, ids, x)
+    y, rc, _ = _run(bd, wb, tenants, ids, x, layout=layout)
     assert rc == bd.BD_OK
     y_ref = O.apply_multi(wb, "bf16", tenants, ids, x, "bf16")
     assert_apply_close(y, y_ref)
 
 
+@pytest.mark.parametrize("layout", [0, 1])
 @pytest.mark.parametrize("mode", [0, 1, 2, 3])
-@pytest.mark.parametrize("d_out,d_in", [(1100, 544), (64, 4096), (2050, 256), (130, 96)])
-def test_delta_only_tight(bd, mode, d_out, d_in):
+@pytest.mark.parametrize("d_out,d_in", [(1100, 544), (64, 4096), (2050, 256), (130, 96), (600, 640)])
+def test_delta_only_tight(bd, mode, d_out, d_in, layout):
     """W_base = 0: the bound now constrains the delta product by itself; with fp32
     outputs it must also hold at 1e-5."""
     G = 32 if d_in % 128 else 128
     wb, tenants, ids, x = _problem(d_out + d_in + mode, d_out, d_in, 9, 3, (mode,), G=G,
                                    zero_base=True)
     y_ref = O.apply_multi(wb, "bf16", tenants, ids, x, "bf16")
-    y, rc, _ = _run(bd, wb, tenants, ids, x, y_dtype="f32")
+    y, rc, _ = _run(bd, wb, tenants, ids, x, y_dtype="f32", layout=layout)
     assert rc == bd.BD_OK
     assert_apply_close(y, y_ref)
     assert_apply_close(y, y_ref, tol=1e-5, what="delta only (fp32 out)")
 
 
-def test_mixed_modes_and_group_sizes(bd):
+@pytest.mark.parametrize("layout", [0, 1])
+def test_mixed_modes_and_group_sizes(bd, layout):
     rng = np.random.default_rng(12)
     d_out, d_in = 520, 2048
     wb = bf16_bits(rng.normal(0, 0.02, size=(d_out, d_in)))
@@ -112,7 +123,7 @@ def test_mixed_modes_and_group_sizes(bd):
     B = 40
     x = activations(rng, B, d_in)
     ids = rng.integers(-1, len(tenants), size=B).astype(np.int32)
-    y, rc, _ = _run(bd, wb, tenants, ids, x, y_dtype="f32")
+    y, rc, _ = _run(bd, wb, tenants, ids, x, y_dtype="f32", layout=layout)
     assert rc == bd.BD_OK
     assert_apply_close(y, O.apply_multi(wb, "bf16", tenants, ids, x, "bf16"), tol=1e-5)
 
@@ -189,7 +200,8 @@ def _sampled_rows_check(bd, d_out, d_in, tenants, ids, x, wb, rows, y):
     assert_apply_close(y[:, rows], y_ref)
 
 
-def test_decode_config_up_proj(bd):
+@pytest.mark.parametrize("layout", [0, 1])
+def test_decode_config_up_proj(bd, layout):
     """Decode GEMV at full size: up_proj 14336 x 4096 bf16 base, 64 resident tenants with
     group-128 fp16 scales, 64 tokens, one per tenant (a seeded permutation). Checked on
     256 sampled output rows plus full-tensor properties."""
@@ -199,7 +211,7 @@ def test_decode_config_up_proj(bd):
     tenants = [random_tenant(rng, d_out, d_in, 0, 128) for _ in range(T)]
     ids = rng.permutation(T).astype(np.int32)
     x = activations(rng, T, d_in)
-    y, rc, _ = _run(bd, wb, tenants, ids, x)
+    y, rc, _ = _run(bd, wb, tenants, ids, x, layout=layout)
     assert rc == bd.BD_OK
     rows = np.sort(rng.choice(d_out, 256, replace=False))
     _sampled_rows_check(bd, d_out, d_in, tenants, ids, x, wb, rows, y)
@@ -217,7 +229,7 @@ def test_mixed_config_layer(bd):
         wb = bf16_bits(rng.normal(0, 0.02, size=(d_out, d_in)))
         tenants = [random_tenant(rng, d_out, d_in, int(rng.integers(1, 3))) for _ in range(T)]
         x = activations(rng, B, d_in)
-        y, rc, _ = _run(bd, wb, tenants, ids, x)
+        y, rc, _ = _run(bd, wb, tenants, ids, x, layout=1)
         assert rc == bd.BD_OK, name
         rows = np.sort(rng.choice(d_out, 64, replace=False))
         _sampled_rows_check(bd, d_out, d_in, tenants, ids, x, wb, rows, y)
@@ -228,3 +240,34 @@ def test_launches_are_counted(bd):
     wb, tenants, ids, x = _problem(1, 128, 256, 4, 2, (0,))
     _run(bd, wb, tenants, ids, x)
     assert bd.bd_launch_count() - n0 == 3  # bucket, base product, delta
+
+
+@pytest.mark.parametrize("d_out,d_in,mode,G", [(1100, 640, 0, 128), (513, 544, 0, 32),
+                                               (300, 4096, 1, 128), (70, 256, 2, 128),
+                                               (9, 128, 3, 128), (1024, 4096, 0, 128)])
+@pytest.mark.parametrize("sdt", ["f16", "f32"])
+def test_prepare_tenant_layout(bd, d_out, d_in, mode, G, sdt):
+    """bd_prepare_tenant writes exactly the documented tiled layout: tile (rb, w) of
+    512 rows x 8 words at word offset (rb * ceil(d_in/256) + w) * 4096, zero padding;
+    group-128 scales tiled as [row][2] per tile; other scales copied unchanged."""
+    rng = np.random.default_rng(d_out + d_in + mode)
+    t = random_tenant(rng, d_out, d_in, mode, G, sdt)
+    s_t, sc_t = bd.bd_prepare_tenant(dev(t["signs"]), dev(t["scales"]), mode, G, d_out, d_in)
+    got_s, got_sc = host(s_t), host(sc_t)
+    nrt, nwin, wpr = -(-d_out // 512), -(-d_in // 256), d_in // 32
+    want = np.zeros((nrt, nwin, 512, 8), dtype=np.uint32)
+    for rb in range(nrt):
+        for w in range(nwin):
+            rows = t["signs"][rb * 512:(rb + 1) * 512, w * 8:min((w + 1) * 8, wpr)]
+            want[rb, w, :rows.shape[0], :rows.shape[1]] = rows
+    np.testing.assert_array_equal(got_s, want.reshape(-1))
+    sc = np.asarray(t["scales"])
+    if mode == 0 and G == 128:
+        ws = np.zeros((nrt, nwin, 512, 2), dtype=sc.dtype)
+        for rb in range(nrt):
+            for w in range(nwin):
+                blk = sc[rb * 512:(rb + 1) * 512, w * 2:min((w + 1) * 2, d_in // 128)]
+                ws[rb, w, :blk.shape[0], :blk.shape[1]] = blk
+        np.testing.assert_array_equal(got_sc.view(sc.dtype), ws.reshape(-1))
+    else:
+        np.testing.assert_array_equal(got_sc.view(sc.dtype)[:sc.size], sc.reshape(-1))
