@@ -11,6 +11,7 @@ static const char* const kKernelNames[K_KIND_COUNT] = {
     "delta_stats",       "stats_final",  "scale_signpack", "col_scale_signpack",
     "scale_final",       "reconstruct",  "tenant_bucket",  "base_gemv",
     "base_tc",           "delta_lut",    "select_fixup",   "prepare",
+    "tc_gather",         "delta_tc",
 };
 
 const char* kernel_name(int32_t kind) {

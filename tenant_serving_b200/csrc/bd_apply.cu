@@ -39,31 +39,53 @@ constexpr int kMaxTenants = 16384;
 constexpr int kMaxBatch = 65536;
 
 // ------------------------------------------------------------------------------------
-// token groups
+// planning: token groups for the lookup-table kernel, segments for the tensor-core one
 // ------------------------------------------------------------------------------------
-// Tokens are grouped by tenant (a counting sort) and every tenant's tokens are cut into
-// groups of at most kGroupTokens; one delta CTA serves one group for one block of rows.
-// Workspace layout (int32): [0] n_groups, [1..3] pad, then grp_tenant[max_groups],
-// grp_start[max_groups], grp_len[max_groups] (offsets into perm), perm[batch].
+// Tokens are grouped by tenant (a counting sort). A tenant with at least tc_min tokens
+// whose record the tensor-core path supports gets tensor-core segments of <= 128 tokens;
+// every other tenant's tokens (and the base-only tokens) are cut into lookup-table groups
+// of <= kGroupTokens.
+// Workspace layout (int32): [0] n_groups, [1] n_tc, [2..3] pad, grp_tenant[max_groups],
+// grp_start[max_groups], grp_len[max_groups], tc_tenant[max_tc], tc_start[max_tc],
+// tc_count[max_tc], tc_xrow[max_tc] (first row in the gathered X), perm[batch]; and, in
+// a region of its own, a copy of each tensor-core segment's tenant record.
 constexpr int kGroupTokens = 2;
+constexpr int kTcMaxTokens = 128;
 
 inline int max_groups_for(int64_t batch, int32_t n_tenants) {
   const int64_t keys = batch < (int64_t)n_tenants + 1 ? batch : (int64_t)n_tenants + 1;
   return (int)((batch + kGroupTokens - 1) / kGroupTokens + keys);
 }
 
+__device__ __forceinline__ bool tc_eligible(const bd_tenant& T, int64_t d_in) {
+  const bool mode_ok = (T.mode == BD_SCALE_GROUP && T.group_size >= 64 &&
+                        (T.group_size & (T.group_size - 1)) == 0 && (d_in % T.group_size) == 0) ||
+                       T.mode == BD_SCALE_ROW || T.mode == BD_SCALE_TENSOR;
+  const bool ptr_ok = T.signs != nullptr && T.scales != nullptr &&
+                      ((reinterpret_cast<uintptr_t>(T.signs) | reinterpret_cast<uintptr_t>(T.scales)) & 15u) == 0;
+  // the tensor-core kernel streams whole tiles of the serving layout
+  return mode_ok && ptr_ok && T.layout == BD_LAYOUT_TILED && T.reserved == 0;
+}
+
 __global__ void __launch_bounds__(1024) k_tenant_bucket(const int32_t* __restrict__ ids, int batch,
-                                                        int n_tenants, int max_groups,
+                                                        int n_tenants, int max_groups, int max_tc,
+                                                        const bd_tenant* __restrict__ tenants,
+                                                        int tc_min, int64_t d_in,
                                                         int32_t* __restrict__ seg_base,
+                                                        bd_tenant* __restrict__ tc_rec,
                                                         uint32_t* __restrict__ status) {
   extern __shared__ int32_t cnt[];  // n_tenants + 1 counters (last = base only)
-  __shared__ int32_t warp_tot[32], warp_grp[32];
+  __shared__ int32_t wsum[4][32];
   __shared__ int32_t bad;
   const int nkeys = n_tenants + 1;
   int32_t* grp_tenant = seg_base + 4;
   int32_t* grp_start = grp_tenant + max_groups;
   int32_t* grp_len = grp_start + max_groups;
-  int32_t* perm = grp_len + max_groups;
+  int32_t* tc_tenant = grp_len + max_groups;
+  int32_t* tc_start = tc_tenant + max_tc;
+  int32_t* tc_count = tc_start + max_tc;
+  int32_t* tc_xrow = tc_count + max_tc;
+  int32_t* perm = tc_xrow + max_tc;
   if (threadIdx.x == 0) {
     status[0] = 0;  // the status word reports this call
     bad = 0;
@@ -79,60 +101,92 @@ __global__ void __launch_bounds__(1024) k_tenant_bucket(const int32_t* __restric
     atomicAdd(&cnt[u < 0 ? n_tenants : u], 1);
   }
   __syncthreads();
-  // exclusive scans of token counts and of group counts, contiguous keys per thread
+  // per key: tokens, lookup groups, tensor-core segments, gathered-X rows
+  auto plan = [&](int k, int c, int& ng, int& nt, int& nx) {
+    ng = nt = nx = 0;
+    if (c == 0) return;
+    const bool tc = max_tc > 0 && k < n_tenants && c >= tc_min && tc_eligible(tenants[k], d_in);
+    if (tc) {
+      nt = (c + kTcMaxTokens - 1) / kTcMaxTokens;
+      for (int j = 0; j < c; j += kTcMaxTokens) nx += (min(kTcMaxTokens, c - j) + 15) & ~15;
+    } else {
+      ng = (c + kGroupTokens - 1) / kGroupTokens;
+    }
+  };
   const int per = (nkeys + blockDim.x - 1) / blockDim.x;
   const int k0 = threadIdx.x * per, k1 = min(nkeys, k0 + per);
-  int tot = 0, ng = 0;
+  int v[4] = {0, 0, 0, 0};  // tokens, groups, tc segments, X rows
   for (int k = k0; k < k1; ++k) {
-    tot += cnt[k];
-    ng += (cnt[k] + kGroupTokens - 1) / kGroupTokens;
+    int ng, nt, nx;
+    plan(k, cnt[k], ng, nt, nx);
+    v[0] += cnt[k];
+    v[1] += ng;
+    v[2] += nt;
+    v[3] += nx;
   }
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  int itot = tot, ing = ng;
+  int inc[4] = {v[0], v[1], v[2], v[3]};
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    int a = __shfl_up_sync(0xffffffffu, itot, o), b = __shfl_up_sync(0xffffffffu, ing, o);
-    if (lane >= o) {
-      itot += a;
-      ing += b;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int a = __shfl_up_sync(0xffffffffu, inc[i], o);
+      if (lane >= o) inc[i] += a;
     }
   }
   if (lane == 31) {
-    warp_tot[w] = itot;
-    warp_grp[w] = ing;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) wsum[i][w] = inc[i];
   }
   __syncthreads();
   if (w == 0) {
     const int nw = blockDim.x >> 5;
-    int a = lane < nw ? warp_tot[lane] : 0, b = lane < nw ? warp_grp[lane] : 0;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      int c = __shfl_up_sync(0xffffffffu, a, o), d = __shfl_up_sync(0xffffffffu, b, o);
-      if (lane >= o) {
-        a += c;
-        b += d;
+    for (int i = 0; i < 4; ++i) {
+      int a = lane < nw ? wsum[i][lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int c = __shfl_up_sync(0xffffffffu, a, o);
+        if (lane >= o) a += c;
       }
-    }
-    if (lane < nw) {
-      warp_tot[lane] = a;
-      warp_grp[lane] = b;
+      if (lane < nw) wsum[i][lane] = a;
     }
   }
   __syncthreads();
-  int off = itot - tot + (w > 0 ? warp_tot[w - 1] : 0);
-  int gidx = ing - ng + (w > 0 ? warp_grp[w - 1] : 0);
+  int off = inc[0] - v[0] + (w > 0 ? wsum[0][w - 1] : 0);
+  int gidx = inc[1] - v[1] + (w > 0 ? wsum[1][w - 1] : 0);
+  int tidx = inc[2] - v[2] + (w > 0 ? wsum[2][w - 1] : 0);
+  int xrow = inc[3] - v[3] + (w > 0 ? wsum[3][w - 1] : 0);
   for (int k = k0; k < k1; ++k) {
     const int c = cnt[k];
-    for (int j = 0; j < c; j += kGroupTokens) {
-      grp_tenant[gidx] = (k == n_tenants) ? -1 : k;
-      grp_start[gidx] = off + j;
-      grp_len[gidx] = min(kGroupTokens, c - j);
-      ++gidx;
+    int ng, nt, nx;
+    plan(k, c, ng, nt, nx);
+    if (nt > 0) {
+      for (int j = 0; j < c; j += kTcMaxTokens) {
+        const int n = min(kTcMaxTokens, c - j);
+        tc_tenant[tidx] = k;
+        tc_rec[tidx] = tenants[k];
+        tc_start[tidx] = off + j;
+        tc_count[tidx] = n;
+        tc_xrow[tidx] = xrow;
+        xrow += (n + 15) & ~15;
+        ++tidx;
+      }
+    } else {
+      for (int j = 0; j < c; j += kGroupTokens) {
+        grp_tenant[gidx] = (k == n_tenants) ? -1 : k;
+        grp_start[gidx] = off + j;
+        grp_len[gidx] = min(kGroupTokens, c - j);
+        ++gidx;
+      }
     }
     cnt[k] = off;  // becomes the scatter cursor
     off += c;
   }
-  if (threadIdx.x == blockDim.x - 1) seg_base[0] = gidx;  // last thread holds the total
+  if (threadIdx.x == blockDim.x - 1) {  // the last thread holds the totals
+    seg_base[0] = gidx;
+    seg_base[1] = tidx;
+  }
   __syncthreads();
   for (int t = threadIdx.x; t < batch; t += blockDim.x) {
     int u = ids[t];
@@ -585,8 +639,8 @@ __device__ __forceinline__ void lut_lane_constants(int q, int wp, uint32_t (&sel
 template <bool XBF16>
 __global__ void __launch_bounds__(LUT_THREADS, 1) k_delta_lut(
     const bd_tenant* __restrict__ tenants, bool scale_f16, const int32_t* __restrict__ seg_base,
-    int max_groups, const void* __restrict__ x, const float* __restrict__ y_part, int ksplit,
-    int64_t d_out, int64_t d_in, int batch, void* __restrict__ y, bool y_bf16,
+    int max_groups, int max_tc, const void* __restrict__ x, const float* __restrict__ y_part,
+    int ksplit, int64_t d_out, int64_t d_in, int batch, void* __restrict__ y, bool y_bf16,
     uint32_t* __restrict__ status) {
   extern __shared__ __align__(16) uint8_t smem[];
   const uint32_t base = sh_addr(smem);
@@ -600,7 +654,7 @@ __global__ void __launch_bounds__(LUT_THREADS, 1) k_delta_lut(
   const int32_t* grp_tenant = seg_base + 4;
   const int32_t* grp_start = grp_tenant + max_groups;
   const int32_t* grp_len = grp_start + max_groups;
-  const int32_t* perm = grp_len + max_groups;
+  const int32_t* perm = grp_len + max_groups + 4 * max_tc;
   // the (token group, 512-row tile) space is split evenly over the CTAs; a piece is up to
   // LUT_NSB consecutive tiles of one group
   const int n_groups = seg_base[0];
@@ -735,18 +789,41 @@ __global__ void __launch_bounds__(LUT_THREADS, 1) k_delta_lut(
 // ------------------------------------------------------------------------------------
 // host side
 // ------------------------------------------------------------------------------------
+bd_status launch_delta_tc(const bd_tenant* tenants, const int32_t* seg, int max_groups, int max_tc,
+                          const void* x, int64_t d_out, int64_t d_in, int64_t batch, __half* xg,
+                          int64_t xg_rows, float* xinv, const float* y_part, int ksplit, void* y,
+                          bool y_bf16, uint32_t* status, cudaStream_t s);
+
+// A tenant with at least this many tokens in a batch (and a supported record) goes to the
+// tensor-core delta kernel; below it the lookup-table kernel is cheaper per token.
+#ifndef BD_TC_MIN_TOKENS
+#define BD_TC_MIN_TOKENS 8
+#endif
+constexpr int kTcMinTokens = BD_TC_MIN_TOKENS;
+
 namespace {
 struct ApplyLayout {
-  int max_groups;
+  int max_groups, max_tc;
   TcPlan tc;
   int ksplit;
-  size_t off_seg, off_part, total;
+  int64_t xg_rows;
+  size_t off_seg, off_tcrec, off_part, off_xg, off_xinv, total;
 };
 
-ApplyLayout layout_apply(int64_t d_out, int64_t d_in, int64_t batch, int32_t n_tenants, bool tc) {
+ApplyLayout layout_apply(int64_t d_out, int64_t d_in, int64_t batch, int32_t n_tenants, bool tc,
+                         bool tc_delta) {
   ApplyLayout L;
   L.max_groups = max_groups_for(batch, n_tenants);
   if (L.max_groups < 1) L.max_groups = 1;
+  // a batch smaller than the many-token threshold has no tensor-core segment at all
+  if (tc_delta && batch >= kTcMinTokens) {
+    // segments: at most one per many-token tenant plus one per extra 128 tokens
+    int64_t by_tokens = batch / kTcMinTokens, by_tenants = n_tenants;
+    L.max_tc = (int)((by_tokens < by_tenants ? by_tokens : by_tenants) + batch / kTcMaxTokens + 1);
+  } else {
+    L.max_tc = 0;
+  }
+  L.xg_rows = tc_delta ? batch + 15 * (int64_t)L.max_tc : 0;
   L.ksplit = 1;
   if (tc) {
     L.tc = plan_base_tc(d_out, d_in, batch);
@@ -754,18 +831,25 @@ ApplyLayout layout_apply(int64_t d_out, int64_t d_in, int64_t batch, int32_t n_t
   }
   size_t off = kStatusBytes;
   L.off_seg = off;
-  off = align_up(off + (16 + 3 * (size_t)L.max_groups * 4 + (size_t)batch * 4), 256);
+  off = align_up(off + (16 + 3 * (size_t)L.max_groups * 4 + 4 * (size_t)L.max_tc * 4 + (size_t)batch * 4), 256);
+  L.off_tcrec = off;
+  off = align_up(off + (size_t)L.max_tc * sizeof(bd_tenant), 256);
   L.off_part = off;
   off = align_up(off + (size_t)L.ksplit * batch * d_out * sizeof(float), 256);
+  L.off_xg = off;
+  off = align_up(off + (size_t)L.xg_rows * d_in * 2, 256);
+  L.off_xinv = off;
+  off = align_up(off + (size_t)L.xg_rows * sizeof(float), 256);
   L.total = off;
   return L;
 }
+
 }  // namespace
 
 size_t apply_workspace_size(int64_t d_out, int64_t d_in, int64_t batch, int32_t n_tenants) {
   if (d_out < 1 || d_in < 32 || batch < 0 || n_tenants < 0) return 0;
-  const size_t a = layout_apply(d_out, d_in, batch, n_tenants, true).total;
-  const size_t b = layout_apply(d_out, d_in, batch, n_tenants, false).total;
+  const size_t a = layout_apply(d_out, d_in, batch, n_tenants, true, (d_in % 64) == 0).total;
+  const size_t b = layout_apply(d_out, d_in, batch, n_tenants, false, false).total;
   return a > b ? a : b;
 }
 
@@ -785,7 +869,9 @@ bd_status apply_impl(const void* w_base, int32_t w_dtype, int64_t d_out, int64_t
       (tenants && (reinterpret_cast<uintptr_t>(tenants) & 7u)))
     return BD_ERR_ALIGN;
   const bool tc = w_dtype == BD_BF16;
-  ApplyLayout L = layout_apply(d_out, d_in, batch, n_tenants, tc);
+  // the tensor-core delta path needs bf16 activations, fp16 scales and 64-column stages
+  const bool tc_delta = tc && scale_dtype == BD_F16 && (d_in % 64) == 0;
+  ApplyLayout L = layout_apply(d_out, d_in, batch, n_tenants, tc, tc_delta);
   if (!workspace || ws_bytes < L.total) return BD_ERR_WORKSPACE;
   if (!aligned16(workspace)) return BD_ERR_ALIGN;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -806,7 +892,8 @@ bd_status apply_impl(const void* w_base, int32_t w_dtype, int64_t d_out, int64_t
   }
   launch_begin(K_TENANT_BUCKET, s);
   k_tenant_bucket<<<1, 1024, bucket_smem, s>>>(tenant_ids, (int)batch, n_tenants, L.max_groups,
-                                               seg, status);
+                                               L.max_tc, tenants, kTcMinTokens, d_in, seg,
+                                               reinterpret_cast<bd_tenant*>(ws + L.off_tcrec), status);
   launch_end(K_TENANT_BUCKET, s);
   BD_LAUNCH_CHECK();
 
@@ -823,7 +910,17 @@ bd_status apply_impl(const void* w_base, int32_t w_dtype, int64_t d_out, int64_t
     BD_LAUNCH_CHECK();
   }
 
-  // 3. delta product over the (token group, row) space, fused with the combine
+  // 3. tensor-core delta for the many-token tenants, fused with the combine
+  if (L.max_tc > 0) {
+    bd_status st = launch_delta_tc(reinterpret_cast<const bd_tenant*>(ws + L.off_tcrec), seg,
+                                   L.max_groups, L.max_tc, x, d_out, d_in, batch,
+                                   reinterpret_cast<__half*>(ws + L.off_xg), L.xg_rows,
+                                   reinterpret_cast<float*>(ws + L.off_xinv), y_part, L.ksplit, y,
+                                   y_dtype == BD_BF16, status, s);
+    if (st != BD_OK) return st;
+  }
+
+  // 4. lookup-table delta over the (token group, row) space, fused with the combine
   auto kfn = tc ? k_delta_lut<true> : k_delta_lut<false>;
   static bool lut_attr[2] = {false, false};
   if (!lut_attr[tc ? 1 : 0]) {
@@ -836,9 +933,9 @@ bd_status apply_impl(const void* w_base, int32_t w_dtype, int64_t d_out, int64_t
   }
   launch_begin(K_DELTA_LUT, s);
   kfn<<<(unsigned)sm_count(), LUT_THREADS, LUT_SMEM, s>>>(tenants, scale_dtype == BD_F16, seg,
-                                                         L.max_groups, x, y_part, L.ksplit, d_out,
-                                                         d_in, (int)batch, y, y_dtype == BD_BF16,
-                                                         status);
+                                                         L.max_groups, L.max_tc, x, y_part, L.ksplit,
+                                                         d_out, d_in, (int)batch, y,
+                                                         y_dtype == BD_BF16, status);
   launch_end(K_DELTA_LUT, s);
   BD_LAUNCH_CHECK();
   return BD_OK;

@@ -26,6 +26,8 @@ enum KernelKind : int32_t {
   K_DELTA_LUT,           // per-tenant sign-LUT delta product + combine
   K_SELECT_FIXUP,        // compress: re-read of groups touched by the clip
   K_PREPARE,             // re-tiling of a tenant into the serving layout
+  K_TC_GATHER,           // gather + fp16 scaling of the tensor-core segments' tokens
+  K_DELTA_TC,            // tcgen05 delta product of many-token tenants + combine
   K_KIND_COUNT
 };
 
