@@ -43,6 +43,7 @@ N_TENANTS = 100
 BATCH = 512
 GROUP = 128
 ZIPF_S = 1.1
+TC_MIN_TOKENS = 8  # the library's many-token threshold (tensor-core delta from this count on)
 
 
 def parse():
@@ -62,11 +63,13 @@ def parse():
 
 
 def load_peaks():
+    """(HBM GB/s, (bf16 TFLOP/s burst, sustained), source)."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
         d = json.load(open(path))
-        return d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0), "measured"
-    return 6650.0, 1590.0, "fallback"
+        return (d.get("hbm_gbs", 6650.0),
+                (d.get("bf16_tflops", 1590.0), d.get("bf16_tflops_sustained", 1400.0)), "measured")
+    return 6650.0, (1590.0, 1400.0), "fallback"
 
 
 # ------------------------------------------------------------------------------------
@@ -263,7 +266,7 @@ def bench_serving(args, rank, pg, log, peaks):
     clocks.start()
     time.sleep(0.3)
     n0 = bd.bd_launch_count()
-    bd.bd_profile_enable(True, capacity=args.steps * len(step_calls[0]) * 4 + 16)
+    bd.bd_profile_enable(True, capacity=args.steps * len(step_calls[0]) * 8 + 16)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
@@ -290,16 +293,33 @@ def bench_serving(args, rank, pg, log, peaks):
     torch.cuda.synchronize()
     ms_plain = max_over_ranks(pg, f0.elapsed_time(f1))
 
-    # algorithmic bytes of the timed steps
+    # algorithmic bytes of the timed steps. The planner sends a tenant with at least
+    # TC_MIN_TOKENS tokens in the batch (all tenants here are tiled, fp16, group 128) to the
+    # tensor-core delta kernel and the others to the lookup-table kernel; each delta kernel
+    # is charged the sign words + scales of its tenants and the y rows of its tokens.
     base_bytes = sum(d_out * d_in * 2 for _, d_out, d_in in LLAMA3_8B_PROJECTIONS) * args.layers
+    base_flops_per_token = sum(2 * d_out * d_in for _, d_out, d_in in LLAMA3_8B_PROJECTIONS) * args.layers
     delta_bytes_per_tenant = sum(d_out * d_in // 8 + d_out * (d_in // GROUP) * 2
                                  for _, d_out, d_in in LLAMA3_8B_PROJECTIONS) * args.layers
-    io_bytes = sum(B * d_in * 2 + B * d_out * 2 for _, d_out, d_in in LLAMA3_8B_PROJECTIONS) * args.layers
+    y_bytes_per_token = sum(d_out * 2 for _, d_out, _ in LLAMA3_8B_PROJECTIONS) * args.layers
+    x_bytes_per_token = sum(d_in * 2 for _, _, d_in in LLAMA3_8B_PROJECTIONS) * args.layers
+    io_bytes = B * (x_bytes_per_token + y_bytes_per_token)
+    step_bytes, lut_bytes, tc_bytes = [], 0.0, 0.0
+    for s in range(args.warmup, steps_total):
+        cnt = np.bincount(ids_host[s], minlength=args.tenants)
+        d = int((cnt > 0).sum())
+        big = cnt >= TC_MIN_TOKENS
+        step_bytes.append(base_bytes + d * delta_bytes_per_tenant + io_bytes)
+        tc_bytes += int(big.sum()) * delta_bytes_per_tenant + int(cnt[big].sum()) * y_bytes_per_token
+        small = (cnt > 0) & ~big
+        lut_bytes += int(small.sum()) * delta_bytes_per_tenant + int(cnt[small].sum()) * y_bytes_per_token
     distinct = [len(np.unique(ids_host[s])) for s in range(args.warmup, steps_total)]
-    step_bytes = [base_bytes + d * delta_bytes_per_tenant + io_bytes for d in distinct]
     total_bytes = float(sum(step_bytes))
-    delta_kernel_bytes = float(sum(d * delta_bytes_per_tenant for d in distinct)) + \
-        args.steps * args.layers * sum(B * d_out * 2 for _, d_out, _ in LLAMA3_8B_PROJECTIONS)
+    kernel_work = {  # kernel -> (amount over the timed steps, unit, bound)
+        "delta_lut": (lut_bytes, "GB/s", "hbm"),
+        "delta_tc": (tc_bytes, "GB/s", "hbm"),
+        "base_tc": (float(base_flops_per_token) * B * args.steps, "TFLOP/s", "tensor"),
+    }
 
     # e2e through the public API: H2D of this step's inputs (pinned), the 224 calls,
     # D2H of the last projection's output
@@ -334,11 +354,13 @@ def bench_serving(args, rank, pg, log, peaks):
     # dominant kernel by total device time
     dom = max(prof.items(), key=lambda kv: kv[1][1]) if prof else ("delta_lut", (0, 0.0))
     dname, (dl, dms) = dom
-    dom_bytes = delta_kernel_bytes if dname == "delta_lut" else None
-    if dname == "base_tc":
-        dom_bytes = float(base_bytes) * args.steps
-    achieved = dom_bytes / (dms / 1e3) / 1e9 if dom_bytes and dms > 0 else None
-    hbm_peak, _, peak_src = peaks
+    hbm_peak, tensor_peaks, peak_src = peaks
+    work, unit, bound = kernel_work.get(dname, (None, "GB/s", "hbm"))
+    achieved = None
+    if work and dms > 0:
+        achieved = work / (dms / 1e3) / (1e12 if unit == "TFLOP/s" else 1e9)
+    # a kernel timed inside a long step: the sustained tensor peak
+    peak = tensor_peaks[1] if unit == "TFLOP/s" else hbm_peak
     res = {
         "value": value, "ms_per_step": ms_max / args.steps, "ms_per_step_unprofiled": ms_plain / args.steps,
         "hbm_gbs": hbm_gbs, "hbm_frac": hbm_gbs / hbm_peak, "gpu_launches": launches,
@@ -347,10 +369,16 @@ def bench_serving(args, rank, pg, log, peaks):
                 "d2h_bytes_per_step": d2h},
         "kernels": {k: {"launches": v[0], "total_ms": v[1], "share": v[1] / sum(x[1] for x in prof.values())}
                     for k, v in prof.items()},
-        "roofline": {"kernel": dname, "bound": "hbm", "achieved": achieved, "peak": hbm_peak,
-                     "unit": "GB/s", "frac": (achieved / hbm_peak) if achieved else None,
-                     "traffic": None, "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)",
+        "roofline": {"kernel": dname, "bound": bound, "achieved": achieved, "peak": peak,
+                     "unit": unit, "frac": (achieved / peak) if achieved else None,
+                     "traffic": None,
+                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json "
+                                    f"{'bf16_tflops_sustained' if unit == 'TFLOP/s' else 'hbm_gbs'})",
                      "avg_launch_us": dms / dl * 1e3 if dl else None},
+        "kernel_rates": {k: {"achieved": kernel_work[k][0] / (prof[k][1] / 1e3) /
+                                         (1e12 if kernel_work[k][1] == "TFLOP/s" else 1e9),
+                             "unit": kernel_work[k][1]}
+                         for k in kernel_work if k in prof and prof[k][1] > 0},
         "step_bytes_mean": float(np.mean(step_bytes)),
     }
     del layers
@@ -390,10 +418,10 @@ def bench_compress(args, log, peaks):
         for _ in range(2):
             one_pass()
         torch.cuda.synchronize()
-        bd.bd_profile_enable(True, capacity=len(mats) * 8 + 16)
+        reps = 3
+        bd.bd_profile_enable(True, capacity=len(mats) * reps * 8 + 16)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
-        reps = 3
         e0.record()
         for _ in range(reps):
             one_pass()

@@ -761,25 +761,47 @@ __global__ void __launch_bounds__(LUT_THREADS, 1) k_delta_lut(
     }
     __syncthreads();
     // ---- combine with the base product, write y in request order
+    // each thread owns up to LUT_RPT rows x 2 tokens; the split-K partials of all of them
+    // are loaded together (independent loads) before any is added
+    constexpr int LUT_RPT = (LUT_PASS + LUT_THREADS - 1) / LUT_THREADS;
     float rs = 1.f;
     if (P.u >= 0 && P.mode == BD_SCALE_TENSOR) rs = ld_scale(P.T.scales, scale_f16, 0);
-    for (int tt = 0; tt < P.ntok; ++tt) {
+    float bsum[2][LUT_RPT];
+#pragma unroll
+    for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+      for (int k = 0; k < LUT_RPT; ++k) bsum[tt][k] = 0.f;
+    for (int kz = 0; kz < ksplit; ++kz) {
+      const float* part = y_part + (int64_t)kz * batch * d_out + P.r0 + tid;
+#pragma unroll
+      for (int tt = 0; tt < 2; ++tt) {
+        const int t = tt == 0 ? P.t0 : P.t1;
+#pragma unroll
+        for (int k = 0; k < LUT_RPT; ++k)
+          if (tt < P.ntok && tid + k * LUT_THREADS < P.rows)
+            bsum[tt][k] += part[(int64_t)t * d_out + k * LUT_THREADS];
+      }
+    }
+#pragma unroll
+    for (int tt = 0; tt < 2; ++tt) {
       const int t = tt == 0 ? P.t0 : P.t1;
-      for (int rl = tid; rl < P.rows; rl += LUT_THREADS) {
-        const int64_t row = P.r0 + rl;
-        float bsum = 0.f;
-        for (int kz = 0; kz < ksplit; ++kz) bsum += y_part[((int64_t)kz * batch + t) * d_out + row];
-        float d = 0.f;
-        if (P.u >= 0) {
-          float sc = rs;
-          if (P.mode == BD_SCALE_ROW) sc = ld_scale(P.T.scales, scale_f16, row);
-          d = sc * out_s[tt * LUT_PASS + rl];
+#pragma unroll
+      for (int k = 0; k < LUT_RPT; ++k) {
+        const int rl = tid + k * LUT_THREADS;
+        if (tt < P.ntok && rl < P.rows) {
+          const int64_t row = P.r0 + rl;
+          float d = 0.f;
+          if (P.u >= 0) {
+            float sc = rs;
+            if (P.mode == BD_SCALE_ROW) sc = ld_scale(P.T.scales, scale_f16, row);
+            d = sc * out_s[tt * LUT_PASS + rl];
+          }
+          const float v = bsum[tt][k] + d;
+          if (y_bf16)
+            reinterpret_cast<uint16_t*>(y)[(int64_t)t * d_out + row] = (uint16_t)f2bf_bits(v);
+          else
+            reinterpret_cast<float*>(y)[(int64_t)t * d_out + row] = v;
         }
-        const float v = bsum + d;
-        if (y_bf16)
-          reinterpret_cast<uint16_t*>(y)[(int64_t)t * d_out + row] = (uint16_t)f2bf_bits(v);
-        else
-          reinterpret_cast<float*>(y)[(int64_t)t * d_out + row] = v;
       }
     }
     __syncthreads();

@@ -154,6 +154,17 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* v) {
       "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
       : "memory");
 }
+// 32 lanes x 16 consecutive 32-bit columns of tensor memory into 16 registers per thread.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -403,22 +414,34 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_delta_tc(
       const int npad = (cur.count + 15) & ~15;
       const uint32_t lane_addr =
           tmem_base + (uint32_t)ab * DT_ACC_STRIDE + ((uint32_t)(q4 * 32) << 16);
-      for (int c0 = 0; c0 < npad; c0 += 32) {
-        uint32_t rr[32];
-        tmem_ld32(lane_addr + (uint32_t)c0, rr);
+      for (int c0 = 0; c0 < npad; c0 += 16) {
+        uint32_t rr[16];
+        tmem_ld16(lane_addr + (uint32_t)c0, rr);
         if (row < d_out) {
+          // 16 tokens at a time: token ids and 2^-e first, then every split-K partial of
+          // all 16 outputs as independent loads, then the stores
+          int tok[16];
+          float v[16];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
+          for (int j = 0; j < 16; ++j) {
             const int c = c0 + j;
-            if (c < cur.count) {
-              const int t = sg.perm[cur.start + c];
-              float base = 0.f;
-              for (int kz = 0; kz < ksplit; ++kz) base += y_part[((int64_t)kz * batch + t) * d_out + row];
-              const float v = base + __uint_as_float(rr[j]) * xinv[cur.xrow + c];
+            const bool ok = c < cur.count;
+            tok[j] = ok ? sg.perm[cur.start + c] : 0;
+            v[j] = ok ? __uint_as_float(rr[j]) * xinv[cur.xrow + c] : 0.f;
+          }
+          for (int kz = 0; kz < ksplit; ++kz) {
+            const float* part = y_part + (int64_t)kz * batch * d_out + row;
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              if (c0 + j < cur.count) v[j] += part[(int64_t)tok[j] * d_out];
+          }
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            if (c0 + j < cur.count) {
               if (y_bf16)
-                reinterpret_cast<uint16_t*>(y)[(int64_t)t * d_out + row] = (uint16_t)f2bf_bits(v);
+                reinterpret_cast<uint16_t*>(y)[(int64_t)tok[j] * d_out + row] = (uint16_t)f2bf_bits(v[j]);
               else
-                reinterpret_cast<float*>(y)[(int64_t)t * d_out + row] = v;
+                reinterpret_cast<float*>(y)[(int64_t)tok[j] * d_out + row] = v[j];
             }
           }
         }
