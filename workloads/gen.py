@@ -27,7 +27,7 @@ import math
 import numpy as np
 
 __all__ = [
-    "LLAMA3_8B_PROJECTIONS",
+    "LLAMA3_8B_PROJECTIONS", "LLAMA3_8B_FUSED",
     "bf16_bits",
     "bf16_bits_to_f32",
     "weight_pair",
@@ -49,6 +49,16 @@ LLAMA3_8B_PROJECTIONS = (
     ("o", 4096, 4096),
     ("gate", 14336, 4096),
     ("up", 14336, 4096),
+    ("down", 4096, 14336),
+)
+
+# The same layer as serving engines apply it: projections that read the same input are
+# stacked along d_out (q | k | v and gate | up), so a layer is 4 products instead of 7
+# with identical rows, columns, weights and outputs.
+LLAMA3_8B_FUSED = (
+    ("qkv", 6144, 4096),
+    ("o", 4096, 4096),
+    ("gate_up", 28672, 4096),
     ("down", 4096, 14336),
 )
 
