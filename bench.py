@@ -131,17 +131,23 @@ class ClockSampler:
 # our arm
 # ------------------------------------------------------------------------------------
 def setup_dist(args):
+    """One process per GPU under torch.distributed.run (RANK / WORLD_SIZE / LOCAL_RANK /
+    MASTER_* from the environment). NCCL on GPUs; gloo where there is no GPU (the rank
+    logic's CPU tests). The group's short timeout turns a missing rank into an error."""
+    import datetime
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
+    on_gpu = torch.cuda.is_available()
+    if on_gpu:
+        torch.cuda.set_device(local)
     pg = None
     if world > 1:
-        import datetime
         import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
-                                device_id=torch.device("cuda", local))
+        kw = {"device_id": torch.device("cuda", local)} if on_gpu else {}
+        dist.init_process_group("nccl" if on_gpu else "gloo",
+                                timeout=datetime.timedelta(seconds=120), **kw)
         pg = dist
     return world, rank, local, pg
 
@@ -151,22 +157,37 @@ def barrier(pg):
         pg.barrier()
 
 
-def max_over_ranks(pg, v: float) -> float:
-    if pg is None:
-        return v
+def _reduce(pg, v: float, op) -> float:
     import torch
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    dev = "cuda" if pg.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    pg.all_reduce(t, op=op)
     return float(t.item())
+
+
+def max_over_ranks(pg, v: float) -> float:
+    return v if pg is None else _reduce(pg, v, pg.ReduceOp.MAX)
 
 
 def sum_over_ranks(pg, v: float) -> float:
-    if pg is None:
-        return v
-    import torch
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    pg.all_reduce(t, op=pg.ReduceOp.SUM)
-    return float(t.item())
+    return v if pg is None else _reduce(pg, v, pg.ReduceOp.SUM)
+
+
+def whole_job_rate(pg, units: float, ms: float):
+    """Units of all ranks / the slowest rank's time: (units_all, ms_max, units per s)."""
+    units_all = sum_over_ranks(pg, units)
+    ms_max = max_over_ranks(pg, ms)
+    return units_all, ms_max, units_all / (ms_max / 1e3)
+
+
+def serving_config(args, world: int) -> dict:
+    return {"workload": "serving: 32-layer Llama-3-8B-shaped projection stack "
+                        "(q, k, v, o, gate, up, down; applied as fused qkv / o / gate_up / down, "
+                        "128 calls), bf16 base + 100 resident tenants (sign words + fp16 "
+                        "group-128 scales), batch 512, Zipf(1.1) tenant ids, one decode step per step",
+            "layers": args.layers, "tenants": args.tenants, "batch": args.batch,
+            "group_size": GROUP, "l2": "inputs larger than L2 (~112 GB resident)",
+            "parallelism": f"replicas x{world}"}
 
 
 def zipf_ids_host(rng, batch, n, s):
@@ -350,9 +371,7 @@ def bench_serving(args, rank, pg, log, peaks):
     h2d = B * 4096 * 2 + B * 14336 * 2 + B * 4
     d2h = B * 4096 * 2
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    tokens_all = sum_over_ranks(pg, float(B * args.steps))
-    value = tokens_all / (ms_max / 1e3)
+    tokens_all, _, value = whole_job_rate(pg, float(B * args.steps), ms)
     e2e_value = tokens_all / (ms_e2e / 1e3)
     hbm_gbs = total_bytes / (ms_max / 1e3) / 1e9
 
@@ -506,8 +525,7 @@ def reference_arm(args):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * BATCH / value, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "serving: 32-layer Llama-3-8B-shaped projection stack, 100 "
-                                   "tenants, batch 512, Zipf(1.1) ids (bounded sample)"},
+            "config": serving_config(args, world),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -550,14 +568,7 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": "serving: 32-layer Llama-3-8B-shaped projection stack "
-                                   "(q, k, v, o, gate, up, down; applied as fused qkv / o / "
-                                   "gate_up / down, 128 calls), bf16 base + 100 resident tenants "
-                                   "(sign words + fp16 group-128 scales), batch 512, Zipf(1.1) "
-                                   "tenant ids, one decode step per step",
-                       "layers": args.layers, "tenants": args.tenants, "batch": args.batch,
-                       "group_size": GROUP, "l2": "inputs larger than L2 (~112 GB resident)",
-                       "parallelism": f"replicas x{world}"},
+            "config": serving_config(args, world),
             "hbm_gbs": res["hbm_gbs"], "hbm_frac_of_measured_peak": res["hbm_frac"],
             "roofline": res["roofline"], "cpu_baseline": cpu, "e2e": res["e2e"],
             "gpu_launches": res["gpu_launches"], "clocks": res["clocks"],
