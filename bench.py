@@ -47,6 +47,27 @@ GROUP = 128
 ZIPF_S = 1.1
 TC_MIN_TOKENS = 8  # the library's many-token threshold (tensor-core delta from this count on)
 
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum, mean over the 4
+# fused calls of a layer) from the ncu capture in profiles/delta_lut_serving_layer.md,
+# keyed by the hash of the sources the kernel was built from: once they change the
+# number no longer describes the kernel and the roofline reports traffic = null.
+NCU_TRAFFIC = {
+    "delta_lut": {"sources": ["bd_apply.cu", "bd_internal.cuh"], "sha256_16": "4961a89f5eaf80fb",
+                  "bytes_per_launch": 773.1e6},
+}
+
+
+def ncu_traffic(kernel: str):
+    import hashlib
+    rec = NCU_TRAFFIC.get(kernel)
+    if rec is None:
+        return None
+    h = hashlib.sha256()
+    for f in rec["sources"]:
+        with open(os.path.join(ROOT, "tenant_serving_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return rec["bytes_per_launch"] if h.hexdigest()[:16] == rec["sha256_16"] else None
+
 
 def parse():
     p = argparse.ArgumentParser()
@@ -395,7 +416,8 @@ def bench_serving(args, rank, pg, log, peaks):
                     for k, v in prof.items()},
         "roofline": {"kernel": dname, "bound": bound, "achieved": achieved, "peak": peak,
                      "unit": unit, "frac": (achieved / peak) if achieved else None,
-                     "traffic": None,
+                     "traffic": ncu_traffic(dname),
+                     "algorithmic_per_launch": (work / dl) if (work and dl) else None,
                      "peak_source": f"{peak_src} (MEASURED_PEAKS.json "
                                     f"{'bf16_tflops_sustained' if unit == 'TFLOP/s' else 'hbm_gbs'})",
                      "avg_launch_us": dms / dl * 1e3 if dl else None},
@@ -574,7 +596,7 @@ def main():
             "gpu_launches": res["gpu_launches"], "clocks": res["clocks"],
             "ms_per_step_profiled": res["ms_per_step_profiled"],
             "distinct_tenants_mean": res["distinct_tenants_mean"],
-            "kernels": res["kernels"], "compress": comp,
+            "kernels": res["kernels"], "kernel_rates": res["kernel_rates"], "compress": comp,
         }
         print(json.dumps(line))
     if pg is not None:
