@@ -42,7 +42,7 @@ constexpr int kMaxBatch = 65536;
 // planning: token groups for the lookup-table kernel, segments for the tensor-core one
 // ------------------------------------------------------------------------------------
 // Tokens are grouped by tenant (a counting sort). A tenant with at least tc_min tokens
-// whose record the tensor-core path supports gets tensor-core segments of <= 128 tokens;
+// whose record the tensor-core path supports gets tensor-core segments of <= kTcSegTokens tokens;
 // every other tenant's tokens (and the base-only tokens) are cut into lookup-table groups
 // of <= kGroupTokens.
 // Workspace layout (int32): [0] n_groups, [1] n_tc, [2..3] pad, grp_tenant[max_groups],
@@ -50,7 +50,7 @@ constexpr int kMaxBatch = 65536;
 // tc_count[max_tc], tc_xrow[max_tc] (first row in the gathered X), perm[batch]; and, in
 // a region of its own, a copy of each tensor-core segment's tenant record.
 constexpr int kGroupTokens = 2;
-constexpr int kTcMaxTokens = 128;
+constexpr int kTcMaxTokens = kTcSegTokens;
 
 inline int max_groups_for(int64_t batch, int32_t n_tenants) {
   const int64_t keys = batch < (int64_t)n_tenants + 1 ? batch : (int64_t)n_tenants + 1;
@@ -75,7 +75,7 @@ __global__ void __launch_bounds__(1024) k_tenant_bucket(const int32_t* __restric
                                                         bd_tenant* __restrict__ tc_rec,
                                                         uint32_t* __restrict__ status) {
   extern __shared__ int32_t cnt[];  // n_tenants + 1 counters (last = base only)
-  __shared__ int32_t wsum[4][32];
+  __shared__ int32_t wsum[5][32];
   __shared__ int32_t bad;
   const int nkeys = n_tenants + 1;
   int32_t* grp_tenant = seg_base + 4;
@@ -101,48 +101,52 @@ __global__ void __launch_bounds__(1024) k_tenant_bucket(const int32_t* __restric
     atomicAdd(&cnt[u < 0 ? n_tenants : u], 1);
   }
   __syncthreads();
-  // per key: tokens, lookup groups, tensor-core segments, gathered-X rows
-  auto plan = [&](int k, int c, int& ng, int& nt, int& nx) {
-    ng = nt = nx = 0;
+  // per key: tokens, full lookup groups (kGroupTokens tokens), remainder groups, tensor-core
+  // segments, gathered-X rows. All full groups are numbered before all remainder groups,
+  // so that the lookup-table kernel meets one kind of group for long stretches.
+  auto plan = [&](int k, int c, int& ng, int& nr, int& nt, int& nx) {
+    ng = nr = nt = nx = 0;
     if (c == 0) return;
     const bool tc = max_tc > 0 && k < n_tenants && c >= tc_min && tc_eligible(tenants[k], d_in);
     if (tc) {
       nt = (c + kTcMaxTokens - 1) / kTcMaxTokens;
       for (int j = 0; j < c; j += kTcMaxTokens) nx += (min(kTcMaxTokens, c - j) + 15) & ~15;
     } else {
-      ng = (c + kGroupTokens - 1) / kGroupTokens;
+      ng = c / kGroupTokens;
+      nr = (c % kGroupTokens) ? 1 : 0;
     }
   };
   const int per = (nkeys + blockDim.x - 1) / blockDim.x;
   const int k0 = threadIdx.x * per, k1 = min(nkeys, k0 + per);
-  int v[4] = {0, 0, 0, 0};  // tokens, groups, tc segments, X rows
+  int v[5] = {0, 0, 0, 0, 0};  // tokens, full groups, tc segments, X rows, remainder groups
   for (int k = k0; k < k1; ++k) {
-    int ng, nt, nx;
-    plan(k, cnt[k], ng, nt, nx);
+    int ng, nr, nt, nx;
+    plan(k, cnt[k], ng, nr, nt, nx);
     v[0] += cnt[k];
     v[1] += ng;
     v[2] += nt;
     v[3] += nx;
+    v[4] += nr;
   }
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  int inc[4] = {v[0], v[1], v[2], v[3]};
+  int inc[5] = {v[0], v[1], v[2], v[3], v[4]};
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 5; ++i) {
       const int a = __shfl_up_sync(0xffffffffu, inc[i], o);
       if (lane >= o) inc[i] += a;
     }
   }
   if (lane == 31) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) wsum[i][w] = inc[i];
+    for (int i = 0; i < 5; ++i) wsum[i][w] = inc[i];
   }
   __syncthreads();
   if (w == 0) {
     const int nw = blockDim.x >> 5;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 5; ++i) {
       int a = lane < nw ? wsum[i][lane] : 0;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -157,10 +161,12 @@ __global__ void __launch_bounds__(1024) k_tenant_bucket(const int32_t* __restric
   int gidx = inc[1] - v[1] + (w > 0 ? wsum[1][w - 1] : 0);
   int tidx = inc[2] - v[2] + (w > 0 ? wsum[2][w - 1] : 0);
   int xrow = inc[3] - v[3] + (w > 0 ? wsum[3][w - 1] : 0);
+  const int n_full = wsum[1][(blockDim.x >> 5) - 1];  // all full groups come first
+  int ridx = n_full + inc[4] - v[4] + (w > 0 ? wsum[4][w - 1] : 0);
   for (int k = k0; k < k1; ++k) {
     const int c = cnt[k];
-    int ng, nt, nx;
-    plan(k, c, ng, nt, nx);
+    int ng, nr, nt, nx;
+    plan(k, c, ng, nr, nt, nx);
     if (nt > 0) {
       for (int j = 0; j < c; j += kTcMaxTokens) {
         const int n = min(kTcMaxTokens, c - j);
@@ -174,17 +180,18 @@ __global__ void __launch_bounds__(1024) k_tenant_bucket(const int32_t* __restric
       }
     } else {
       for (int j = 0; j < c; j += kGroupTokens) {
-        grp_tenant[gidx] = (k == n_tenants) ? -1 : k;
-        grp_start[gidx] = off + j;
-        grp_len[gidx] = min(kGroupTokens, c - j);
-        ++gidx;
+        const bool full = c - j >= kGroupTokens;
+        const int gi = full ? gidx++ : ridx++;
+        grp_tenant[gi] = (k == n_tenants) ? -1 : k;
+        grp_start[gi] = off + j;
+        grp_len[gi] = min(kGroupTokens, c - j);
       }
     }
     cnt[k] = off;  // becomes the scatter cursor
     off += c;
   }
   if (threadIdx.x == blockDim.x - 1) {  // the last thread holds the totals
-    seg_base[0] = gidx;
+    seg_base[0] = ridx;
     seg_base[1] = tidx;
   }
   __syncthreads();
@@ -839,7 +846,7 @@ ApplyLayout layout_apply(int64_t d_out, int64_t d_in, int64_t batch, int32_t n_t
   if (L.max_groups < 1) L.max_groups = 1;
   // a batch smaller than the many-token threshold has no tensor-core segment at all
   if (tc_delta && batch >= kTcMinTokens) {
-    // segments: at most one per many-token tenant plus one per extra 128 tokens
+    // segments: at most one per many-token tenant plus one per extra kTcSegTokens tokens
     int64_t by_tokens = batch / kTcMinTokens, by_tenants = n_tenants;
     L.max_tc = (int)((by_tokens < by_tenants ? by_tokens : by_tenants) + batch / kTcMaxTokens + 1);
   } else {

@@ -39,7 +39,9 @@ __global__ void __launch_bounds__(128, 1) k_base_tc(const __grid_constant__ CUte
   int* issued_out = reinterpret_cast<int*>(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m_blk = blockIdx.x, n_blk = blockIdx.y, kz = blockIdx.z;
+  // the N blocks of one row block are neighbours in launch order, so they stream the same
+  // W_base tiles at about the same time and all but the first read them from L2
+  const int n_blk = blockIdx.x, m_blk = blockIdx.y, kz = blockIdx.z;
   const int kb0 = kz * kb_per_split;
   const int kb1 = min(kblocks, kb0 + kb_per_split);
   const int nkb = kb1 - kb0;  // >= 1 by construction on the host
@@ -234,7 +236,8 @@ bd_status launch_base_tc(const TcPlan& p, const void* w_base, const void* x, int
     }
     attr_set = true;
   }
-  dim3 grid(p.tiles_m, p.tiles_n, p.ksplit);
+  if (p.tiles_m > 65535) return BD_ERR_SHAPE;  // row blocks run along grid y
+  dim3 grid(p.tiles_n, p.tiles_m, p.ksplit);
   launch_begin(K_BASE_TC, s);
   k_base_tc<<<grid, 128, p.smem, s>>>(tw, tx, d_out, (int)batch, p.n_tile, p.stages, p.kblocks,
                                       p.kb_per_split, y_part, status);

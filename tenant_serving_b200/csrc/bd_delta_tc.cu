@@ -31,7 +31,7 @@ namespace bd {
 constexpr int DT_BM = 128;            // rows per work item
 constexpr int DT_BK = 64;             // K per stage (64 fp16 = one 128-byte swizzle row)
 constexpr int DT_KPW = 4;             // stages per 256-column window
-constexpr int DT_NMAX = 128;          // tokens per segment
+constexpr int DT_NMAX = kTcSegTokens;  // tokens per segment
 constexpr int DT_AW = 2;              // A ring depth in windows (tensor memory)
 constexpr int DT_XW_MAX = 8;          // X ring depth in windows (shared memory), fewer for wide segments
 constexpr int DT_WSLOTS = 16;         // sign-window ring depth (64 KB of signs in flight)

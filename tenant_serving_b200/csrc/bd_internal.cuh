@@ -13,6 +13,10 @@ namespace bd {
 // ------------------------------------------------------------------------------------
 // kernel kinds (for launch accounting and per-kernel timing)
 // ------------------------------------------------------------------------------------
+// Tokens per tensor-core delta segment (the MMA's N, rounded up to 16). 64 keeps one
+// window of a segment's activations at 32 KB, so four windows fit the shared-memory ring.
+constexpr int kTcSegTokens = 64;
+
 enum KernelKind : int32_t {
   K_DELTA_STATS = 0,     // fused delta + whole-matrix shifted sums for the clip
   K_STATS_FINAL,         // fixed-order merge of the partial sums -> mean, std, lo, hi

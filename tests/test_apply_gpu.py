@@ -305,7 +305,7 @@ def _many_token_problem(seed, d_out, d_in, counts, mode, G, zero_base=False, x_s
 @pytest.mark.parametrize("layout", [0, 1])
 @pytest.mark.parametrize("mode,G", [(0, 128), (0, 64), (0, 256), (1, 128), (3, 128), (2, 128)])
 def test_many_token_tenants_delta_only(bd, mode, G, layout):
-    """300 tokens (two segments of <= 256), 8 (the smallest many-token tenant), 7, 20 and
+    """300 tokens (five tensor-core segments), 8 (the smallest many-token tenant), 7, 20 and
     1 token; 200 rows (a partial 128-row tile), 384 columns (a partial 256-column tile of
     the serving layout; 768 for groups of 256). Column scales (mode 2) stay on the
     lookup-table path."""
