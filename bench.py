@@ -45,7 +45,7 @@ N_TENANTS = 100
 BATCH = 512
 GROUP = 128
 ZIPF_S = 1.1
-TC_MIN_TOKENS = 8  # the library's many-token threshold (tensor-core delta from this count on)
+TC_MIN_TOKENS = 6  # the library's many-token threshold (tensor-core delta from this count on)
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum, mean over the 4
 # fused calls of a layer) from the ncu capture in profiles/delta_lut_serving_layer.md,

@@ -251,14 +251,17 @@ __global__ void __launch_bounds__(256) k_base_gemv_f32(const float* __restrict__
 // in shared memory for every sign byte v; then one byte of signs costs one table read
 // per token.
 //   lanes: q = lane >> 1 picks one of 16 rows, wp = lane & 1 one half of the window
-//   (words 4wp..4wp+3). At step (k, j) a lane reads word 4wp + ((k + q/4) & 3) and its
-//   byte (j + q) & 3: the 32 lanes read 32 different staged words and 32 different
-//   table chunks (= 32 different banks), so neither read has bank conflicts.
-//   table page: it sits at shared address 0x10000, entry (v, token, chunk) at
-//   0x10000 + v * 256 + 4 * (32 * token + chunk). One PRMT of the sign word with the
-//   lane's slot constant (which carries the 0x1 of 0x10000 in its upper half) yields the
-//   whole 32-bit shared address of token 0's entry; token 1's is 128 bytes further, an
-//   immediate. A lookup is PRMT + ld.shared + FADD.
+//   (words 4wp..4wp+3). At step (k, j) a lane reads word 4wp + ((k + q/4 + 2wp) & 3)
+//   and its byte (j + q) & 3: the 32 lanes read 32 different staged words (32 banks),
+//   and each half-warp reads 16 different table chunks modulo 16.
+//   table page: it sits at shared address 0x10000. For a 2-token group entry
+//   (v, chunk, token) is at 0x10000 + v * 256 + 8 * chunk + 4 * token: the two tokens sit
+//   side by side, one 8-byte ld.shared returns both, and each half-warp's 16 lanes cover
+//   the 32 banks once. For a 1-token group entry (v, chunk) is at 0x10000 + v * 256 +
+//   4 * chunk, and the 32 lanes' 4-byte reads cover the 32 banks once. One PRMT of the
+//   sign word with the lane's slot constant (entry stride x chunk, plus the 0x1 of
+//   0x10000 in its upper half) yields the whole 32-bit shared address of the entry.
+//   A lookup is PRMT + ld.shared(.v2) + FADD per token.
 //   Group-128 scales are one per lane per row (words 4wp..4wp+3 are one group) and are
 //   staged next to the sign words.
 constexpr int LUT_THREADS = 256;    // 8 warps, 64 rows each per stage
@@ -288,10 +291,13 @@ __device__ __forceinline__ float lds_f32(uint32_t a) {
   asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
   return v;
 }
-__device__ __forceinline__ float lds_f32_128(uint32_t a) {
-  float v;
-  asm volatile("ld.shared.f32 %0, [%1+128];" : "=f"(v) : "r"(a));
+__device__ __forceinline__ float2 lds_f32x2(uint32_t a) {
+  float2 v;
+  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a));
   return v;
+}
+__device__ __forceinline__ void sts_f32x2(uint32_t a, float x, float y) {
+  asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(a), "f"(x), "f"(y) : "memory");
 }
 __device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
   uint32_t v;
@@ -448,52 +454,61 @@ __device__ __forceinline__ void lut_build(const LutPiece& P, int win, int b, int
       for (int k = 0; k < 8; ++k) sc[k] = lds_f32(xs + 2048 + 32 * c + 4 * k);
     }
   }
+  // both tokens' 16 low-nibble sums (a second token of 0 for single-token groups)
+  float lo16[2][16];
+  float xv[2][8];
 #pragma unroll
   for (int tt = 0; tt < 2; ++tt) {
-    if (tt < P.ntok) {
-      float xv[8];
-      if (col < d_in) {
-        if (XBF16) {
-          uint4 v;
-          asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                       : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                       : "r"(xs + 1024 * tt + 16 * c));
-          const uint32_t a[4] = {v.x, v.y, v.z, v.w};
+    if (tt < P.ntok && col < d_in) {
+      if (XBF16) {
+        uint4 v;
+        asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                     : "r"(xs + 1024 * tt + 16 * c));
+        const uint32_t a[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            xv[2 * k] = bf16lo(a[k]);
-            xv[2 * k + 1] = bf16hi(a[k]);
-          }
-        } else {
-#pragma unroll
-          for (int k = 0; k < 8; ++k) xv[k] = lds_f32(xs + 1024 * tt + 32 * c + 4 * k);
-        }
-        if (P.mode == BD_SCALE_COL) {
-#pragma unroll
-          for (int k = 0; k < 8; ++k) xv[k] *= sc[k];
+        for (int k = 0; k < 4; ++k) {
+          xv[tt][2 * k] = bf16lo(a[k]);
+          xv[tt][2 * k + 1] = bf16hi(a[k]);
         }
       } else {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) xv[k] = 0.f;
+        for (int k = 0; k < 8; ++k) xv[tt][k] = lds_f32(xs + 1024 * tt + 32 * c + 4 * k);
       }
-      float p01[4], p23[4];
+      if (P.mode == BD_SCALE_COL) {
 #pragma unroll
-      for (int n = 0; n < 4; ++n) {
-        p01[n] = ((n & 1) ? xv[0] : -xv[0]) + ((n & 2) ? xv[1] : -xv[1]);
-        p23[n] = ((n & 1) ? xv[2] : -xv[2]) + ((n & 2) ? xv[3] : -xv[3]);
+        for (int k = 0; k < 8; ++k) xv[tt][k] *= sc[k];
       }
-      float lo16[16];
+    } else {
 #pragma unroll
-      for (int lo = 0; lo < 16; ++lo) lo16[lo] = p01[lo & 3] + p23[lo >> 2];
+      for (int k = 0; k < 8; ++k) xv[tt][k] = 0.f;
+    }
+    float p01[4], p23[4];
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int h = warp + 8 * hh;
-        const float hi = (((h & 1) ? xv[4] : -xv[4]) + ((h & 2) ? xv[5] : -xv[5])) +
-                         (((h & 4) ? xv[6] : -xv[6]) + ((h & 8) ? xv[7] : -xv[7]));
-        const uint32_t base = LUT_ADDR + (uint32_t)(h << 12) + 4u * (uint32_t)(32 * tt + c);
+    for (int n = 0; n < 4; ++n) {
+      p01[n] = ((n & 1) ? xv[tt][0] : -xv[tt][0]) + ((n & 2) ? xv[tt][1] : -xv[tt][1]);
+      p23[n] = ((n & 1) ? xv[tt][2] : -xv[tt][2]) + ((n & 2) ? xv[tt][3] : -xv[tt][3]);
+    }
 #pragma unroll
-        for (int lo = 0; lo < 16; ++lo) sts_f32(base + (uint32_t)lo * 256u, lo16[lo] + hi);
-      }
+    for (int lo = 0; lo < 16; ++lo) lo16[tt][lo] = p01[lo & 3] + p23[lo >> 2];
+  }
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    const int h = warp + 8 * hh;
+    float hi[2];
+#pragma unroll
+    for (int tt = 0; tt < 2; ++tt)
+      hi[tt] = (((h & 1) ? xv[tt][4] : -xv[tt][4]) + ((h & 2) ? xv[tt][5] : -xv[tt][5])) +
+               (((h & 4) ? xv[tt][6] : -xv[tt][6]) + ((h & 8) ? xv[tt][7] : -xv[tt][7]));
+    if (P.ntok == 2) {
+      const uint32_t base = LUT_ADDR + (uint32_t)(h << 12) + 8u * (uint32_t)c;
+#pragma unroll
+      for (int lo = 0; lo < 16; ++lo)
+        sts_f32x2(base + (uint32_t)lo * 256u, lo16[0][lo] + hi[0], lo16[1][lo] + hi[1]);
+    } else {
+      const uint32_t base = LUT_ADDR + (uint32_t)(h << 12) + 4u * (uint32_t)c;
+#pragma unroll
+      for (int lo = 0; lo < 16; ++lo) sts_f32(base + (uint32_t)lo * 256u, lo16[0][lo] + hi[0]);
     }
   }
 }
@@ -511,16 +526,17 @@ __device__ __forceinline__ float2 lut_rows_generic(uint32_t wrow, uint32_t srow,
   if (rl >= P.rows) return make_float2(0.f, 0.f);
 #pragma unroll 1
   for (int k = 0; k < 4; ++k) {
-    const int wi = 4 * wp + ((k + (q >> 2)) & 3);
+    const int wi = 4 * wp + ((k + (q >> 2) + 2 * wp) & 3);
     const int64_t col = (int64_t)win * LUT_W + 32 * wi;
     if (col >= d_in) continue;
     const uint32_t word = lds_u32(wrow + 4u * (uint32_t)wi);
     float p0 = 0.f, p1 = 0.f;
     for (int j = 0; j < 4; ++j) {
       const int b = (j + q) & 3;
-      const uint32_t idx = LUT_ADDR + (((word >> (8 * b)) & 0xFFu) << 8) + 4u * (uint32_t)(4 * wi + b);
+      const uint32_t idx = LUT_ADDR + (((word >> (8 * b)) & 0xFFu) << 8) +
+                           (NT == 2 ? 8u : 4u) * (uint32_t)(4 * wi + b);
       p0 += lds_f32(idx);
-      if (NT == 2) p1 += lds_f32_128(idx);
+      if (NT == 2) p1 += lds_f32(idx + 4u);
     }
     float sw = 1.f;
     if (P.sc_kind == 1) {  // staged group-128 scales: group (wi >> 2) of the window
@@ -546,6 +562,15 @@ __device__ __forceinline__ void lut_piece(const LutPiece& P, float (&acc)[LUT_NS
                                           int warp, int q, int wp) {
   const bool f16s = P.scale_f16 != 0;
   const int ssz = GENERIC ? (f16s ? 2 : 4) : (SC == 2 ? 4 : 2);
+  // 2-token tables have 8-byte entries: the slot bytes (entry stride x chunk, <= 124 for
+  // the 4-byte stride) double, the 0x1 of 0x10000 in the upper half stays
+  uint32_t sl[4][2];
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh)
+      sl[k][hh] = NT == 2 ? (((slot2[k][hh] & 0xFFFFu) << 1) | (slot2[k][hh] & 0xFFFF0000u))
+                          : slot2[k][hh];
   const int rows = P.rows;
   const int nsb = (rows + LUT_SB - 1) / LUT_SB;  // 1..4
   int pw = 0, ps = 0;
@@ -597,9 +622,14 @@ __device__ __forceinline__ void lut_piece(const LutPiece& P, float (&acc)[LUT_NS
                 float v0[4], v1[4];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                  const uint32_t idx = __byte_perm(wd[k], slot2[k][j >> 1], sel[j]);
-                  v0[j] = lds_f32(idx);
-                  if (NT == 2) v1[j] = lds_f32_128(idx);
+                  const uint32_t idx = __byte_perm(wd[k], sl[k][j >> 1], sel[j]);
+                  if (NT == 2) {
+                    const float2 e = lds_f32x2(idx);
+                    v0[j] = e.x;
+                    v1[j] = e.y;
+                  } else {
+                    v0[j] = lds_f32(idx);
+                  }
                 }
                 w0[k] = (v0[0] + v0[1]) + (v0[2] + v0[3]);
                 if (NT == 2) w1[k] = (v1[0] + v1[1]) + (v1[2] + v1[3]);
@@ -623,7 +653,7 @@ __device__ __forceinline__ void lut_piece(const LutPiece& P, float (&acc)[LUT_NS
 }
 
 // Per-lane lookup constants (see the comment above k_delta_lut's lookup loop).
-__device__ __forceinline__ void lut_lane_constants(int q, int wp, uint32_t (&sel)[4],
+__device__ __forceinline__ void lut_lane_constants(int q, int wp, uint32_t estride, uint32_t (&sel)[4],
                                                    uint32_t (&slot2)[4][2], uint32_t (&wofs)[4]) {
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
@@ -632,12 +662,12 @@ __device__ __forceinline__ void lut_lane_constants(int q, int wp, uint32_t (&sel
   }
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    const int wi = 4 * wp + ((k + (q >> 2)) & 3);
+    const int wi = 4 * wp + ((k + (q >> 2) + 2 * wp) & 3);
     wofs[k] = 4u * (uint32_t)wi;
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
-      const uint32_t s0 = 4u * (uint32_t)(4 * wi + ((2 * hh + q) & 3));
-      const uint32_t s1 = 4u * (uint32_t)(4 * wi + ((2 * hh + 1 + q) & 3));
+      const uint32_t s0 = estride * (uint32_t)(4 * wi + ((2 * hh + q) & 3));
+      const uint32_t s1 = estride * (uint32_t)(4 * wi + ((2 * hh + 1 + q) & 3));
       slot2[k][hh] = s0 | (s1 << 8) | (LUT_ADDR & 0xFFFF0000u);
     }
   }
@@ -677,7 +707,7 @@ __global__ void __launch_bounds__(LUT_THREADS, 1) k_delta_lut(
   // per-lane lookup constants. sel[j]: byte 0 <- slot byte (j & 1) of slot2[k][j >> 1],
   // byte 1 <- sign byte (j + q) & 3, bytes 2-3 <- 0x0001 (the table's 0x10000).
   uint32_t sel[4], slot2[4][2], wofs[4];
-  lut_lane_constants(q, wp, sel, slot2, wofs);
+  lut_lane_constants(q, wp, 4u, sel, slot2, wofs);  // 1-token entry stride; lut_piece doubles it
 
   while (pos < end) {
     if (tid == 0) {
@@ -826,7 +856,7 @@ bd_status launch_delta_tc(const bd_tenant* tenants, const int32_t* seg, int max_
 // A tenant with at least this many tokens in a batch (and a supported record) goes to the
 // tensor-core delta kernel; below it the lookup-table kernel is cheaper per token.
 #ifndef BD_TC_MIN_TOKENS
-#define BD_TC_MIN_TOKENS 8
+#define BD_TC_MIN_TOKENS 6
 #endif
 constexpr int kTcMinTokens = BD_TC_MIN_TOKENS;
 
