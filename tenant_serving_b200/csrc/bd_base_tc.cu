@@ -204,14 +204,30 @@ TcPlan plan_base_tc(int64_t d_out, int64_t d_in, int64_t batch) {
   p.n_tile = ((per + 15) / 16) * 16;
   p.tiles_m = (int)((d_out + TC_BM - 1) / TC_BM);
   p.kblocks = (int)((d_in + TC_BK - 1) / TC_BK);
+  // K splits: one CTA per SM at a time, so the time goes as the number of waves times the
+  // K blocks of a CTA. Each extra split also writes and re-reads batch x d_out fp32
+  // partial sums; that traffic (at ~5 TB/s) is charged in units of one K block's MMA
+  // time (4 MMAs of N/2 cycles, at least ~46 cycles each, at ~1.9 GHz). At least 4 K
+  // blocks per CTA.
   const int sms = sm_count();
   const int base_ctas = p.tiles_m * p.tiles_n;
-  int want = (sms + base_ctas - 1) / base_ctas;  // splits to cover the SMs once
-  if (want < 1) want = 1;
-  int kb_per = (p.kblocks + want - 1) / want;
-  if (kb_per < 4) kb_per = 4 < p.kblocks ? 4 : p.kblocks;
-  p.kb_per_split = kb_per;
-  p.ksplit = (p.kblocks + kb_per - 1) / kb_per;
+  const double kb_seconds = 4.0 * (p.n_tile / 2 > 46 ? p.n_tile / 2 : 46) / 1.9e9;
+  const double split_units = 8.0 * (double)batch * (double)d_out / 5e12 / kb_seconds;
+  int best_kb = p.kblocks;
+  double best_cost = 1e30;
+  for (int k = 1; k <= 16; ++k) {
+    const int kb_per = (p.kblocks + k - 1) / k;
+    if (k > 1 && kb_per < 4) break;
+    const int splits = (p.kblocks + kb_per - 1) / kb_per;
+    const int64_t waves = ((int64_t)base_ctas * splits + sms - 1) / sms;
+    const double cost = (double)waves * kb_per + (splits - 1) * split_units;
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best_kb = kb_per;
+    }
+  }
+  p.kb_per_split = best_kb;
+  p.ksplit = (p.kblocks + best_kb - 1) / best_kb;
   const size_t stage_bytes = (size_t)TC_BM * TC_BK * 2 + (size_t)p.n_tile * TC_BK * 2;
   int st = (int)((200 * 1024) / stage_bytes);
   if (st > 8) st = 8;
