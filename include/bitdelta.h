@@ -212,8 +212,15 @@ size_t bd_apply_workspace_size(int64_t d_out, int64_t d_in, int64_t batch, int32
  * ("BitDelta Guide", "Systems Mechanics: 1. Decoupled Forward Pass", and "2. Fused
  * Dequantization": sign bits stay packed in memory and are unpacked on chip).
  * The base product W_base X is computed once for the whole batch; the tokens are
- * grouped by tenant on the device (no host synchronisation) and each tenant's packed
- * signs and scales are streamed once per group of its tokens.
+ * grouped by tenant on the device (no host synchronisation). Two delta kernels share the
+ * work, chosen per tenant on the device:
+ *   - a tenant with at least 6 tokens in the batch, stored in the TILED layout with
+ *     fp16 scales in GROUP (group_size >= 64), ROW or TENSOR mode (bf16 w_base and
+ *     d_in % 64 == 0), is a dense product on the tensor cores, in segments of <= 64 of
+ *     its tokens; its activations are scaled per token by a power of two into fp16 for
+ *     that product (exact for bf16 values in fp16's normal range);
+ *   - every other tenant goes through the sign lookup-table kernel, its packed signs and
+ *     scales streamed once per group of <= 2 of its tokens.
  *
  *   w_base      : [d_out][d_in], w_dtype BD_BF16 (tensor-core path) or BD_F32.
  *   tenants     : device array of n_tenants bd_tenant records (n_tenants >= 0).

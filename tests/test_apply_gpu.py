@@ -241,7 +241,7 @@ def test_launches_are_counted(bd):
     wb, tenants, ids, x = _problem(1, 128, 256, 4, 2, (0,))
     _run(bd, wb, tenants, ids, x)
     assert bd.bd_launch_count() - n0 == 3  # bucket, base product, lookup-table delta
-    # from 8 tokens on the tensor-core delta (gather + product) is launched as well
+    # from 6 tokens in a batch on the tensor-core delta (gather + product) is launched too
     n0 = bd.bd_launch_count()
     wb, tenants, ids, x = _problem(1, 128, 256, 16, 2, (0,))
     _run(bd, wb, tenants, ids, x)
