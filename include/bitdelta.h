@@ -257,6 +257,18 @@ const char* bd_status_string(int32_t status);
  * was loaded (all calls, all streams). */
 int64_t bd_launch_count(void);
 
+/* bd_selftest_wait_timeout — exercises the failure-detection path of the kernels'
+ * bounded waits on the device, without a fault. The method's pages have no counterpart;
+ * this is a test aid. It launches one kernel whose thread waits on a barrier that nothing
+ * ever completes, through the same bounded wait the tensor-core kernels use; after
+ * limit_cycles SM clock cycles the wait gives up, BD_DEV_TIMEOUT is set in the status
+ * word of `workspace` (cleared first) and the kernel ends normally, so the context stays
+ * usable. Read the outcome with bd_get_status (BD_ERR_TIMEOUT).
+ *   workspace    : device, >= 256 bytes, 16-byte aligned (its status block is used).
+ *   limit_cycles : 1 .. 4e9 (the kernels' own limit, ~2 s); BD_ERR_CONFIG otherwise. */
+bd_status bd_selftest_wait_timeout(void* workspace, size_t ws_bytes, int64_t limit_cycles,
+                                   void* stream);
+
 /* Optional per-kernel timing. While enabled, every kernel the library launches is
  * bracketed by two CUDA events recorded on its launch stream (at most `capacity`
  * launches are recorded; later ones are counted but not timed). bd_profile_collect

@@ -38,7 +38,7 @@ EXPORTS = (
     "bd_compress", "bd_compress_noalloc", "bd_compress_workspace_size", "bd_reconstruct",
     "bd_apply_multi", "bd_prepared_signs_bytes", "bd_prepared_scales_bytes", "bd_prepare_tenant",
     "bd_apply_workspace_size", "bd_get_status", "bd_status_string", "bd_launch_count",
-    "bd_profile_enable", "bd_profile_collect", "bd_kernel_name",
+    "bd_profile_enable", "bd_profile_collect", "bd_kernel_name", "bd_selftest_wait_timeout",
 )
 
 
@@ -107,6 +107,8 @@ def lib():
     L.bd_profile_collect.restype = c_int32
     L.bd_kernel_name.argtypes = [c_int32]
     L.bd_kernel_name.restype = ctypes.c_char_p
+    L.bd_selftest_wait_timeout.argtypes = [c_void_p, c_size_t, c_int64, c_void_p]
+    L.bd_selftest_wait_timeout.restype = c_int32
     _LIB = L
     return L
 
@@ -312,6 +314,14 @@ def bd_get_status(workspace, stream=None):
 
 def bd_launch_count() -> int:
     return int(lib().bd_launch_count())
+
+
+def bd_selftest_wait_timeout(workspace, limit_cycles: int, stream=None) -> int:
+    """Wrap ``bd_selftest_wait_timeout``: returns the host status of the launch; the
+    device outcome is read with bd_get_status(workspace)."""
+    _require_cuda(workspace)
+    return int(lib().bd_selftest_wait_timeout(_ptr(workspace), workspace.numel() * workspace.element_size(),
+                                              int(limit_cycles), _stream(stream)))
 
 
 def bd_profile_enable(on: bool, capacity: int = 65536):

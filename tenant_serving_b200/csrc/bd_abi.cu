@@ -1,5 +1,6 @@
 // Status strings, device status read-back, launch accounting and per-kernel timing.
 #include "bd_internal.cuh"
+#include "bd_tc.cuh"
 
 #include <atomic>
 #include <mutex>
@@ -11,7 +12,7 @@ static const char* const kKernelNames[K_KIND_COUNT] = {
     "delta_stats",       "stats_final",  "scale_signpack", "col_scale_signpack",
     "scale_final",       "reconstruct",  "tenant_bucket",  "base_gemv",
     "base_tc",           "delta_lut",    "select_fixup",   "prepare",
-    "tc_gather",         "delta_tc",
+    "tc_gather",         "delta_tc",     "selftest_wait",
 };
 
 const char* kernel_name(int32_t kind) {
@@ -119,6 +120,40 @@ extern "C" bd_status bd_get_status(const void* workspace, uint32_t* flags, void*
 }
 
 extern "C" int64_t bd_launch_count(void) { return g_launches.load(); }
+
+namespace bd {
+// One thread waits on an mbarrier that nothing ever arrives on, through the same bounded
+// wait the tensor-core kernels use: the wait must give up after limit_cycles, set
+// BD_DEV_TIMEOUT and let the kernel end normally.
+__global__ void k_selftest_wait(long long limit_cycles, uint32_t* __restrict__ status) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;  // never raised
+  if (threadIdx.x == 0) {
+    status[0] = 0;
+    abort_flag = 0;
+    mbar_init(&bar, 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 &&
+      !mbar_wait(&bar, 0, reinterpret_cast<volatile int*>(&abort_flag), limit_cycles))
+    atomicOr(status, BD_DEV_TIMEOUT);
+}
+}  // namespace bd
+
+extern "C" bd_status bd_selftest_wait_timeout(void* workspace, size_t ws_bytes,
+                                              int64_t limit_cycles, void* stream) {
+  if (!workspace) return BD_ERR_NULL;
+  if (ws_bytes < kStatusBytes) return BD_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) & 15u) return BD_ERR_ALIGN;
+  if (limit_cycles < 1 || limit_cycles > kWaitCycles) return BD_ERR_CONFIG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  launch_begin(K_SELFTEST_WAIT, s);
+  k_selftest_wait<<<1, 32, 0, s>>>((long long)limit_cycles, static_cast<uint32_t*>(workspace));
+  launch_end(K_SELFTEST_WAIT, s);
+  BD_LAUNCH_CHECK();
+  return BD_OK;
+}
 
 extern "C" bd_status bd_profile_enable(int32_t on, int32_t capacity) {
   std::lock_guard<std::mutex> lk(g_prof.mu);

@@ -32,6 +32,7 @@ enum KernelKind : int32_t {
   K_PREPARE,             // re-tiling of a tenant into the serving layout
   K_TC_GATHER,           // gather + fp16 scaling of the tensor-core segments' tokens
   K_DELTA_TC,            // tcgen05 delta product of many-token tenants + combine
+  K_SELFTEST_WAIT,       // failure-detection self test: a bounded wait that runs out
   K_KIND_COUNT
 };
 

@@ -113,3 +113,13 @@ def test_reconstruct_and_apply_host_validation(lib):
 
 def test_launch_count_starts_at_zero_without_gpu_work(lib):
     assert bd.bd_launch_count() >= 0
+
+
+def test_selftest_wait_timeout_host_validation(lib):
+    fake = ctypes.c_void_p(0x1000)
+    st = lib.bd_selftest_wait_timeout
+    assert st(None, 256, 1000, None) == bd.BD_ERR_NULL
+    assert st(fake, 64, 1000, None) == bd.BD_ERR_WORKSPACE
+    assert st(ctypes.c_void_p(0x1008), 256, 1000, None) == bd.BD_ERR_ALIGN
+    assert st(fake, 256, 0, None) == bd.BD_ERR_CONFIG
+    assert st(fake, 256, 5_000_000_000, None) == bd.BD_ERR_CONFIG
