@@ -227,7 +227,7 @@ __global__ void k_stats_final(const uint4* __restrict__ wb, const uint4* __restr
 // arithmetic is 32-bit (d_in < 2^31 is checked on the host) and the group size is a power
 // of two, so group indices are shifts.
 template <bool BF16, int SEGC, bool CLIP, bool GROUP>
-__global__ void __launch_bounds__(256, 3) k_scale_signpack(
+__global__ void __launch_bounds__(256, 4) k_scale_signpack(
     const uint8_t* __restrict__ wb, const uint8_t* __restrict__ wf, int64_t d_out, int d_in,
     int lg, int seg_chunks, int nseg, const ClipParams* __restrict__ clipp,
     uint32_t* __restrict__ signs, float* __restrict__ scales, double* __restrict__ partials) {
