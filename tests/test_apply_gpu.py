@@ -11,8 +11,8 @@ import pytest
 
 import oracle as O
 from helpers import APPLY_TOL, assert_apply_close, dev, host
-from workloads import (LLAMA3_8B_PROJECTIONS, activations, bf16_bits, random_tenant, tiny_config,
-                       weight_pair, zipf_ids)
+from workloads import (LLAMA3_8B_FUSED, LLAMA3_8B_PROJECTIONS, activations, bf16_bits,
+                       random_tenant, tiny_config, weight_pair, zipf_ids)
 
 pytestmark = pytest.mark.gpu
 
@@ -234,6 +234,28 @@ def test_mixed_config_layer(bd):
         assert rc == bd.BD_OK, name
         rows = np.sort(rng.choice(d_out, 64, replace=False))
         _sampled_rows_check(bd, d_out, d_in, tenants, ids, x, wb, rows, y)
+
+
+@pytest.mark.parametrize("call", ["qkv", "o", "gate_up", "down"])
+def test_serving_config_fused_call(bd, call):
+    """The serving bench's launch configuration at full size: one fused call of a layer
+    (qkv 6144x4096, o 4096x4096, gate_up 28672x4096, down 4096x14336), bf16 base, 100
+    tenants with fp16 group-128 scales in the tiled serving layout, 512 tokens with
+    Zipf(1.1) ids (both delta kernels and the split-K base product take part). Checked
+    on 64 sampled output rows."""
+    shapes = {n: (o, i) for n, o, i in LLAMA3_8B_FUSED}
+    d_out, d_in = shapes[call]
+    rng = np.random.default_rng(7000 + d_out + d_in)
+    B, T = 512, 100
+    ids = zipf_ids(rng, B, T, 1.1)
+    wb = bf16_bits(rng.normal(0, 0.02, size=(d_out, d_in)))
+    tenants = [random_tenant(rng, d_out, d_in, 0, 128) for _ in range(T)]
+    x = activations(rng, B, d_in)
+    y, rc, flags = _run(bd, wb, tenants, ids, x, layout=1)
+    assert rc == bd.BD_OK and flags == 0
+    rows = np.sort(rng.choice(d_out, 64, replace=False))
+    _sampled_rows_check(bd, d_out, d_in, tenants, ids, x, wb, rows, y)
+    assert np.isfinite(y).all()
 
 
 def test_launches_are_counted(bd):
