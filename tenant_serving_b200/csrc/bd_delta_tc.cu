@@ -35,6 +35,10 @@ constexpr int DT_NMAX = kTcSegTokens;  // tokens per segment
 constexpr int DT_AW = 2;              // A ring depth in windows (tensor memory)
 constexpr int DT_XW_MAX = 8;          // X ring depth in windows (shared memory), fewer for wide segments
 constexpr int DT_WSLOTS = 16;         // sign-window ring depth (64 KB of signs in flight)
+constexpr int DT_WDONE = 8;           // "window's MMAs done" barriers (>= A and X ring depths)
+// a window waits on wdone of window w - ring depth; the slot may not be reused by a later
+// window before that wait, which holds while both ring depths are <= DT_WDONE
+static_assert(DT_XW_MAX <= DT_WDONE && DT_AW <= DT_WDONE, "window-done ring too short");
 constexpr int DT_THREADS = 15 * 32;   // 0-7 expand A, 8-11 epilogue, 12 MMA, 13 X loader, 14 sign loader
 constexpr uint32_t DT_TMEM_COLS = 512;  // [0,256): two accumulators, [256,512): A ring (2 windows)
 constexpr uint32_t DT_ACC_STRIDE = 128;
@@ -258,11 +262,13 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_delta_tc(
   uint8_t* sb = smem;
   uint8_t* sw = sb + (size_t)xwin * xw_bytes;
   uint8_t* ss = sw + (size_t)DT_WSLOTS * DT_WIN_SIGN_BYTES;
+  // full_x: X window landed (TMA); full_a: the producers stored the window's A and saw its
+  // X land (one barrier for the MMA issuer to wait on); wdone[w % DT_WDONE]: window w's
+  // MMAs completed, which frees both its A slot and its X slot
   uint64_t* full_x = reinterpret_cast<uint64_t*>(ss + (size_t)DT_WSLOTS * DT_WIN_SCALE_BYTES);
-  uint64_t* empty_x = full_x + DT_XW_MAX;
-  uint64_t* full_a = empty_x + DT_XW_MAX;
-  uint64_t* empty_a = full_a + DT_AW;
-  uint64_t* full_w = empty_a + DT_AW;
+  uint64_t* wdone = full_x + DT_XW_MAX;
+  uint64_t* full_a = wdone + DT_WDONE;
+  uint64_t* full_w = full_a + DT_AW;
   uint64_t* empty_w = full_w + DT_WSLOTS;
   uint64_t* acc_full = empty_w + DT_WSLOTS;  // [2]
   uint64_t* acc_empty = acc_full + 2;        // [2]
@@ -272,14 +278,9 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_delta_tc(
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
-    for (int i = 0; i < xwin; ++i) {
-      mbar_init(&full_x[i], 1);
-      mbar_init(&empty_x[i], 1);
-    }
-    for (int i = 0; i < DT_AW; ++i) {
-      mbar_init(&full_a[i], 256);
-      mbar_init(&empty_a[i], 1);
-    }
+    for (int i = 0; i < xwin; ++i) mbar_init(&full_x[i], 1);
+    for (int i = 0; i < DT_WDONE; ++i) mbar_init(&wdone[i], 1);
+    for (int i = 0; i < DT_AW; ++i) mbar_init(&full_a[i], 256);
     for (int i = 0; i < DT_WSLOTS; ++i) {
       mbar_init(&full_w[i], 1);
       mbar_init(&empty_w[i], 256);
@@ -304,7 +305,7 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_delta_tc(
     const int q4 = warp & 3, h = warp >> 2;
     const int r = q4 * 32 + lane;
     const uint32_t a_lane = tmem_base + ((uint32_t)(q4 * 32) << 16) + DT_A_COL0 + (uint32_t)(16 * h);
-    Ring A, W;
+    Ring A, W, X;  // A: window count and A slot; X: the window's X slot
     bool stop = false;
     Item nxt = load_item(sg, tc_rec, item_index(0), mtiles);
     for (int i = 0; i < nloc && !stop; ++i) {
@@ -366,11 +367,14 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_delta_tc(
           for (int j = 0; j < DT_KPW; ++j) wsel[j] = 0u, scl[j] = 0u;
         }
         // the A window slot must have been read by the MMAs of two windows ago
-        if (A.n >= DT_AW &&
-            !__all_sync(0xffffffffu, mbar_wait(&empty_a[A.slot], A.phase ^ 1u, abort_flag))) {
-          *abort_flag = 1;
-          stop = true;
-          break;
+        if (A.n >= DT_AW) {
+          const int pw = A.n - DT_AW;
+          if (!__all_sync(0xffffffffu, mbar_wait(&wdone[pw % DT_WDONE],
+                                                 (uint32_t)(pw / DT_WDONE) & 1u, abort_flag))) {
+            *abort_flag = 1;
+            stop = true;
+            break;
+          }
         }
         tc_fence_after();
         const uint32_t abase = a_lane + (uint32_t)A.slot * (DT_KPW * 32u);
@@ -390,9 +394,16 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_delta_tc(
           tmem_st16(abase + (uint32_t)j * 32u, v);
         }
         tmem_wait_st();
+        // publish the window once its X has landed too, so that the MMA issuer waits once
+        if (!__all_sync(0xffffffffu, mbar_wait(&full_x[X.slot], X.phase, abort_flag))) {
+          *abort_flag = 1;
+          stop = true;
+          break;
+        }
         tc_fence_before();
         mbar_arrive(&full_a[A.slot]);
         A.next(DT_AW);
+        X.next(xwin);
       }
     }
     tmem_wait_st();
@@ -468,8 +479,7 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_delta_tc(
         const uint32_t idesc = umma_idesc_f16(DT_BM, npad, false);
         const uint32_t d_tmem = tmem_base + (uint32_t)ab * DT_ACC_STRIDE;
         for (int win = 0; win < nwin; ++win) {
-          if (!mbar_wait(&full_x[X.slot], X.phase, abort_flag) ||
-              !mbar_wait(&full_a[A.slot], A.phase, abort_flag)) {
+          if (!mbar_wait(&full_a[A.slot], A.phase, abort_flag)) {
             *abort_flag = 1;
             stop = true;
             break;
@@ -489,8 +499,7 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_delta_tc(
               umma_f16_ts<1>(d_tmem, a0 + (uint32_t)((k / 4) * 32 + (k % 4) * 8),
                              b0 + (uint64_t)(((k / 4) * b_bytes + (k % 4) * 32) >> 4), idesc);
           }
-          umma_commit(&empty_a[A.slot]);
-          umma_commit(&empty_x[X.slot]);
+          umma_commit(&wdone[A.n % DT_WDONE]);  // frees this window's A and X slots
           A.next(DT_AW);
           X.next(xwin);
         }
@@ -515,7 +524,9 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_delta_tc(
           nxrow = sg.xrow[sn];
         }
         for (int win = 0; win < nwin; ++win) {
-          if (X.n >= xwin && !mbar_wait(&empty_x[X.slot], X.phase ^ 1u, abort_flag)) {
+          // the slot's previous fill (window X.n - xwin) must have been read by its MMAs
+          if (X.n >= xwin && !mbar_wait(&wdone[(X.n - xwin) % DT_WDONE],
+                                        (uint32_t)((X.n - xwin) / DT_WDONE) & 1u, abort_flag)) {
             *abort_flag = 1;
             stop = true;
             break;
@@ -607,7 +618,7 @@ static EncodeTiledFn2 get_encoder2() {
 size_t delta_tc_smem(int nmax, int xwin) {
   size_t need = 1024 + (size_t)xwin * DT_KPW * nmax * DT_BK * 2 +
                 (size_t)DT_WSLOTS * (DT_WIN_SIGN_BYTES + DT_WIN_SCALE_BYTES) +
-                (size_t)(2 * DT_XW_MAX + 2 * DT_AW + 2 * DT_WSLOTS + 5) * 8 + 16;
+                (size_t)(DT_XW_MAX + DT_WDONE + DT_AW + 2 * DT_WSLOTS + 5) * 8 + 16;
   // at least half of the SM's shared memory: one CTA per SM, so that the 512 tensor-memory
   // columns each CTA allocates never wait on a co-resident CTA
   return need < 120 * 1024 ? 120 * 1024 : need;
