@@ -587,13 +587,16 @@ __device__ __forceinline__ void lut_piece(const LutPiece& P, float (&acc)[LUT_NS
 #pragma unroll
     for (int sb = 0; sb < LUT_NSB; ++sb) {
       if (sb < nsb) {
+        // this stage's copies (the oldest group still pending) have landed for this thread;
+        // the barrier makes them visible to all and also tells that every warp is done with
+        // the previous stage, whose ring slot (bnext) is refilled right after it
+        cp_async_wait<LUT_STAGES - 2>();
+        __syncthreads();
         if (pw < nwin) {
           lut_stage(P, pw, ps, bnext, d_in, P.scale_f16 != 0, x, XBF16, nwin);
           if (++ps == nsb) { ps = 0; ++pw; }
         }
         cp_async_commit();
-        cp_async_wait<LUT_STAGES - 1>();
-        __syncthreads();
         if (sb == 0) {  // new window: build its tables from the staged x slice
           lut_build<XBF16>(P, win, bcur, d_in, P.scale_f16 != 0);
           __syncthreads();
@@ -644,7 +647,6 @@ __device__ __forceinline__ void lut_piece(const LutPiece& P, float (&acc)[LUT_NS
             }
           }
         }
-        __syncthreads();
         bcur = bcur + 1 == LUT_STAGES ? 0 : bcur + 1;
         bnext = bnext + 1 == LUT_STAGES ? 0 : bnext + 1;
       }
@@ -783,6 +785,8 @@ __global__ void __launch_bounds__(LUT_THREADS, 1) k_delta_lut(
       }
 #undef BD_PIECE
     }
+    // the staged results reuse the table page: every warp must be done with its lookups
+    __syncthreads();
     // ---- reduce the two lanes of each row, stage per-token results
 #pragma unroll
     for (int sb = 0; sb < LUT_NSB; ++sb) {
