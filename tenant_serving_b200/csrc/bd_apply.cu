@@ -944,15 +944,9 @@ bd_status apply_impl(const void* w_base, int32_t w_dtype, int64_t d_out, int64_t
 
   // 1. bucket tokens by tenant into groups
   const size_t bucket_smem = (size_t)(n_tenants + 1) * sizeof(int32_t);
-  static bool bucket_attr = false;
-  if (!bucket_attr) {
-    if (cudaFuncSetAttribute(k_tenant_bucket, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (kMaxTenants + 1) * (int)sizeof(int32_t)) != cudaSuccess) {
-      (void)cudaGetLastError();
-      return BD_ERR_CUDA;
-    }
-    bucket_attr = true;
-  }
+  static std::atomic<uint64_t> bucket_attr{0};
+  if (!ensure_dyn_smem(k_tenant_bucket, (kMaxTenants + 1) * (int)sizeof(int32_t), bucket_attr))
+    return BD_ERR_CUDA;
   launch_begin(K_TENANT_BUCKET, s);
   k_tenant_bucket<<<1, 1024, bucket_smem, s>>>(tenant_ids, (int)batch, n_tenants, L.max_groups,
                                                L.max_tc, tenants, kTcMinTokens, d_in, seg,
@@ -985,15 +979,9 @@ bd_status apply_impl(const void* w_base, int32_t w_dtype, int64_t d_out, int64_t
 
   // 4. lookup-table delta over the (token group, row) space, fused with the combine
   auto kfn = tc ? k_delta_lut<true> : k_delta_lut<false>;
-  static bool lut_attr[2] = {false, false};
-  if (!lut_attr[tc ? 1 : 0]) {
-    if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LUT_SMEM) !=
-        cudaSuccess) {
-      (void)cudaGetLastError();
-      return BD_ERR_CUDA;
-    }
-    lut_attr[tc ? 1 : 0] = true;
-  }
+  static std::atomic<uint64_t> lut_attr[2];
+  if (!ensure_dyn_smem(kfn, (int)LUT_SMEM, lut_attr[tc ? 1 : 0])) return BD_ERR_CUDA;
+
   launch_begin(K_DELTA_LUT, s);
   kfn<<<(unsigned)sm_count(), LUT_THREADS, LUT_SMEM, s>>>(tenants, scale_dtype == BD_F16, seg,
                                                          L.max_groups, L.max_tc, x, y_part, L.ksplit,

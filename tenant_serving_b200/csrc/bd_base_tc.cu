@@ -243,15 +243,9 @@ bd_status launch_base_tc(const TcPlan& p, const void* w_base, const void* x, int
   CUtensorMap tw, tx;
   if (!encode_bf16_2d(&tw, w_base, d_out, d_in, TC_BM)) return BD_ERR_CUDA;
   if (!encode_bf16_2d(&tx, x, batch, d_in, p.n_tile)) return BD_ERR_CUDA;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(k_base_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
-        cudaSuccess) {
-      (void)cudaGetLastError();
-      return BD_ERR_CUDA;
-    }
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_set{0};
+  if (!ensure_dyn_smem(k_base_tc, 227 * 1024, attr_set)) return BD_ERR_CUDA;
+
   if (p.tiles_m > 65535) return BD_ERR_SHAPE;  // row blocks run along grid y
   dim3 grid(p.tiles_n, p.tiles_m, p.ksplit);
   launch_begin(K_BASE_TC, s);

@@ -80,8 +80,9 @@ __global__ void __launch_bounds__(256) k_tc_gather(const int32_t* __restrict__ s
   }
   const int t = permv[tc_start[sidx] + r];
   const uint16_t* xt = x + (int64_t)t * d_in;
-  // largest |x| of the token
+  // largest |x| of the token (unrolled so that a lane's loads are in flight together)
   float m = 0.f;
+#pragma unroll 4
   for (int b = lane; b < nblk; b += 32) {
     const uint4* p = reinterpret_cast<const uint4*>(xt + 32 * b);
 #pragma unroll
@@ -102,6 +103,7 @@ __global__ void __launch_bounds__(256) k_tc_gather(const int32_t* __restrict__ s
     if (e > 126) e = 126;  // keep 2^e finite (tokens of only subnormal-sized values)
   }
   const float sc = ldexpf(1.f, e);
+#pragma unroll 2
   for (int b = lane; b < nblk; b += 32) {
     const uint4* p = reinterpret_cast<const uint4*>(xt + 32 * b);
     float v[32];
@@ -658,15 +660,9 @@ bd_status launch_delta_tc(const bd_tenant* tc_rec, const int32_t* seg, int max_g
   if (nmax > DT_NMAX) nmax = DT_NMAX;
   const int xwin = delta_tc_xwin(nmax);
   const size_t smem = delta_tc_smem(nmax, xwin);
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(k_delta_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
-        cudaSuccess) {
-      (void)cudaGetLastError();
-      return BD_ERR_CUDA;
-    }
-    attr = true;
-  }
+  static std::atomic<uint64_t> attr{0};
+  if (!ensure_dyn_smem(k_delta_tc, 227 * 1024, attr)) return BD_ERR_CUDA;
+
   const int64_t mtiles = (d_out + DT_BM - 1) / DT_BM;
   int64_t grid = (int64_t)sm_count();
   if (grid > mtiles * max_tc) grid = mtiles * max_tc;

@@ -1,6 +1,8 @@
 // Internal helpers shared by the library's translation units (not part of the ABI).
 #pragma once
 
+#include <atomic>
+
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -43,6 +45,26 @@ void launch_begin(int32_t kind, cudaStream_t s);
 void launch_end(int32_t kind, cudaStream_t s);
 
 int sm_count();  // multiprocessors of the current device (cached per device)
+
+// Lets `fn` use `bytes` of dynamic shared memory on the current device. The attribute is
+// per device, so it is set once per device (tracked in `done`, one bit per device
+// ordinal < 64; higher ordinals set it on every call). False on a CUDA error (cleared).
+template <typename F>
+inline bool ensure_dyn_smem(F* fn, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return false;
+  }
+  const uint64_t bit = dev < 64 ? (1ull << dev) : 0ull;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return true;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return false;
+  }
+  if (bit) done.fetch_or(bit, std::memory_order_release);
+  return true;
+}
 
 // Device status word, the first 16 bytes of every workspace.
 struct DevStatus {
