@@ -123,3 +123,12 @@ def test_selftest_wait_timeout_host_validation(lib):
     assert st(ctypes.c_void_p(0x1008), 256, 1000, None) == bd.BD_ERR_ALIGN
     assert st(fake, 256, 0, None) == bd.BD_ERR_CONFIG
     assert st(fake, 256, 5_000_000_000, None) == bd.BD_ERR_CONFIG
+
+
+def test_apply_limits(lib):
+    fake = ctypes.c_void_p(0x1000)
+    ap = lib.bd_apply_multi
+    # one past the largest batch and the largest tenant table
+    assert ap(fake, bd.BD_BF16, 8, 256, fake, 1, bd.BD_F16, fake, fake, 65537, fake, bd.BD_BF16, fake, 1 << 40, None) == bd.BD_ERR_SHAPE
+    assert ap(fake, bd.BD_BF16, 8, 256, fake, 16385, bd.BD_F16, fake, fake, 4, fake, bd.BD_BF16, fake, 1 << 40, None) == bd.BD_ERR_SHAPE
+    assert lib.bd_apply_workspace_size(8, 256, 65536, 16384) > 0

@@ -378,3 +378,46 @@ def test_many_token_f32_scales_use_lookup_path(bd):
     y, rc, flags = _run(bd, wb, tenants, ids, x, y_dtype="f32")
     assert rc == bd.BD_OK and flags == 0
     assert_apply_close(y, y_ref, tol=1e-5, per_token=True, what="delta only (fp32 out)")
+
+
+def test_max_batch_many_segments(bd):
+    """The largest batch the call accepts (65536 tokens): two tenants in the tiled layout
+    with 40000 and 20000 tokens (938 tensor-core segments), one with 5 tokens (lookup
+    table) and 5531 base-only tokens, shuffled."""
+    import torch
+    rng = np.random.default_rng(65536)
+    d_out, d_in = 128, 256
+    wb = bf16_bits(rng.normal(0, 0.02, size=(d_out, d_in)))
+    tenants = [random_tenant(rng, d_out, d_in, 0, 128) for _ in range(3)]
+    ids = np.concatenate([np.full(40000, 0), np.full(20000, 1), np.full(5, 2),
+                          np.full(65536 - 60005, -1)]).astype(np.int32)
+    rng.shuffle(ids)
+    x = activations(rng, len(ids), d_in)
+    y, rc, flags = _run(bd, wb, tenants, ids, x, y_dtype="f32", layout=1)
+    assert rc == bd.BD_OK and flags == 0
+    assert_apply_close(y, O.apply_multi(wb, "bf16", tenants, ids, x, "bf16"))
+
+
+def test_max_tenants(bd):
+    """The largest tenant table the call accepts (16384 records, one device buffer of
+    sign words and one of scales), 2048 tokens spread over it."""
+    import torch
+    rng = np.random.default_rng(16384)
+    d_out, d_in, T, B = 64, 256, 16384, 2048
+    wb = bf16_bits(rng.normal(0, 0.02, size=(d_out, d_in)))
+    words = rng.integers(0, 2 ** 32, size=(T, d_out, d_in // 32), dtype=np.uint64).astype(np.uint32)
+    z = rng.normal(0.0, 1.0, size=(T, d_out, d_in // 128))
+    scales = (0.001 * np.sqrt(2 / np.pi) * np.exp(0.1 * z)).astype(np.float16)
+    words_d, scales_d = dev(words), dev(scales)
+    recs = [(words_d[u], scales_d[u], 0, 128) for u in range(T)]
+    table = bd.TenantTable(recs, "cuda")
+    ids = rng.integers(-1, T, size=B).astype(np.int32)
+    x = activations(rng, B, d_in)
+    y, ws = bd.bd_apply_multi(dev(wb), table, dev(ids), dev(x), y_dtype=torch.float32)
+    assert bd.bd_get_status(ws) == (bd.BD_OK, 0)
+    used = sorted(set(int(u) for u in ids if u >= 0))
+    ref_t = [{"signs": words[u], "scales": scales[u], "scale_dtype": "f16", "mode": 0,
+              "group_size": 128} for u in used]
+    remap = {u: i for i, u in enumerate(used)}
+    ids_ref = np.array([remap[int(u)] if u >= 0 else -1 for u in ids], dtype=np.int32)
+    assert_apply_close(host(y), O.apply_multi(wb, "bf16", ref_t, ids_ref, x, "bf16"))
