@@ -164,3 +164,25 @@ def test_compress_then_reconstruct_validation_threshold(bd):
     rec = host(bd.bd_reconstruct(signs, scales, bd.BD_SCALE_GROUP, 128, 256, 512))
     d = O.delta(wb, wf)
     assert np.abs(rec - d).mean() < GOLD["validation_threshold"]["max_mean_abs_error"]
+
+
+@pytest.mark.parametrize("clip", [False, True])
+def test_bf16_llama_gate_full_sampled(bd, clip):
+    """The bench's compress configuration on its largest matrix: gate_proj 14336 x 4096
+    bf16, group 128, with and without the 3-sigma clip. The clip statistics are checked
+    over the whole matrix; signs (bit-exact) and scales on 256 sampled rows."""
+    d_out, d_in = 14336, 4096
+    wb, wf = weight_pair(14336, d_out, d_in, "bf16")
+    signs, scales, stats = _gpu_compress(bd, wb, wf, "bf16", O.MODE_GROUP, 128, clip, 3.0)
+    d = O.delta(O.decode(wb, "bf16"), O.decode(wf, "bf16"))
+    rows = np.sort(np.random.default_rng(3).choice(d_out, 256, replace=False))
+    dr = d[rows]
+    if clip:
+        m, s, lo, hi = O.clip_stats(d, 3.0)
+        assert abs(stats[0] - m) <= 1e-9 * max(1.0, abs(m)) + 1e-12 * s
+        assert abs(stats[1] - s) <= 1e-9 * s
+        dr = O.clip(dr, lo, hi)
+    ref_scales = O.abs_mean_scales(dr, O.MODE_GROUP, 128)
+    ref_signs = O.pack_bits(O.sign_bits(dr))
+    np.testing.assert_array_equal(signs.reshape(d_out, d_in // 32)[rows], ref_signs)
+    assert_scales_close(scales.reshape(d_out, d_in // 128)[rows], ref_scales)
