@@ -4,24 +4,27 @@
 // per-tenant delta product) and "2. Fused Dequantization ..." (sign bits stay packed in
 // HBM and are expanded on chip). The pages give no kernel for this GPU; the design here:
 //
-//   k_tenant_bucket  one CTA: counting sort of the tenant ids, every tenant's tokens cut
-//                    into groups of <= 2 (tenant, start, length) plus a token
-//                    permutation. Invalid ids set a status bit and join the base-only
-//                    tokens. No host synchronisation.
+//   k_tenant_bucket  one CTA: counting sort of the tenant ids and the token permutation.
+//                    A tenant with enough tokens (and a record the tensor-core kernel
+//                    supports) gets segments of <= kTcSegTokens tokens for k_delta_tc;
+//                    every other tenant's tokens, and the base-only ones, are cut into
+//                    groups of <= 2 for k_delta_lut. Invalid ids set a status bit and
+//                    join the base-only tokens. No host synchronisation.
 //   base product     bf16: tcgen05 tensor-core GEMM (bd_base_tc.cu), fp32: k_base_gemv.
 //                    Both write fp32 partial sums y_part[kz][t][row].
-//   k_delta_lut      persistent CTAs split the (token group, row) space evenly; groups
-//                    of one tenant are adjacent in it, so its sign words come from HBM
-//                    once and from L2 for the other groups. A CTA streams the
-//                    words through shared memory 256 columns at a time and, per token,
-//                    turns every byte of signs into ONE table lookup: for each 8-column
-//                    chunk a 256-entry table holds sum_j (+/-) x_j for every sign
-//                    pattern (built per window from two 16-entry nibble tables). The
-//                    lookup order is rotated by row so the 32 lanes of a warp always hit
-//                    32 different banks. Group scales multiply per 32-bit word, column
-//                    scales are folded into x before the tables are built, row / tensor
-//                    scales multiply at the end. The epilogue adds the base partial sums
-//                    in a fixed order and writes y (bf16 or fp32) in request order.
+//   k_delta_tc       (bd_delta_tc.cu) the many-token tenants' delta as a tcgen05
+//                    contraction with the +/-s matrix expanded into tensor memory.
+//   k_delta_lut      persistent CTAs split the (token group, 512-row tile) space evenly.
+//                    A CTA streams the tenant's sign words through shared memory 256
+//                    columns at a time and, per token, turns every byte of signs into ONE
+//                    table lookup: for each 8-column chunk a 256-entry table holds
+//                    sum_j (+/-) x_j for every sign pattern (built per window from two
+//                    16-entry nibble tables). The lookup order is rotated by row so the
+//                    lanes of a warp hit distinct banks. Group-128 scales multiply once per
+//                    128 columns, column scales are folded into x before the tables are
+//                    built, row / tensor scales multiply at the end.
+//   Both delta kernels add the base partial sums in a fixed order and write y (bf16 or
+//   fp32) in request order.
 #include "bd_internal.cuh"
 
 namespace bd {
@@ -240,10 +243,10 @@ __global__ void __launch_bounds__(256) k_base_gemv_f32(const float* __restrict__
 // ------------------------------------------------------------------------------------
 // delta product with per-chunk sign lookup tables
 // ------------------------------------------------------------------------------------
-// Persistent CTAs (one per SM, 32 warps) split the flattened (token group, output row)
+// Persistent CTAs (one per SM, 8 warps) split the flattened (token group, 512-row tile)
 // space evenly; a CTA walks its share in pieces of at most 2048 rows of one group
-// (<= 2 tokens of one tenant). Groups of one tenant are adjacent in that space, so the
-// CTAs working on a tenant run at the same time and its sign words come from HBM once.
+// (<= 2 tokens of one tenant). A tenant split over several groups has its sign words
+// streamed once per group.
 //
 // A piece streams the tenant's sign words 256 columns (8 words) x 512 rows per stage
 // through a 6-deep cp.async ring. Per 256-column window and token, a table
