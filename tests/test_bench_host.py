@@ -41,3 +41,19 @@ def test_fused_layer_has_the_projection_rows():
     from workloads import LLAMA3_8B_FUSED, LLAMA3_8B_PROJECTIONS
     rows = lambda t: sum(o * i for _, o, i in t)  # noqa: E731
     assert rows(LLAMA3_8B_FUSED) == rows(LLAMA3_8B_PROJECTIONS)
+
+
+def test_cpu_baseline_sample_is_bounded_and_positive():
+    import time
+    t0 = time.perf_counter()
+    value, cores, desc = bench.oracle_sample(0.2)
+    assert value > 0 and cores >= 1 and "oracle" in desc
+    assert time.perf_counter() - t0 < 60
+
+
+def test_both_arms_report_the_same_config():
+    class A:  # the fields serving_config reads
+        layers, tenants, batch = 32, 100, 512
+    cfg = bench.serving_config(A, 1)
+    assert cfg["batch"] == 512 and cfg["tenants"] == 100 and "fused" in cfg["workload"]
+    assert bench.serving_config(A, 8)["parallelism"] == "replicas x8"
