@@ -45,6 +45,7 @@ N_TENANTS = 100
 BATCH = 512
 GROUP = 128
 ZIPF_S = 1.1
+COMPRESS_STREAMS = 4  # compress calls of the stack are spread over this many streams
 TC_MIN_TOKENS = 6  # the library's many-token threshold (tensor-core delta from this count on)
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum, mean over the 4
@@ -457,9 +458,25 @@ def bench_compress(args, log, peaks):
                              dtype=torch.uint8, device="cuda")
             bufs.append((signs, scales, ws))
 
+        # the matrices are independent: calls go round-robin to COMPRESS_STREAMS streams
+        # (each with its own workspace), so a small matrix's launch ramp and tail overlap
+        # another matrix's kernels; the main stream waits for all of them
+        main_s = torch.cuda.current_stream()
+        streams = [torch.cuda.Stream() for _ in range(COMPRESS_STREAMS)]
+
         def one_pass():
-            for (d_out, d_in, wb, wf), (signs, scales, ws) in zip(mats, bufs):
-                bd.bd_compress(wb, wf, cfg, signs=signs, scales=scales, workspace=ws)
+            start = torch.cuda.Event()
+            start.record(main_s)
+            for st in streams:
+                st.wait_event(start)
+            for i, ((d_out, d_in, wb, wf), (signs, scales, ws)) in enumerate(zip(mats, bufs)):
+                st = streams[i % len(streams)]
+                bd.bd_compress(wb, wf, cfg, signs=signs, scales=scales, workspace=ws,
+                               stream=st)
+            for st in streams:
+                done = torch.cuda.Event()
+                done.record(st)
+                main_s.wait_event(done)
 
         for _ in range(2):
             one_pass()
@@ -468,10 +485,10 @@ def bench_compress(args, log, peaks):
         bd.bd_profile_enable(True, capacity=len(mats) * reps * 8 + 16)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
-        e0.record()
+        e0.record(main_s)
         for _ in range(reps):
             one_pass()
-        e1.record()
+        e1.record(main_s)
         torch.cuda.synchronize()
         prof = bd.bd_profile_collect()
         bd.bd_profile_enable(False)
@@ -481,6 +498,7 @@ def bench_compress(args, log, peaks):
         main = prof.get("scale_signpack", (0, 0.0))
         main_gbs = alg * reps / (main[1] / 1e3) / 1e9 if main[1] else None
         out[label] = {"ms_per_stack": ms, "params": params, "gbs": gbs, "frac": gbs / peaks[0],
+                      "streams": COMPRESS_STREAMS,
                       "tparams_per_s": params / (ms / 1e3) / 1e12,
                       "kernels": {k: {"launches": v[0], "total_ms": v[1] / reps} for k, v in prof.items()},
                       "signpack_kernel_gbs": main_gbs}
