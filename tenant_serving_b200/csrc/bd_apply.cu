@@ -861,7 +861,9 @@ bd_status launch_delta_tc(const bd_tenant* tenants, const int32_t* seg, int max_
                           bool y_bf16, uint32_t* status, cudaStream_t s);
 
 // A tenant with at least this many tokens in a batch (and a supported record) goes to the
-// tensor-core delta kernel; below it the lookup-table kernel is cheaper per token.
+// tensor-core delta kernel; below it the lookup-table kernel is cheaper per token (6 is
+// the crossover measured on B200; both kernels compute the same product, so a build may
+// set another value with -DBD_TC_MIN_TOKENS=n, n >= 1, to re-tune it).
 #ifndef BD_TC_MIN_TOKENS
 #define BD_TC_MIN_TOKENS 6
 #endif
