@@ -502,10 +502,53 @@ def bench_compress(args, log, peaks):
                       "tparams_per_s": params / (ms / 1e3) / 1e12,
                       "kernels": {k: {"launches": v[0], "total_ms": v[1] / reps} for k, v in prof.items()},
                       "signpack_kernel_gbs": main_gbs}
+        if not clip:
+            out["reconstruct_merged"] = _bench_reconstruct(bd, mats, bufs, streams, main_s,
+                                                           params, peaks)
         del bufs
     del mats
     torch.cuda.empty_cache()
     return out
+
+
+def _bench_reconstruct(bd, mats, bufs, streams, main_s, params, peaks):
+    """The merged weight W_u = W_base + Delta_hat of every matrix of the stack, in bf16,
+    from the signs and scales compress just wrote (bd_reconstruct with w_base). Same
+    stream arrangement as compress; one reused output buffer per stream."""
+    import torch
+    biggest = max(d_out * d_in for d_out, d_in, _, _ in mats)
+    outs = [torch.empty(biggest, dtype=torch.bfloat16, device="cuda") for _ in streams]
+
+    def one_pass():
+        start = torch.cuda.Event()
+        start.record(main_s)
+        for st in streams:
+            st.wait_event(start)
+        for i, ((d_out, d_in, wb, wf), (signs, scales, ws)) in enumerate(zip(mats, bufs)):
+            k = i % len(streams)
+            bd.bd_reconstruct(signs, scales, bd.BD_SCALE_GROUP, GROUP, d_out, d_in, w_base=wb,
+                              out=outs[k][: d_out * d_in].view(d_out, d_in), stream=streams[k])
+        for st in streams:
+            done = torch.cuda.Event()
+            done.record(st)
+            main_s.wait_event(done)
+
+    for _ in range(2):
+        one_pass()
+    torch.cuda.synchronize()
+    reps = 3
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(main_s)
+    for _ in range(reps):
+        one_pass()
+    e1.record(main_s)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    # sign bits + fp32 group scales + bf16 W_base read, bf16 W_u written
+    alg = params * (1 / 8 + 4 / GROUP + 2 + 2)
+    gbs = alg / (ms / 1e3) / 1e9
+    return {"ms_per_stack": ms, "gbs": gbs, "frac": gbs / peaks[0], "streams": len(streams)}
 
 
 # ------------------------------------------------------------------------------------
