@@ -46,15 +46,22 @@ BATCH = 512
 GROUP = 128
 ZIPF_S = 1.1
 COMPRESS_STREAMS = 4  # compress calls of the stack are spread over this many streams
-TC_MIN_TOKENS = 6  # the library's many-token threshold (tensor-core delta from this count on)
 
-# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum, mean over the 4
-# fused calls of a layer) from the ncu capture in profiles/delta_lut_serving_layer.md,
-# keyed by the hash of the sources the kernel was built from: once they change the
-# number no longer describes the kernel and the roofline reports traffic = null.
+
+def tc_min_tokens() -> int:
+    """The library's many-token threshold (tensor-core delta from this token count on),
+    read from the built library so that the byte accounting follows the build."""
+    import tenant_serving_b200 as bd
+    return bd.bd_tc_min_tokens()
+
+
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of a kernel from
+# an ncu capture summarised under profiles/, keyed by the hash of the sources the kernel
+# was built from: once they change, the number no longer describes the kernel and the
+# roofline reports traffic = null.
 NCU_TRAFFIC = {
-    "delta_lut": {"sources": ["bd_apply.cu", "bd_internal.cuh"], "sha256_16": "c6fbd2335af22e5b",
-                  "bytes_per_launch": 642.6e6},
+    "delta_lut": {"sources": ["bd_delta_lut.cu", "bd_internal.cuh", "bd_tc.cuh"],
+                  "sha256_16": "0000000000000000", "bytes_per_launch": None},
 }
 
 
@@ -342,9 +349,10 @@ def bench_serving(args, rank, pg, log, peaks):
     ms_prof = max_over_ranks(pg, f0.elapsed_time(f1))
 
     # algorithmic bytes of the timed steps. The planner sends a tenant with at least
-    # TC_MIN_TOKENS tokens in the batch (all tenants here are tiled, fp16, group 128) to the
+    # tc_min tokens in the batch (all tenants here are tiled, fp16, group 128) to the
     # tensor-core delta kernel and the others to the lookup-table kernel; each delta kernel
     # is charged the sign words + scales of its tenants and the y rows of its tokens.
+    tc_min = tc_min_tokens()
     base_bytes = sum(d_out * d_in * 2 for _, d_out, d_in in LLAMA3_8B_FUSED) * args.layers
     base_flops_per_token = sum(2 * d_out * d_in for _, d_out, d_in in LLAMA3_8B_FUSED) * args.layers
     delta_bytes_per_tenant = sum(d_out * d_in // 8 + d_out * (d_in // GROUP) * 2
@@ -356,7 +364,7 @@ def bench_serving(args, rank, pg, log, peaks):
     for s in range(args.warmup, steps_total):
         cnt = np.bincount(ids_host[s], minlength=args.tenants)
         d = int((cnt > 0).sum())
-        big = cnt >= TC_MIN_TOKENS
+        big = cnt >= tc_min
         step_bytes.append(base_bytes + d * delta_bytes_per_tenant + io_bytes)
         tc_bytes += int(big.sum()) * delta_bytes_per_tenant + int(cnt[big].sum()) * y_bytes_per_token
         small = (cnt > 0) & ~big

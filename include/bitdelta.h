@@ -204,6 +204,12 @@ bd_status bd_prepare_tenant(const uint32_t* signs, const void* scales, int32_t s
                             int32_t mode, int32_t group_size, int64_t d_out, int64_t d_in,
                             uint32_t* signs_out, void* scales_out, void* stream);
 
+/* The many-token threshold built into the library: a tenant with at least this many
+ * tokens in a batch (and a record the tensor-core path supports) goes to the tensor-core
+ * delta; every other tenant goes through the lookup-table delta, at most 4 of its tokens
+ * per pass over its bits. */
+int32_t bd_tc_min_tokens(void);
+
 /* Bytes of workspace bd_apply_multi needs. */
 size_t bd_apply_workspace_size(int64_t d_out, int64_t d_in, int64_t batch, int32_t n_tenants);
 
@@ -214,13 +220,15 @@ size_t bd_apply_workspace_size(int64_t d_out, int64_t d_in, int64_t batch, int32
  * The base product W_base X is computed once for the whole batch; the tokens are
  * grouped by tenant on the device (no host synchronisation). Two delta kernels share the
  * work, chosen per tenant on the device:
- *   - a tenant with at least 6 tokens in the batch, stored in the TILED layout with
+ *   - a tenant with at least bd_tc_min_tokens() tokens in the batch (5 as built),
+ *     stored in the TILED layout with
  *     fp16 scales in GROUP (group_size >= 64), ROW or TENSOR mode (bf16 w_base and
  *     d_in % 64 == 0), is a dense product on the tensor cores, in segments of <= 64 of
  *     its tokens; its activations are scaled per token by a power of two into fp16 for
  *     that product (exact for bf16 values in fp16's normal range);
  *   - every other tenant goes through the sign lookup-table kernel, its packed signs and
- *     scales streamed once per group of <= 2 of its tokens.
+ *     scales streamed once per group of <= 4 of its tokens (once in all when it has at
+ *     most 4 tokens in the batch).
  *
  *   w_base      : [d_out][d_in], w_dtype BD_BF16 (tensor-core path) or BD_F32.
  *   tenants     : device array of n_tenants bd_tenant records (n_tenants >= 0).

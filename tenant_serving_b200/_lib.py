@@ -39,6 +39,7 @@ EXPORTS = (
     "bd_apply_multi", "bd_prepared_signs_bytes", "bd_prepared_scales_bytes", "bd_prepare_tenant",
     "bd_apply_workspace_size", "bd_get_status", "bd_status_string", "bd_launch_count",
     "bd_profile_enable", "bd_profile_collect", "bd_kernel_name", "bd_selftest_wait_timeout",
+    "bd_tc_min_tokens",
 )
 
 
@@ -109,6 +110,8 @@ def lib():
     L.bd_kernel_name.restype = ctypes.c_char_p
     L.bd_selftest_wait_timeout.argtypes = [c_void_p, c_size_t, c_int64, c_void_p]
     L.bd_selftest_wait_timeout.restype = c_int32
+    L.bd_tc_min_tokens.argtypes = []
+    L.bd_tc_min_tokens.restype = c_int32
     _LIB = L
     return L
 
@@ -310,6 +313,11 @@ def bd_get_status(workspace, stream=None):
     f = c_uint32(0)
     rc = lib().bd_get_status(_ptr(workspace), ctypes.byref(f), _stream(stream))
     return int(rc), int(f.value)
+
+
+def bd_tc_min_tokens() -> int:
+    """The library's many-token threshold (tensor-core delta from this token count on)."""
+    return int(lib().bd_tc_min_tokens())
 
 
 def bd_launch_count() -> int:

@@ -8,21 +8,15 @@
 //                    A tenant with enough tokens (and a record the tensor-core kernel
 //                    supports) gets segments of <= kTcSegTokens tokens for k_delta_tc;
 //                    every other tenant's tokens, and the base-only ones, are cut into
-//                    groups of <= 2 for k_delta_lut. Invalid ids set a status bit and
-//                    join the base-only tokens. No host synchronisation.
+//                    lookup groups of <= 4 for k_delta_lut. Invalid ids set a status bit
+//                    and join the base-only tokens. No host synchronisation.
 //   base product     bf16: tcgen05 tensor-core GEMM (bd_base_tc.cu), fp32: k_base_gemv.
 //                    Both write fp32 partial sums y_part[kz][t][row].
 //   k_delta_tc       (bd_delta_tc.cu) the many-token tenants' delta as a tcgen05
 //                    contraction with the +/-s matrix expanded into tensor memory.
-//   k_delta_lut      persistent CTAs split the (token group, 512-row tile) space evenly.
-//                    A CTA streams the tenant's sign words through shared memory 256
-//                    columns at a time and, per token, turns every byte of signs into ONE
-//                    table lookup: for each 8-column chunk a 256-entry table holds
-//                    sum_j (+/-) x_j for every sign pattern (built per window from two
-//                    16-entry nibble tables). The lookup order is rotated by row so the
-//                    lanes of a warp hit distinct banks. Group-128 scales multiply once per
-//                    128 columns, column scales are folded into x before the tables are
-//                    built, row / tensor scales multiply at the end.
+//   k_delta_lut      (bd_delta_lut.cu) the few-token tenants' delta through per-chunk
+//                    sign lookup tables in shared memory, all tokens of a group served by
+//                    one pass over the tenant's bits.
 //   Both delta kernels add the base partial sums in a fixed order and write y (bf16 or
 //   fp32) in request order.
 #include "bd_internal.cuh"
@@ -42,22 +36,23 @@ constexpr int kMaxTenants = 16384;
 constexpr int kMaxBatch = 65536;
 
 // ------------------------------------------------------------------------------------
-// planning: token groups for the lookup-table kernel, segments for the tensor-core one
+// planning: lookup groups for the lookup-table kernel, segments for the tensor-core one
 // ------------------------------------------------------------------------------------
 // Tokens are grouped by tenant (a counting sort). A tenant with at least tc_min tokens
-// whose record the tensor-core path supports gets tensor-core segments of <= kTcSegTokens tokens;
-// every other tenant's tokens (and the base-only tokens) are cut into lookup-table groups
-// of <= kGroupTokens.
-// Workspace layout (int32): [0] n_groups, [1] n_tc, [2..3] pad, grp_tenant[max_groups],
+// whose record the tensor-core path supports gets tensor-core segments of <= kTcSegTokens
+// tokens; every other tenant's tokens are cut into lookup groups of <= kLutTokens (one pass
+// over the tenant's bits per group), and the base-only tokens into groups of the same size.
+// Groups are numbered by class: all groups of 4 tokens first, then 3, 2, 1, then the
+// base-only groups, so that the lookup kernel meets one kind of group for long stretches.
+// Workspace layout (int32): the kSegHeader words, grp_tenant[max_groups],
 // grp_start[max_groups], grp_len[max_groups], tc_tenant[max_tc], tc_start[max_tc],
-// tc_count[max_tc], tc_xrow[max_tc] (first row in the gathered X), perm[batch]; and, in
-// a region of its own, a copy of each tensor-core segment's tenant record.
-constexpr int kGroupTokens = 2;
+// tc_count[max_tc], tc_xrow[max_tc] (first row in the gathered X), perm[batch]; and, in a
+// region of its own, a copy of each tensor-core segment's tenant record.
 constexpr int kTcMaxTokens = kTcSegTokens;
 
 inline int max_groups_for(int64_t batch, int32_t n_tenants) {
   const int64_t keys = batch < (int64_t)n_tenants + 1 ? batch : (int64_t)n_tenants + 1;
-  return (int)((batch + kGroupTokens - 1) / kGroupTokens + keys);
+  return (int)((batch + kLutTokens - 1) / kLutTokens + keys);
 }
 
 __device__ __forceinline__ bool tc_eligible(const bd_tenant& T, int64_t d_in) {
@@ -70,6 +65,8 @@ __device__ __forceinline__ bool tc_eligible(const bd_tenant& T, int64_t d_in) {
   return mode_ok && ptr_ok && T.layout == BD_LAYOUT_TILED && T.reserved == 0;
 }
 
+constexpr int kPlanQ = 3 + kLutClasses;  // tokens, tc segments, gathered X rows, groups per class
+
 __global__ void __launch_bounds__(1024) k_tenant_bucket(const int32_t* __restrict__ ids, int batch,
                                                         int n_tenants, int max_groups, int max_tc,
                                                         const bd_tenant* __restrict__ tenants,
@@ -78,10 +75,10 @@ __global__ void __launch_bounds__(1024) k_tenant_bucket(const int32_t* __restric
                                                         bd_tenant* __restrict__ tc_rec,
                                                         uint32_t* __restrict__ status) {
   extern __shared__ int32_t cnt[];  // n_tenants + 1 counters (last = base only)
-  __shared__ int32_t wsum[5][32];
+  __shared__ int32_t wsum[kPlanQ][32];
   __shared__ int32_t bad;
   const int nkeys = n_tenants + 1;
-  int32_t* grp_tenant = seg_base + 4;
+  int32_t* grp_tenant = seg_base + kSegHeader;
   int32_t* grp_start = grp_tenant + max_groups;
   int32_t* grp_len = grp_start + max_groups;
   int32_t* tc_tenant = grp_len + max_groups;
@@ -104,52 +101,57 @@ __global__ void __launch_bounds__(1024) k_tenant_bucket(const int32_t* __restric
     atomicAdd(&cnt[u < 0 ? n_tenants : u], 1);
   }
   __syncthreads();
-  // per key: tokens, full lookup groups (kGroupTokens tokens), remainder groups, tensor-core
-  // segments, gathered-X rows. All full groups are numbered before all remainder groups,
-  // so that the lookup-table kernel meets one kind of group for long stretches.
-  auto plan = [&](int k, int c, int& ng, int& nr, int& nt, int& nx) {
-    ng = nr = nt = nx = 0;
+  // per key: q[0] tokens, q[1] tensor-core segments, q[2] gathered-X rows, q[3 + k] lookup
+  // groups of class k (k = 0..3: tenant groups of 4 - k tokens; k = 4: base-only groups)
+  auto plan = [&](int k, int c, int (&q)[kPlanQ]) {
+#pragma unroll
+    for (int i = 0; i < kPlanQ; ++i) q[i] = 0;
+    q[0] = c;
     if (c == 0) return;
     const bool tc = max_tc > 0 && k < n_tenants && c >= tc_min && tc_eligible(tenants[k], d_in);
     if (tc) {
-      nt = (c + kTcMaxTokens - 1) / kTcMaxTokens;
-      for (int j = 0; j < c; j += kTcMaxTokens) nx += (min(kTcMaxTokens, c - j) + 15) & ~15;
+      q[1] = (c + kTcMaxTokens - 1) / kTcMaxTokens;
+      for (int j = 0; j < c; j += kTcMaxTokens) q[2] += (min(kTcMaxTokens, c - j) + 15) & ~15;
+    } else if (k == n_tenants) {
+      q[3 + 4] = (c + kLutTokens - 1) / kLutTokens;
     } else {
-      ng = c / kGroupTokens;
-      nr = (c % kGroupTokens) ? 1 : 0;
+      q[3 + 0] = c / kLutTokens;
+      const int rem = c % kLutTokens;
+      if (rem) q[3 + (kLutTokens - rem)] = 1;
     }
   };
   const int per = (nkeys + blockDim.x - 1) / blockDim.x;
   const int k0 = threadIdx.x * per, k1 = min(nkeys, k0 + per);
-  int v[5] = {0, 0, 0, 0, 0};  // tokens, full groups, tc segments, X rows, remainder groups
+  int v[kPlanQ];
+#pragma unroll
+  for (int i = 0; i < kPlanQ; ++i) v[i] = 0;
   for (int k = k0; k < k1; ++k) {
-    int ng, nr, nt, nx;
-    plan(k, cnt[k], ng, nr, nt, nx);
-    v[0] += cnt[k];
-    v[1] += ng;
-    v[2] += nt;
-    v[3] += nx;
-    v[4] += nr;
+    int q[kPlanQ];
+    plan(k, cnt[k], q);
+#pragma unroll
+    for (int i = 0; i < kPlanQ; ++i) v[i] += q[i];
   }
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  int inc[5] = {v[0], v[1], v[2], v[3], v[4]};
+  int inc[kPlanQ];
+#pragma unroll
+  for (int i = 0; i < kPlanQ; ++i) inc[i] = v[i];
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
 #pragma unroll
-    for (int i = 0; i < 5; ++i) {
+    for (int i = 0; i < kPlanQ; ++i) {
       const int a = __shfl_up_sync(0xffffffffu, inc[i], o);
       if (lane >= o) inc[i] += a;
     }
   }
   if (lane == 31) {
 #pragma unroll
-    for (int i = 0; i < 5; ++i) wsum[i][w] = inc[i];
+    for (int i = 0; i < kPlanQ; ++i) wsum[i][w] = inc[i];
   }
   __syncthreads();
   if (w == 0) {
     const int nw = blockDim.x >> 5;
 #pragma unroll
-    for (int i = 0; i < 5; ++i) {
+    for (int i = 0; i < kPlanQ; ++i) {
       int a = lane < nw ? wsum[i][lane] : 0;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -160,17 +162,23 @@ __global__ void __launch_bounds__(1024) k_tenant_bucket(const int32_t* __restric
     }
   }
   __syncthreads();
-  int off = inc[0] - v[0] + (w > 0 ? wsum[0][w - 1] : 0);
-  int gidx = inc[1] - v[1] + (w > 0 ? wsum[1][w - 1] : 0);
-  int tidx = inc[2] - v[2] + (w > 0 ? wsum[2][w - 1] : 0);
-  int xrow = inc[3] - v[3] + (w > 0 ? wsum[3][w - 1] : 0);
-  const int n_full = wsum[1][(blockDim.x >> 5) - 1];  // all full groups come first
-  int ridx = n_full + inc[4] - v[4] + (w > 0 ? wsum[4][w - 1] : 0);
+  const int last = (blockDim.x >> 5) - 1;
+  int ex[kPlanQ];  // this thread's exclusive prefix of each quantity
+#pragma unroll
+  for (int i = 0; i < kPlanQ; ++i) ex[i] = inc[i] - v[i] + (w > 0 ? wsum[i][w - 1] : 0);
+  int off = ex[0], tidx = ex[1], xrow = ex[2];
+  int gnext[kLutClasses];  // next group index of each class
+  int cstart = 0;
+#pragma unroll
+  for (int k = 0; k < kLutClasses; ++k) {
+    gnext[k] = cstart + ex[3 + k];
+    cstart += wsum[3 + k][last];
+  }
   for (int k = k0; k < k1; ++k) {
     const int c = cnt[k];
-    int ng, nr, nt, nx;
-    plan(k, c, ng, nr, nt, nx);
-    if (nt > 0) {
+    int q[kPlanQ];
+    plan(k, c, q);
+    if (q[1] > 0) {
       for (int j = 0; j < c; j += kTcMaxTokens) {
         const int n = min(kTcMaxTokens, c - j);
         tc_tenant[tidx] = k;
@@ -182,20 +190,24 @@ __global__ void __launch_bounds__(1024) k_tenant_bucket(const int32_t* __restric
         ++tidx;
       }
     } else {
-      for (int j = 0; j < c; j += kGroupTokens) {
-        const bool full = c - j >= kGroupTokens;
-        const int gi = full ? gidx++ : ridx++;
+      for (int j = 0; j < c; j += kLutTokens) {
+        const int len = min(kLutTokens, c - j);
+        const int cls = k == n_tenants ? 4 : kLutTokens - len;
+        const int gi = gnext[cls]++;
         grp_tenant[gi] = (k == n_tenants) ? -1 : k;
         grp_start[gi] = off + j;
-        grp_len[gi] = min(kGroupTokens, c - j);
+        grp_len[gi] = len;
       }
     }
     cnt[k] = off;  // becomes the scatter cursor
     off += c;
   }
   if (threadIdx.x == blockDim.x - 1) {  // the last thread holds the totals
-    seg_base[0] = ridx;
+    seg_base[0] = cstart;
     seg_base[1] = tidx;
+#pragma unroll
+    for (int k = 0; k < kLutClasses; ++k) seg_base[2 + k] = wsum[3 + k][last];
+    seg_base[2 + kLutClasses] = 0;
   }
   __syncthreads();
   for (int t = threadIdx.x; t < batch; t += blockDim.x) {
@@ -241,633 +253,28 @@ __global__ void __launch_bounds__(256) k_base_gemv_f32(const float* __restrict__
 }
 
 // ------------------------------------------------------------------------------------
-// delta product with per-chunk sign lookup tables
-// ------------------------------------------------------------------------------------
-// Persistent CTAs (one per SM, 8 warps) split the flattened (token group, 512-row tile)
-// space evenly; a CTA walks its share in pieces of at most 2048 rows of one group
-// (<= 2 tokens of one tenant). A tenant split over several groups has its sign words
-// streamed once per group.
-//
-// A piece streams the tenant's sign words 256 columns (8 words) x 512 rows per stage
-// through a 6-deep cp.async ring. Per 256-column window and token, a table
-// T[v][c] = sum_j (bit j of v ? +x : -x)[8c + j] over the 8 columns of chunk c is built
-// in shared memory for every sign byte v; then one byte of signs costs one table read
-// per token.
-//   lanes: q = lane >> 1 picks one of 16 rows, wp = lane & 1 one half of the window
-//   (words 4wp..4wp+3). At step (k, j) a lane reads word 4wp + ((k + q/4 + 2wp) & 3)
-//   and its byte (j + q) & 3: the 32 lanes read 32 different staged words (32 banks),
-//   and each half-warp reads 16 different table chunks modulo 16.
-//   table page: it sits at shared address 0x10000. For a 2-token group entry
-//   (v, chunk, token) is at 0x10000 + v * 256 + 8 * chunk + 4 * token: the two tokens sit
-//   side by side, one 8-byte ld.shared returns both, and each half-warp's 16 lanes cover
-//   the 32 banks once. For a 1-token group entry (v, chunk) is at 0x10000 + v * 256 +
-//   4 * chunk, and the 32 lanes' 4-byte reads cover the 32 banks once. One PRMT of the
-//   sign word with the lane's slot constant (entry stride x chunk, plus the 0x1 of
-//   0x10000 in its upper half) yields the whole 32-bit shared address of the entry.
-//   A lookup is PRMT + ld.shared(.v2) + FADD per token.
-//   Group-128 scales are one per lane per row (words 4wp..4wp+3 are one group) and are
-//   staged next to the sign words.
-constexpr int LUT_THREADS = 256;    // 8 warps, 64 rows each per stage
-constexpr int LUT_RG = 4;           // 16-row groups per warp per stage
-constexpr int LUT_WARPS = LUT_THREADS / 32;
-constexpr int LUT_W = 256;          // columns per window
-constexpr int LUT_SB = 512;         // rows per stage: one 16-row slice per warp
-constexpr int LUT_NSB = 4;          // stages (sub-blocks) per window of a piece
-constexpr int LUT_PASS = LUT_SB * LUT_NSB;  // rows per piece
-constexpr int LUT_STAGES = 6;       // cp.async ring depth
-constexpr int LUT_SC = 8;           // staged scale bytes per row per window
-constexpr uint32_t LUT_BITS_STAGE = LUT_SB * 32;
-constexpr uint32_t LUT_SC_STAGE = LUT_SB * LUT_SC;
-constexpr uint32_t LUT_ADDR = 0x10000;  // shared address of the table page
-constexpr uint32_t LUT_HALF = 3 * (LUT_BITS_STAGE + LUT_SC_STAGE);  // ring stages below / above
-constexpr uint32_t LUT_LOW = LUT_ADDR - LUT_HALF;    // first ring byte; dynamic smem must start <=
-constexpr uint32_t LUT_X_STAGE = 4096;  // per ring slot: x of 2 tokens + column scales
-constexpr uint32_t LUT_XBASE = 0x20000 + LUT_HALF;   // x slots of the ring
-constexpr uint32_t LUT_PIECE = LUT_XBASE + LUT_STAGES * LUT_X_STAGE;  // piece descriptor
-constexpr size_t LUT_SMEM = LUT_PIECE + 128;  // requested from the dynamic base
-
-__device__ __forceinline__ uint32_t sh_addr(const void* p) {
-  return (uint32_t)__cvta_generic_to_shared(p);
-}
-__device__ __forceinline__ float lds_f32(uint32_t a) {
-  float v;
-  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
-  return v;
-}
-__device__ __forceinline__ float2 lds_f32x2(uint32_t a) {
-  float2 v;
-  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a));
-  return v;
-}
-__device__ __forceinline__ void sts_f32x2(uint32_t a, float x, float y) {
-  asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(a), "f"(x), "f"(y) : "memory");
-}
-__device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
-  uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
-  return v;
-}
-__device__ __forceinline__ float lds_f16(uint32_t a) {
-  unsigned short v;
-  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
-  return __half2float(__ushort_as_half(v));
-}
-__device__ __forceinline__ void sts_f32(uint32_t a, float v) {
-  asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
-}
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-__device__ __forceinline__ float ld_scale(const void* s, bool f16, int64_t i) {
-  return f16 ? __half2float(reinterpret_cast<const __half*>(s)[i]) : reinterpret_cast<const float*>(s)[i];
-}
-
-struct LutPiece {
-  bd_tenant T;
-  int u, mode, G, ntok, t0, t1, rows, sc_kind, layout, pos_step, scale_f16;
-  int64_t rb0;      // first 512-row tile of the piece
-  int64_t r0;
-  int64_t bstride;  // sign words between consecutive 512-row stages
-  int64_t half_stride;  // sign words between rows r and r + 256
-  int64_t sstride;  // staged-scale bytes between consecutive stages
-  int whole;
-};
-
-__device__ __forceinline__ uint32_t lut_bits_stage(int b) {
-  return b < 3 ? LUT_LOW + (uint32_t)b * LUT_BITS_STAGE
-               : 0x20000u + (uint32_t)(b - 3) * LUT_BITS_STAGE;
-}
-__device__ __forceinline__ uint32_t lut_sc_stage(int b) {
-  return b < 3 ? LUT_LOW + 3 * LUT_BITS_STAGE + (uint32_t)b * LUT_SC_STAGE
-               : 0x20000u + 3 * LUT_BITS_STAGE + (uint32_t)(b - 3) * LUT_SC_STAGE;
-}
-
-__device__ __forceinline__ uint32_t lut_x_stage(int b) { return LUT_XBASE + (uint32_t)b * LUT_X_STAGE; }
-
-// Issue the copies of stage (win, sb) into ring buffer b. Staged scales are 2 per row
-// (2 * ssz bytes, row stride 2 * ssz).
-__device__ __forceinline__ void lut_stage(const LutPiece& P, int win, int sb,
-                                          int b, int64_t d_in, bool scale_f16, const void* x,
-                                          bool xbf16, int nwin) {
-  const int tid = threadIdx.x;
-  const int rb = sb * LUT_SB;
-  const int ssz = scale_f16 ? 2 : 4;
-  if (P.layout == BD_LAYOUT_TILED) {
-    // one contiguous 16 KB tile of sign words and (group-128) a 2 / 4 KB tile of scales
-    const int64_t tile = (P.rb0 + sb) * nwin + win;
-    const uint32_t* src = P.T.signs + tile * 4096;
-#pragma unroll
-    for (int c = 0; c < 1024; c += LUT_THREADS)
-      cp_async16(lut_bits_stage(b) + (uint32_t)(c + tid) * 16u, src + (c + tid) * 4);
-    if (P.sc_kind == 1) {
-      const uint8_t* ssrc = reinterpret_cast<const uint8_t*>(P.T.scales) + tile * 1024 * ssz;
-      for (int c = tid; c * 16 < 1024 * ssz; c += LUT_THREADS)
-        cp_async16(lut_sc_stage(b) + (uint32_t)c * 16u, ssrc + c * 16);
-    }
-  } else {
-    if (P.whole) {
-      // two 16-byte copies per thread: rows tid/2 and tid/2 + 256 of the stage, half tid & 1
-      const int64_t wpr = d_in >> 5;
-      // 16-byte copies: copy c = row (c >> 1), half (c & 1) of the stage
-      for (int c = tid; c < 1024; c += LUT_THREADS) {
-        const int row = c >> 1;
-        if (rb + row < P.rows)
-          cp_async16(lut_bits_stage(b) + (uint32_t)c * 16u,
-                     P.T.signs + (P.r0 + rb + row) * wpr + (c & 1) * 4 + win * 8);
-      }
-    } else {
-      const int64_t wpr = d_in >> 5;
-      const int64_t w0 = (int64_t)win * (LUT_W / 32);
-      const int nr = min(LUT_SB, P.rows - rb);
-      const uint32_t* src = P.T.signs + (P.r0 + rb) * wpr + w0;
-      for (int i = tid; i < nr * 8; i += LUT_THREADS) {
-        const int rl = i >> 3, k = i & 7;
-        if (w0 + k < wpr) cp_async4(lut_bits_stage(b) + rl * 32 + k * 4, src + rl * wpr + k);
-      }
-    }
-    if (P.sc_kind == 1) {
-      const int64_t per_row = (d_in / 128) * ssz;
-      for (int r = tid; r < LUT_SB && rb + r < P.rows; r += LUT_THREADS) {
-        const uint8_t* sp = reinterpret_cast<const uint8_t*>(P.T.scales) + (P.r0 + rb + r) * per_row +
-                            win * 2 * ssz;
-        const uint32_t sd = lut_sc_stage(b) + (uint32_t)(r * 2 * ssz);
-        if (scale_f16) cp_async4(sd, sp);
-        else cp_async8(sd, sp);
-      }
-    }
-  }
-  // the first stage of a window also brings the window's slice of x (both tokens) and,
-  // for column scales, the window's scales: [x0 1 KB][x1 1 KB][col scales 1 KB]
-  if (sb == 0 && tid < 3 * 64) {
-    const int part = tid >> 6, k = tid & 63;  // 64 x 16 B per part (LUT_THREADS >= 192)
-    const int64_t col0 = (int64_t)win * LUT_W;
-    const int xb = xbf16 ? 2 : 4;
-    const uint32_t dst = lut_x_stage(b) + (uint32_t)(part * 1024 + k * 16);
-    if (part < 2) {
-      const int64_t col = col0 + (int64_t)k * (16 / xb);
-      if (part < P.ntok && k * 16 < LUT_W * xb && col < d_in) {
-        const int t = part == 0 ? P.t0 : P.t1;
-        cp_async16(dst, reinterpret_cast<const uint8_t*>(x) + ((int64_t)t * d_in + col) * xb);
-      }
-    } else if (P.mode == BD_SCALE_COL) {
-      const int64_t col = col0 + (int64_t)k * (16 / ssz);
-      if (k * 16 < LUT_W * ssz && col < d_in)
-        cp_async16(dst, reinterpret_cast<const uint8_t*>(P.T.scales) + col * ssz);
-    }
-  }
-}
-
-// Build the sign tables of one window for the piece's tokens from the x slice (and
-// column scales) staged in ring slot b.
-template <bool XBF16>
-__device__ __forceinline__ void lut_build(const LutPiece& P, int win, int b, int64_t d_in,
-                                          bool scale_f16) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int c = lane;  // chunk of the window
-  // this thread fills the sign patterns with high nibble h and h + 8 (h = warp, 8 warps)
-  const int64_t col = (int64_t)win * LUT_W + 8 * c;
-  const uint32_t xs = lut_x_stage(b);
-  float sc[8];
-  if (P.mode == BD_SCALE_COL) {
-    if (scale_f16) {
-      uint4 v;
-      asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                   : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(xs + 2048 + 16 * c));
-      const uint32_t a[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const __half2 hh = *reinterpret_cast<const __half2*>(&a[k]);
-        sc[2 * k] = __low2float(hh);
-        sc[2 * k + 1] = __high2float(hh);
-      }
-    } else {
-#pragma unroll
-      for (int k = 0; k < 8; ++k) sc[k] = lds_f32(xs + 2048 + 32 * c + 4 * k);
-    }
-  }
-  // both tokens' 16 low-nibble sums (a second token of 0 for single-token groups)
-  float lo16[2][16];
-  float xv[2][8];
-#pragma unroll
-  for (int tt = 0; tt < 2; ++tt) {
-    if (tt < P.ntok && col < d_in) {
-      if (XBF16) {
-        uint4 v;
-        asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                     : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                     : "r"(xs + 1024 * tt + 16 * c));
-        const uint32_t a[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          xv[tt][2 * k] = bf16lo(a[k]);
-          xv[tt][2 * k + 1] = bf16hi(a[k]);
-        }
-      } else {
-#pragma unroll
-        for (int k = 0; k < 8; ++k) xv[tt][k] = lds_f32(xs + 1024 * tt + 32 * c + 4 * k);
-      }
-      if (P.mode == BD_SCALE_COL) {
-#pragma unroll
-        for (int k = 0; k < 8; ++k) xv[tt][k] *= sc[k];
-      }
-    } else {
-#pragma unroll
-      for (int k = 0; k < 8; ++k) xv[tt][k] = 0.f;
-    }
-    float p01[4], p23[4];
-#pragma unroll
-    for (int n = 0; n < 4; ++n) {
-      p01[n] = ((n & 1) ? xv[tt][0] : -xv[tt][0]) + ((n & 2) ? xv[tt][1] : -xv[tt][1]);
-      p23[n] = ((n & 1) ? xv[tt][2] : -xv[tt][2]) + ((n & 2) ? xv[tt][3] : -xv[tt][3]);
-    }
-#pragma unroll
-    for (int lo = 0; lo < 16; ++lo) lo16[tt][lo] = p01[lo & 3] + p23[lo >> 2];
-  }
-#pragma unroll
-  for (int hh = 0; hh < 2; ++hh) {
-    const int h = warp + 8 * hh;
-    float hi[2];
-#pragma unroll
-    for (int tt = 0; tt < 2; ++tt)
-      hi[tt] = (((h & 1) ? xv[tt][4] : -xv[tt][4]) + ((h & 2) ? xv[tt][5] : -xv[tt][5])) +
-               (((h & 4) ? xv[tt][6] : -xv[tt][6]) + ((h & 8) ? xv[tt][7] : -xv[tt][7]));
-    if (P.ntok == 2) {
-      const uint32_t base = LUT_ADDR + (uint32_t)(h << 12) + 8u * (uint32_t)c;
-#pragma unroll
-      for (int lo = 0; lo < 16; ++lo)
-        sts_f32x2(base + (uint32_t)lo * 256u, lo16[0][lo] + hi[0], lo16[1][lo] + hi[1]);
-    } else {
-      const uint32_t base = LUT_ADDR + (uint32_t)(h << 12) + 4u * (uint32_t)c;
-#pragma unroll
-      for (int lo = 0; lo < 16; ++lo) sts_f32(base + (uint32_t)lo * 256u, lo16[0][lo] + hi[0]);
-    }
-  }
-}
-
-// Generic path: group sizes other than 128 (one scale per word from global memory) and
-// windows that run past d_in. Recomputes the lane constants itself (slow path).
-template <int NT>
-__device__ __forceinline__ float2 lut_rows_generic(uint32_t wrow, uint32_t srow, const LutPiece& P,
-                                                int sb, int i, int win, int64_t d_in,
-                                                bool scale_f16) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int q = lane >> 1, wp = lane & 1;
-  const int rl = sb * LUT_SB + warp * (16 * LUT_RG) + i * 16 + q;  // row inside the piece
-  float a0 = 0.f, a1 = 0.f;
-  if (rl >= P.rows) return make_float2(0.f, 0.f);
-#pragma unroll 1
-  for (int k = 0; k < 4; ++k) {
-    const int wi = 4 * wp + ((k + (q >> 2) + 2 * wp) & 3);
-    const int64_t col = (int64_t)win * LUT_W + 32 * wi;
-    if (col >= d_in) continue;
-    const uint32_t word = lds_u32(wrow + 4u * (uint32_t)wi);
-    float p0 = 0.f, p1 = 0.f;
-    for (int j = 0; j < 4; ++j) {
-      const int b = (j + q) & 3;
-      const uint32_t idx = LUT_ADDR + (((word >> (8 * b)) & 0xFFu) << 8) +
-                           (NT == 2 ? 8u : 4u) * (uint32_t)(4 * wi + b);
-      p0 += lds_f32(idx);
-      if (NT == 2) p1 += lds_f32(idx + 4u);
-    }
-    float sw = 1.f;
-    if (P.sc_kind == 1) {  // staged group-128 scales: group (wi >> 2) of the window
-      const uint32_t a = srow + (uint32_t)((wi >> 2) * (scale_f16 ? 2 : 4));
-      sw = scale_f16 ? lds_f16(a) : lds_f32(a);
-    } else if (P.sc_kind == 2) {
-      sw = ld_scale(P.T.scales, scale_f16, (P.r0 + rl) * (d_in / P.G) + col / P.G);
-    }
-    a0 = fmaf(sw, p0, a0);
-    if (NT == 2) a1 = fmaf(sw, p1, a1);
-  }
-  return make_float2(a0, a1);
-}
-
-// The stage loop of one piece. SC: 0 = no per-word scale (row / col / tensor modes, or
-// the generic path, which handles scales itself), 1 = staged fp16 group-128 scales,
-// 2 = staged fp32 group-128 scales. GENERIC: group sizes other than 128 or a last window
-// that runs past d_in.
-template <bool XBF16, int NT, int SC, bool GENERIC>
-__device__ __forceinline__ void lut_piece(const LutPiece& P, float (&acc)[LUT_NSB][LUT_RG][2], int nwin,
-                                          int64_t d_in, const void* x, const uint32_t (&sel)[4],
-                                          const uint32_t (&slot2)[4][2], const uint32_t (&wofs)[4],
-                                          int warp, int q, int wp) {
-  const bool f16s = P.scale_f16 != 0;
-  const int ssz = GENERIC ? (f16s ? 2 : 4) : (SC == 2 ? 4 : 2);
-  // 2-token tables have 8-byte entries: the slot bytes (entry stride x chunk, <= 124 for
-  // the 4-byte stride) double, the 0x1 of 0x10000 in the upper half stays
-  uint32_t sl[4][2];
-#pragma unroll
-  for (int k = 0; k < 4; ++k)
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh)
-      sl[k][hh] = NT == 2 ? (((slot2[k][hh] & 0xFFFFu) << 1) | (slot2[k][hh] & 0xFFFF0000u))
-                          : slot2[k][hh];
-  const int rows = P.rows;
-  const int nsb = (rows + LUT_SB - 1) / LUT_SB;  // 1..4
-  int pw = 0, ps = 0;
-#pragma unroll
-  for (int i = 0; i < LUT_STAGES - 1; ++i) {
-    if (pw < nwin) {
-      lut_stage(P, pw, ps, i, d_in, P.scale_f16 != 0, x, XBF16, nwin);
-      if (++ps == nsb) { ps = 0; ++pw; }
-    }
-    cp_async_commit();
-  }
-  int bcur = 0, bnext = LUT_STAGES - 1;
-  for (int win = 0; win < nwin; ++win) {
-#pragma unroll
-    for (int sb = 0; sb < LUT_NSB; ++sb) {
-      if (sb < nsb) {
-        // this stage's copies (the oldest group still pending) have landed for this thread;
-        // the barrier makes them visible to all and also tells that every warp is done with
-        // the previous stage, whose ring slot (bnext) is refilled right after it
-        cp_async_wait<LUT_STAGES - 2>();
-        __syncthreads();
-        if (pw < nwin) {
-          lut_stage(P, pw, ps, bnext, d_in, P.scale_f16 != 0, x, XBF16, nwin);
-          if (++ps == nsb) { ps = 0; ++pw; }
-        }
-        cp_async_commit();
-        if (sb == 0) {  // new window: build its tables from the staged x slice
-          lut_build<XBF16>(P, win, bcur, d_in, P.scale_f16 != 0);
-          __syncthreads();
-        }
-#pragma unroll
-        for (int i = 0; i < LUT_RG; ++i) {  // the warp's 16-row groups of this stage
-          const int rs = warp * (16 * LUT_RG) + i * 16;  // first row of the group in the stage
-          const uint32_t wrow = lut_bits_stage(bcur) + (uint32_t)((rs + q) * 32);
-          // the fast path runs every row group unconditionally (no branch, so the groups'
-          // loads interleave); rows past the piece read stale staging data and their
-          // results are never written out
-          if (!GENERIC || sb * LUT_SB + rs < rows) {
-            if (!GENERIC) {
-              float s_ = 1.f;
-              if (SC != 0) {
-                const uint32_t sa = lut_sc_stage(bcur) + (uint32_t)((rs + q) * 2 * ssz + wp * ssz);
-                s_ = SC == 1 ? lds_f16(sa) : lds_f32(sa);
-              }
-              // 16 independent table reads per token, summed as a tree (depth 4)
-              uint32_t wd[4];
-#pragma unroll
-              for (int k = 0; k < 4; ++k) wd[k] = lds_u32(wrow + wofs[k]);
-              float w0[4], w1[4];
-#pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                float v0[4], v1[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                  const uint32_t idx = __byte_perm(wd[k], sl[k][j >> 1], sel[j]);
-                  if (NT == 2) {
-                    const float2 e = lds_f32x2(idx);
-                    v0[j] = e.x;
-                    v1[j] = e.y;
-                  } else {
-                    v0[j] = lds_f32(idx);
-                  }
-                }
-                w0[k] = (v0[0] + v0[1]) + (v0[2] + v0[3]);
-                if (NT == 2) w1[k] = (v1[0] + v1[1]) + (v1[2] + v1[3]);
-              }
-              acc[sb][i][0] = fmaf(s_, (w0[0] + w0[1]) + (w0[2] + w0[3]), acc[sb][i][0]);
-              if (NT == 2) acc[sb][i][1] = fmaf(s_, (w1[0] + w1[1]) + (w1[2] + w1[3]), acc[sb][i][1]);
-            } else {
-              const uint32_t srow = lut_sc_stage(bcur) + (uint32_t)((rs + q) * 2 * ssz);
-              const float2 r = lut_rows_generic<NT>(wrow, srow, P, sb, i, win, d_in, f16s);
-              acc[sb][i][0] += r.x;
-              acc[sb][i][1] += r.y;
-            }
-          }
-        }
-        bcur = bcur + 1 == LUT_STAGES ? 0 : bcur + 1;
-        bnext = bnext + 1 == LUT_STAGES ? 0 : bnext + 1;
-      }
-    }
-  }
-}
-
-// Per-lane lookup constants (see the comment above k_delta_lut's lookup loop).
-__device__ __forceinline__ void lut_lane_constants(int q, int wp, uint32_t estride, uint32_t (&sel)[4],
-                                                   uint32_t (&slot2)[4][2], uint32_t (&wofs)[4]) {
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int b = (j + q) & 3;
-    sel[j] = 0x7600u | ((uint32_t)b << 4) | (uint32_t)(4 + (j & 1));
-  }
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int wi = 4 * wp + ((k + (q >> 2) + 2 * wp) & 3);
-    wofs[k] = 4u * (uint32_t)wi;
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const uint32_t s0 = estride * (uint32_t)(4 * wi + ((2 * hh + q) & 3));
-      const uint32_t s1 = estride * (uint32_t)(4 * wi + ((2 * hh + 1 + q) & 3));
-      slot2[k][hh] = s0 | (s1 << 8) | (LUT_ADDR & 0xFFFF0000u);
-    }
-  }
-}
-
-template <bool XBF16>
-__global__ void __launch_bounds__(LUT_THREADS, 1) k_delta_lut(
-    const bd_tenant* __restrict__ tenants, bool scale_f16, const int32_t* __restrict__ seg_base,
-    int max_groups, int max_tc, const void* __restrict__ x, const float* __restrict__ y_part,
-    int ksplit, int64_t d_out, int64_t d_in, int batch, void* __restrict__ y, bool y_bf16,
-    uint32_t* __restrict__ status) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  const uint32_t base = sh_addr(smem);
-  if (base > LUT_LOW) {  // the fixed layout needs the dynamic window to start low enough
-    if (threadIdx.x == 0) atomicOr(status, BD_DEV_INTERNAL);
-    return;
-  }
-  LutPiece& piece = *reinterpret_cast<LutPiece*>(smem + (LUT_PIECE - base));
-  float* out_s = reinterpret_cast<float*>(smem + (LUT_ADDR - base));  // after the last window
-
-  const int32_t* grp_tenant = seg_base + 4;
-  const int32_t* grp_start = grp_tenant + max_groups;
-  const int32_t* grp_len = grp_start + max_groups;
-  const int32_t* perm = grp_len + max_groups + 4 * max_tc;
-  // the (token group, 512-row tile) space is split evenly over the CTAs; a piece is up to
-  // LUT_NSB consecutive tiles of one group
-  const int n_groups = seg_base[0];
-  const int64_t n_rt = (d_out + LUT_SB - 1) / LUT_SB;
-  const int64_t total = (int64_t)n_groups * n_rt;
-  const int64_t share = (total + gridDim.x - 1) / gridDim.x;
-  int64_t pos = (int64_t)blockIdx.x * share;
-  const int64_t end = min(total, pos + share);
-
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int q = lane >> 1, wp = lane & 1;
-  const int nwin = (int)((d_in + LUT_W - 1) / LUT_W);
-  // per-lane lookup constants. sel[j]: byte 0 <- slot byte (j & 1) of slot2[k][j >> 1],
-  // byte 1 <- sign byte (j + q) & 3, bytes 2-3 <- 0x0001 (the table's 0x10000).
-  uint32_t sel[4], slot2[4][2], wofs[4];
-  lut_lane_constants(q, wp, 4u, sel, slot2, wofs);  // 1-token entry stride; lut_piece doubles it
-
-  while (pos < end) {
-    if (tid == 0) {
-      LutPiece Q;
-      const int g = (int)(pos / n_rt);
-      Q.rb0 = pos - (int64_t)g * n_rt;
-      const int64_t ntiles = min((int64_t)LUT_NSB, min(n_rt - Q.rb0, end - pos));
-      Q.r0 = Q.rb0 * LUT_SB;
-      Q.rows = (int)min(ntiles * LUT_SB, d_out - Q.r0);
-      Q.pos_step = (int)ntiles;
-      Q.u = grp_tenant[g];
-      Q.ntok = grp_len[g];
-      Q.t0 = perm[grp_start[g]];
-      Q.t1 = Q.ntok > 1 ? perm[grp_start[g] + 1] : Q.t0;
-      Q.mode = BD_SCALE_GROUP;
-      Q.G = 128;
-      Q.T.signs = nullptr;
-      Q.T.scales = nullptr;
-      if (Q.u >= 0) {
-        Q.T = tenants[Q.u];
-        Q.mode = Q.T.mode;
-        Q.G = Q.T.group_size;
-        // the table lives in device memory, so its records are checked here
-        const bool ok_mode = Q.mode >= BD_SCALE_GROUP && Q.mode <= BD_SCALE_TENSOR;
-        const bool ok_group = Q.mode != BD_SCALE_GROUP ||
-                              (Q.G >= 32 && (Q.G & (Q.G - 1)) == 0 && (d_in % Q.G) == 0);
-        const bool ok_ptr = Q.T.signs != nullptr && Q.T.scales != nullptr &&
-                            ((reinterpret_cast<uintptr_t>(Q.T.signs) |
-                              reinterpret_cast<uintptr_t>(Q.T.scales)) & 15u) == 0;
-        const bool ok_layout = (Q.T.layout == BD_LAYOUT_ROWMAJOR || Q.T.layout == BD_LAYOUT_TILED) &&
-                               Q.T.reserved == 0;
-        if (!(ok_mode && ok_group && ok_ptr && ok_layout)) {
-          atomicOr(status, BD_DEV_TENANT_RECORD);
-          Q.u = -1;  // base product only
-        }
-      }
-      Q.whole = (d_in % LUT_W) == 0;
-      Q.layout = Q.u >= 0 ? Q.T.layout : BD_LAYOUT_ROWMAJOR;
-      // 0: no per-word scale; 1: staged group-128 scales (tiled, or row-major with whole
-      // windows); 2: group scales read from global memory per word
-      Q.sc_kind = Q.mode != BD_SCALE_GROUP
-                      ? 0
-                      : ((Q.G == 128 && (Q.whole || Q.layout == BD_LAYOUT_TILED)) ? 1 : 2);
-      Q.scale_f16 = scale_f16 ? 1 : 0;
-      Q.bstride = (int64_t)LUT_SB * (d_in >> 5);
-      Q.half_stride = (int64_t)256 * (d_in >> 5);
-      Q.sstride = (int64_t)LUT_SB * (d_in / 128) * (scale_f16 ? 2 : 4);
-      piece = Q;
-    }
-    __syncthreads();
-    const LutPiece& P = piece;
-    pos += P.pos_step;
-
-    float acc[LUT_NSB][LUT_RG][2];  // [sub-block][16-row group][token]
-#pragma unroll
-    for (int i = 0; i < LUT_NSB; ++i)
-#pragma unroll
-      for (int j = 0; j < LUT_RG; ++j) acc[i][j][0] = acc[i][j][1] = 0.f;
-
-    if (P.u >= 0) {
-      // one specialised stage loop per (tokens, scale kind, path), chosen once per piece
-      const bool generic = P.sc_kind == 2 || !P.whole;
-      const int ntok = P.ntok;
-#define BD_PIECE(NT, SC, GEN) \
-  lut_piece<XBF16, NT, SC, GEN>(P, acc, nwin, d_in, x, sel, slot2, wofs, warp, q, wp)
-      if (generic) {
-        if (ntok == 2) BD_PIECE(2, 0, true); else BD_PIECE(1, 0, true);
-      } else if (P.sc_kind == 1) {
-        if (scale_f16) { if (ntok == 2) BD_PIECE(2, 1, false); else BD_PIECE(1, 1, false); }
-        else { if (ntok == 2) BD_PIECE(2, 2, false); else BD_PIECE(1, 2, false); }
-      } else {
-        if (ntok == 2) BD_PIECE(2, 0, false); else BD_PIECE(1, 0, false);
-      }
-#undef BD_PIECE
-    }
-    // the staged results reuse the table page: every warp must be done with its lookups
-    __syncthreads();
-    // ---- reduce the two lanes of each row, stage per-token results
-#pragma unroll
-    for (int sb = 0; sb < LUT_NSB; ++sb) {
-#pragma unroll
-      for (int i = 0; i < LUT_RG; ++i) {
-#pragma unroll
-        for (int tt = 0; tt < 2; ++tt) {
-          const float v = acc[sb][i][tt] + __shfl_xor_sync(0xffffffffu, acc[sb][i][tt], 1);
-          const int rl = sb * LUT_SB + warp * (16 * LUT_RG) + i * 16 + q;
-          if (wp == 0) out_s[tt * LUT_PASS + rl] = v;
-        }
-      }
-    }
-    __syncthreads();
-    // ---- combine with the base product, write y in request order
-    // each thread owns up to LUT_RPT rows x 2 tokens; the split-K partials of all of them
-    // are loaded together (independent loads) before any is added
-    constexpr int LUT_RPT = (LUT_PASS + LUT_THREADS - 1) / LUT_THREADS;
-    float rs = 1.f;
-    if (P.u >= 0 && P.mode == BD_SCALE_TENSOR) rs = ld_scale(P.T.scales, scale_f16, 0);
-    float bsum[2][LUT_RPT];
-#pragma unroll
-    for (int tt = 0; tt < 2; ++tt)
-#pragma unroll
-      for (int k = 0; k < LUT_RPT; ++k) bsum[tt][k] = 0.f;
-    for (int kz = 0; kz < ksplit; ++kz) {
-      const float* part = y_part + (int64_t)kz * batch * d_out + P.r0 + tid;
-#pragma unroll
-      for (int tt = 0; tt < 2; ++tt) {
-        const int t = tt == 0 ? P.t0 : P.t1;
-#pragma unroll
-        for (int k = 0; k < LUT_RPT; ++k)
-          if (tt < P.ntok && tid + k * LUT_THREADS < P.rows)
-            bsum[tt][k] += part[(int64_t)t * d_out + k * LUT_THREADS];
-      }
-    }
-#pragma unroll
-    for (int tt = 0; tt < 2; ++tt) {
-      const int t = tt == 0 ? P.t0 : P.t1;
-#pragma unroll
-      for (int k = 0; k < LUT_RPT; ++k) {
-        const int rl = tid + k * LUT_THREADS;
-        if (tt < P.ntok && rl < P.rows) {
-          const int64_t row = P.r0 + rl;
-          float d = 0.f;
-          if (P.u >= 0) {
-            float sc = rs;
-            if (P.mode == BD_SCALE_ROW) sc = ld_scale(P.T.scales, scale_f16, row);
-            d = sc * out_s[tt * LUT_PASS + rl];
-          }
-          const float v = bsum[tt][k] + d;
-          if (y_bf16)
-            reinterpret_cast<uint16_t*>(y)[(int64_t)t * d_out + row] = (uint16_t)f2bf_bits(v);
-          else
-            reinterpret_cast<float*>(y)[(int64_t)t * d_out + row] = v;
-        }
-      }
-    }
-    __syncthreads();
-  }
-}
-
-// ------------------------------------------------------------------------------------
 // host side
 // ------------------------------------------------------------------------------------
 bd_status launch_delta_tc(const bd_tenant* tenants, const int32_t* seg, int max_groups, int max_tc,
                           const void* x, int64_t d_out, int64_t d_in, int64_t batch, __half* xg,
                           int64_t xg_rows, float* xinv, const float* y_part, int ksplit, void* y,
                           bool y_bf16, uint32_t* status, cudaStream_t s);
+bd_status launch_delta_lut(bool xbf16, const bd_tenant* tenants, bool scale_f16, const int32_t* seg,
+                           int max_groups, int max_tc, const void* x, const float* y_part, int ksplit,
+                           int64_t d_out, int64_t d_in, int64_t batch, void* y, bool y_bf16,
+                           uint32_t* status, cudaStream_t s);
 
 // A tenant with at least this many tokens in a batch (and a supported record) goes to the
-// tensor-core delta kernel; below it the lookup-table kernel is cheaper per token (6 is
-// the crossover measured on B200; both kernels compute the same product, so a build may
-// set another value with -DBD_TC_MIN_TOKENS=n, n >= 1, to re-tune it).
+// tensor-core delta kernel; below it the lookup-table kernel serves all of the tenant's
+// tokens (at most kLutTokens) in one pass over its bits. Both kernels compute the same
+// product, so a build may set another value with -DBD_TC_MIN_TOKENS=n, 1 <= n <= 5, to
+// re-tune it; bd_tc_min_tokens() reports the value built in.
 #ifndef BD_TC_MIN_TOKENS
-#define BD_TC_MIN_TOKENS 6
+#define BD_TC_MIN_TOKENS 5
 #endif
 constexpr int kTcMinTokens = BD_TC_MIN_TOKENS;
+static_assert(kTcMinTokens >= 1 && kTcMinTokens <= kLutTokens + 1,
+              "lookup groups hold at most kLutTokens tokens of a tenant");
 
 namespace {
 struct ApplyLayout {
@@ -899,7 +306,7 @@ ApplyLayout layout_apply(int64_t d_out, int64_t d_in, int64_t batch, int32_t n_t
   }
   size_t off = kStatusBytes;
   L.off_seg = off;
-  off = align_up(off + (16 + 3 * (size_t)L.max_groups * 4 + 4 * (size_t)L.max_tc * 4 + (size_t)batch * 4), 256);
+  off = align_up(off + (kSegHeader * 4 + 3 * (size_t)L.max_groups * 4 + 4 * (size_t)L.max_tc * 4 + (size_t)batch * 4), 256);
   L.off_tcrec = off;
   off = align_up(off + (size_t)L.max_tc * sizeof(bd_tenant), 256);
   L.off_part = off;
@@ -982,22 +389,14 @@ bd_status apply_impl(const void* w_base, int32_t w_dtype, int64_t d_out, int64_t
     if (st != BD_OK) return st;
   }
 
-  // 4. lookup-table delta over the (token group, row) space, fused with the combine
-  auto kfn = tc ? k_delta_lut<true> : k_delta_lut<false>;
-  static std::atomic<uint64_t> lut_attr[2];
-  if (!ensure_dyn_smem(kfn, (int)LUT_SMEM, lut_attr[tc ? 1 : 0])) return BD_ERR_CUDA;
-
-  launch_begin(K_DELTA_LUT, s);
-  kfn<<<(unsigned)sm_count(), LUT_THREADS, LUT_SMEM, s>>>(tenants, scale_dtype == BD_F16, seg,
-                                                         L.max_groups, L.max_tc, x, y_part, L.ksplit,
-                                                         d_out, d_in, (int)batch, y,
-                                                         y_dtype == BD_BF16, status);
-  launch_end(K_DELTA_LUT, s);
-  BD_LAUNCH_CHECK();
-  return BD_OK;
+  // 4. lookup-table delta over the (lookup group, row tile) space, fused with the combine
+  return launch_delta_lut(tc, tenants, scale_dtype == BD_F16, seg, L.max_groups, L.max_tc, x, y_part,
+                          L.ksplit, d_out, d_in, batch, y, y_dtype == BD_BF16, status, s);
 }
 
 }  // namespace bd
+
+extern "C" int32_t bd_tc_min_tokens(void) { return bd::kTcMinTokens; }
 
 extern "C" size_t bd_apply_workspace_size(int64_t d_out, int64_t d_in, int64_t batch,
                                           int32_t n_tenants) {

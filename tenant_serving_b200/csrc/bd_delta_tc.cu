@@ -57,7 +57,7 @@ __global__ void __launch_bounds__(256) k_tc_gather(const int32_t* __restrict__ s
   const int n_tc = seg_base[1];
   const int sidx = blockIdx.y;
   if (sidx >= n_tc) return;
-  const int32_t* tc = seg_base + 4 + 3 * max_groups;  // tc_tenant, then the arrays below
+  const int32_t* tc = seg_base + kSegHeader + 3 * max_groups;  // tc_tenant, then the arrays below
   const int32_t* tc_start = tc + max_tc;
   const int32_t* tc_count = tc_start + max_tc;
   const int32_t* tc_xrow = tc_count + max_tc;
@@ -138,18 +138,6 @@ __global__ void __launch_bounds__(256) k_tc_gather(const int32_t* __restrict__ s
 // ------------------------------------------------------------------------------------
 // Persistent: work item = (segment, 128-row tile), items dealt round-robin to the CTAs.
 // All rings run across items.
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-// Bulk copy global -> shared (no tensor map, no multicast), completing on `bar`.
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
 
 // 32 lanes x 16 consecutive 32-bit columns of tensor memory from 16 registers per thread.
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* v) {
@@ -192,7 +180,7 @@ struct TcSegs {
 };
 __device__ __forceinline__ TcSegs tc_segs(const int32_t* seg_base, int max_groups, int max_tc) {
   TcSegs g;
-  const int32_t* tenant = seg_base + 4 + 3 * max_groups;
+  const int32_t* tenant = seg_base + kSegHeader + 3 * max_groups;
   g.start = tenant + max_tc;
   g.count = g.start + max_tc;
   g.xrow = g.count + max_tc;

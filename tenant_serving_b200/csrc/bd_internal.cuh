@@ -19,9 +19,15 @@ namespace bd {
 // window of a segment's activations at 32 KB, so four windows fit the shared-memory ring.
 constexpr int kTcSegTokens = 64;
 
+// Plan written by the tenant-bucket kernel into the apply workspace (int32 words):
+// [0] lookup groups, [1] tensor-core segments, [2..6] lookup groups per class (NT = 4, 3,
+// 2, 1 tokens of a tenant, then base-only groups), [7] unused; then the arrays.
+constexpr int kSegHeader = 8;
+constexpr int kLutTokens = 4;   // tokens of one tenant served by one pass of the lookup kernel
+constexpr int kLutClasses = 5;
+
 enum KernelKind : int32_t {
   K_DELTA_STATS = 0,     // fused delta + whole-matrix shifted sums for the clip
-  K_STATS_FINAL,         // fixed-order merge of the partial sums -> mean, std, lo, hi
   K_SCALE_SIGNPACK,      // clip + abs-mean (group / row / tensor partials) + sign pack
   K_COL_SCALE_SIGNPACK,  // clip + per-column partial abs sums + sign pack
   K_SCALE_FINAL,         // fixed-order row / column / tensor scale reduction
@@ -30,7 +36,7 @@ enum KernelKind : int32_t {
   K_BASE_GEMV,           // CUDA-core base product for small batches / fp32
   K_BASE_TC,             // tcgen05 base product (bf16, fp32 accumulation in TMEM)
   K_DELTA_LUT,           // per-tenant sign-LUT delta product + combine
-  K_SELECT_FIXUP,        // compress: re-read of groups touched by the clip
+  K_CLIP_FIXUP,          // compress: re-read of the groups the clip changes
   K_PREPARE,             // re-tiling of a tenant into the serving layout
   K_TC_GATHER,           // gather + fp16 scaling of the tensor-core segments' tokens
   K_DELTA_TC,            // tcgen05 delta product of many-token tenants + combine

@@ -22,13 +22,16 @@ def _define(path, name):
     return int(m.group(1))
 
 
-def test_many_token_threshold_matches_the_library():
-    assert bench.TC_MIN_TOKENS == _define("bd_apply.cu", "BD_TC_MIN_TOKENS")
+def test_many_token_threshold_comes_from_the_library():
+    from tenant_serving_b200 import build
+    build.build()
+    assert bench.tc_min_tokens() == _define("bd_apply.cu", "BD_TC_MIN_TOKENS")
+    assert not hasattr(bench, "TC_MIN_TOKENS")  # no copy of the value to go stale
 
 
 def test_traffic_record_is_tied_to_the_kernel_sources(tmp_path, monkeypatch):
     rec = bench.NCU_TRAFFIC["delta_lut"]
-    assert bench.ncu_traffic("delta_tc") is None  # no record, no number
+    assert bench.ncu_traffic("nonexistent_kernel") is None  # no record, no number
     got = bench.ncu_traffic("delta_lut")
     assert got in (None, rec["bytes_per_launch"])
     # a source that differs from the captured one gives no traffic number
