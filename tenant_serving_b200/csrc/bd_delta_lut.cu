@@ -7,27 +7,29 @@
 // where a chunk is 8 consecutive columns, v(row, chunk) the row's sign byte of that chunk
 // and T_t[v][chunk] = sum_j (bit j of v ? +x_t : -x_t)[8 chunk + j]: for every chunk a
 // 256-entry table of all signed sums, built in shared memory once per 256-column window.
-// One byte of signs then costs one shared-memory read per token instead of eight
-// multiply-adds, and all NT tokens are served by one pass over the tenant's bits.
+// One byte of signs then costs one shared-memory read per token (one 8-byte read per pair
+// of tokens) instead of eight multiply-adds, and all NT tokens are served by one pass over
+// the tenant's bits.
 //
-// Organisation: persistent, one CTA per SM, 17 warps.
-//   warp 16, producer: walks this CTA's share of the (lookup group, 512-row tile) units,
-//     cut into pieces of <= DL_PMAX consecutive tiles of one group. For every (window,
-//     tile) of a piece it fills one stage of a ring: a header, the tile's 16 KB of sign
-//     words (one bulk copy from the tiled serving layout, or 512 row copies of 32 bytes
-//     from the row-major layout) and the tile's group-128 scales. Per window, the x slices
-//     of the group's tokens (and column scales) go to a two-slot ring of their own.
-//   warps 0-15, consumers: warp w owns rows 32w..32w+31 of every tile, one row per lane.
-//     At the first tile of a window they rebuild the tables (warp w fills the 16 sign
-//     patterns whose high nibble is w); then each lane turns its row's 32 sign bytes into
-//     32 * NT table reads. Lane l takes word (i + l/4) % 8 at slot i and byte (j + l) % 4
-//     at step j, so the 32 lanes of a warp always read 32 different chunks; with tables
-//     laid out [v][chunk], one bank per chunk, the reads are conflict free. One PRMT of
-//     the sign word with a per-lane constant gives v * 256 + 4 * chunk directly.
-//     Running sums per (tile, token) live in tensor memory (4 columns per tile in the
-//     warp's 128-column block), so one build of a window's tables serves every tile of a
-//     piece. At the end of a piece each lane adds the base product's partial sums and
-//     writes y for its rows, in request order.
+// Organisation: persistent, one CTA per SM, 9 warps.
+//   Work: the (lookup group, 512-row tile) units are split over the CTAs by a cost model
+//     (a group of NT tokens costs about what its table reads cost); a CTA walks its share
+//     in pieces of <= DL_PMAX consecutive tiles of one group. Producer and consumers walk
+//     the same sequence, so no per-stage descriptor is exchanged.
+//   warp 8, producer: for every (window, tile) of a piece fills one stage of a ring with
+//     the tile's 16 KB of sign words (one bulk copy from the tiled serving layout, or 512
+//     row copies of 32 bytes from the row-major layout) and its group-128 scales; per
+//     window, the x slices of the group's tokens (and column scales) go to a two-slot
+//     ring of their own, DL_XSLOTS windows deep.
+//   warps 0-7, consumers: warp w owns rows 32w + l and 256 + 32w + l of every tile (lane
+//     l). At the first tile of a window they rebuild the tables, then each lane turns its
+//     rows' sign bytes into table reads. Lane l takes word (i + l/4) % 8 at slot i and byte
+//     (j + l) % 4 at step j, so a warp's 32 lanes always address 32 different chunks and
+//     the reads are bank-conflict free. The tables sit on a 64 KB boundary: one PRMT of the
+//     sign word with a per-lane constant gives the whole shared address of an entry.
+//     Running sums per (tile, row, token) live in tensor memory, so one build of a
+//     window's tables serves every tile of a piece. At the end of a piece each lane adds
+//     the base product's partial sums and writes y for its rows, in request order.
 // Every wait is bounded; on a timeout the kernel sets BD_DEV_TIMEOUT, lets its copies
 // land, frees its tensor memory and returns.
 #include "bd_internal.cuh"
@@ -35,52 +37,81 @@
 
 namespace bd {
 
-constexpr int DL_CWARPS = 16;                       // consumer warps
+#ifndef BD_LUT_CWARPS
+#define BD_LUT_CWARPS 8
+#endif
+constexpr int DL_CWARPS = BD_LUT_CWARPS;            // consumer warps (8 or 16)
 constexpr int DL_THREADS = (DL_CWARPS + 1) * 32;    // + the producer warp
-constexpr int DL_ROWS = 512;                        // rows per tile = 32 per consumer warp
+constexpr int DL_ROWS = 512;                        // rows per tile
+constexpr int DL_RPL = DL_ROWS / (32 * DL_CWARPS);  // rows of a tile per consumer lane
+constexpr int DL_NIB = 16 / DL_CWARPS;              // table high nibbles built per warp
+// tensor memory of a consumer warp: its lane quadrant (warp % 4) and a block of columns;
+// a tile's running sums take 4 columns per row of the lane (tokens 0-3)
+constexpr uint32_t DL_TBLK = 512u / (DL_CWARPS / 4);
+constexpr uint32_t DL_TSTRIDE = 4u * DL_RPL;
+static_assert(DL_CWARPS == 8 || DL_CWARPS == 16, "8 or 16 consumer warps");
 constexpr int DL_W = 256;                           // columns per window (32 chunks)
-constexpr int DL_PMAX = 32;                         // tiles per piece (4 TMEM columns each)
-constexpr int DL_STAGES = 4;
-constexpr uint32_t DL_TABLE_BYTES = 2 * 65536;      // page 0: tokens 0, 1; page 1: tokens 2, 3
+constexpr int DL_PMAX = 32;                         // tiles per piece (DL_TSTRIDE TMEM columns each)
+static_assert(DL_PMAX * 4 * DL_RPL <= (int)(512u / (DL_CWARPS / 4)), "running sums fit the warp's columns");
+constexpr int DL_MAX_STAGES = 4;
+constexpr uint32_t DL_PAGE = 65536;                 // one page of tables (256 v x 256 B)
+constexpr uint32_t DL_TABLE_BYTES = 2 * DL_PAGE;    // page 0: tokens 0, 1; page 1: tokens 2, 3
 constexpr uint32_t DL_SIGN_BYTES = 16384;           // [512 rows][8 words]
 constexpr uint32_t DL_SC_OFF = 16384;               // [512 rows][2] group-128 scales
-constexpr uint32_t DL_SC_BYTES = 4096;
-constexpr uint32_t DL_HDR_OFF = DL_SC_OFF + DL_SC_BYTES;
-constexpr uint32_t DL_STAGE_BYTES = DL_HDR_OFF + 128;
-constexpr uint32_t DL_XTOK_BYTES = 1024;            // one token's window of x (256 x fp32 max)
-constexpr uint32_t DL_XCS_OFF = 4 * DL_XTOK_BYTES;  // column scales of the window
-constexpr uint32_t DL_XSLOT_BYTES = DL_XCS_OFF + 1024;
+constexpr uint32_t DL_STAGE_BYTES = DL_SC_OFF + 4096;
+constexpr int DL_XSLOTS = 4;                        // x ring depth in windows
+// one x slot: 4 tokens' window of x (256 columns) + the window's column scales (fp32 max)
+__host__ __device__ constexpr uint32_t dl_xtok_bytes(bool xbf16) { return xbf16 ? 512u : 1024u; }
+__host__ __device__ constexpr uint32_t dl_xcs_off(bool xbf16) { return 4u * dl_xtok_bytes(xbf16); }
+__host__ __device__ constexpr uint32_t dl_xslot_bytes(bool xbf16) { return dl_xcs_off(xbf16) + 1024u; }
+// after the tables: the x slots, then the piece descriptors, barriers and flags
+__host__ __device__ constexpr uint32_t dl_fixed_bytes(bool xbf16) { return DL_XSLOTS * dl_xslot_bytes(xbf16) + 640u; }
 constexpr uint32_t DL_TMEM_COLS = 512;
-constexpr size_t DL_SMEM = 128 + DL_TABLE_BYTES + DL_STAGES * DL_STAGE_BYTES + 2 * DL_XSLOT_BYTES + 256;
-static_assert(DL_SMEM <= 227 * 1024, "shared memory layout too large");
+constexpr int DL_SMEM = 227 * 1024;                 // the whole per-CTA shared memory
+static_assert(DL_STAGE_BYTES % 128 == 0 && dl_fixed_bytes(true) % 128 == 0 && dl_fixed_bytes(false) % 128 == 0,
+              "16-byte aligned copies");
 
-// header flags
-constexpr int F_WIN0 = 1;      // first tile of a window: rebuild the tables
-constexpr int F_LAST = 2;      // last stage of a piece: write y
-constexpr int F_BASE = 4;      // base-only piece (no delta): write y from the base product
-constexpr int F_END = 8;       // no more work for this CTA
-constexpr int F_FIRSTWIN = 16; // window 0: the running sums start here
 // sign sources
 constexpr int SS_STAGED = 0;   // in the stage (bulk copies)
-constexpr int SS_DIRECT = 1;   // each lane loads its row's words from global memory
+constexpr int SS_DIRECT = 1;   // each lane loads its rows' words from global memory
 // scale kinds
 constexpr int SK_STAGED = 0;   // group-128 scales in the stage ([row][2])
 constexpr int SK_GLOBAL = 1;   // group scales loaded from global memory per word
 constexpr int SK_NONE = 2;     // row / tensor (applied at the end) or column (folded into x)
 
 // Work weight of one (group, tile) unit of class k (groups of 4, 3, 2, 1 tokens, then
-// base-only groups): about the shared-memory reads of its lookups plus its sign stream.
-__host__ __device__ constexpr int lut_class_weight(int k) { return k < 4 ? 17 - 4 * k : 1; }
+// base-only groups): about the cycles of its table reads and sign stream, relative.
+__host__ __device__ constexpr int lut_class_weight(int k) {
+  return k == 0 ? 13 : (k == 1 ? 10 : (k == 2 ? 7 : (k == 3 ? 5 : 1)));
+}
 
-struct DlHdr {
-  const void* scales;
-  const uint32_t* signs;
-  int32_t flags, nt, p, P;
-  int32_t tile0, win, mode, skind;
-  int32_t lg, ssrc, pad0, pad1;
-  int32_t tok[4];
+// Shared-memory layout of the kernel, from the address where its dynamic window starts:
+// the tables on the first 64 KB boundary, ring stages below them and after them, the x
+// slots and barriers right after the tables. The same arithmetic runs on the host (launch
+// check) and in the kernel.
+struct DlLayout {
+  uint32_t tbase, fixed, stage0_lo, stage0_hi;
+  int n_lo, stages;
 };
-static_assert(sizeof(DlHdr) <= 128, "stage header too large");
+__host__ __device__ inline DlLayout dl_layout(uint32_t raw_base, uint32_t raw_bytes, bool xbf16) {
+  DlLayout L;
+  const uint32_t base = (raw_base + 127u) & ~127u;
+  const uint32_t end = raw_base + raw_bytes;
+  L.tbase = (base + DL_PAGE - 1) & ~(DL_PAGE - 1);
+  L.fixed = L.tbase + DL_TABLE_BYTES;
+  L.stage0_lo = base;
+  L.stage0_hi = L.fixed + dl_fixed_bytes(xbf16);
+  L.n_lo = (int)((L.tbase - base) / DL_STAGE_BYTES);
+  const int n_hi = L.stage0_hi <= end ? (int)((end - L.stage0_hi) / DL_STAGE_BYTES) : -1000;
+  int n = L.n_lo + n_hi;
+  if (n > DL_MAX_STAGES) n = DL_MAX_STAGES;
+  L.stages = n;  // < 2: the layout does not fit
+  return L;
+}
+__device__ __forceinline__ uint32_t dl_stage_addr(const DlLayout& L, int i) {
+  return i < L.n_lo ? L.stage0_lo + (uint32_t)i * DL_STAGE_BYTES
+                    : L.stage0_hi + (uint32_t)(i - L.n_lo) * DL_STAGE_BYTES;
+}
 
 // ------------------------------------------------------------------------------------
 // small device helpers
@@ -96,13 +127,27 @@ __device__ __forceinline__ float lds_off(uint32_t a) {
   asm volatile("ld.shared.f32 %0, [%1+%2];" : "=f"(v) : "r"(a), "n"(OFF));
   return v;
 }
+template <int OFF>
+__device__ __forceinline__ float2 lds2_off(uint32_t a) {
+  float2 v;
+  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2+%3];" : "=f"(v.x), "=f"(v.y) : "r"(a), "n"(OFF));
+  return v;
+}
 __device__ __forceinline__ uint32_t lds32(uint32_t a) {
   uint32_t v;
   asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
   return v;
 }
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
 __device__ __forceinline__ void sts32f(uint32_t a, float v) {
   asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
+}
+__device__ __forceinline__ void sts64f(uint32_t a, float x, float y) {
+  asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(a), "f"(x), "f"(y) : "memory");
 }
 // All consumer warps meet on `bar` (count DL_CWARPS, one arrive per warp); the wait is
 // bounded, so a warp that gave up cannot leave the others blocked. Warp-uniform result.
@@ -118,64 +163,199 @@ __device__ __forceinline__ void tmem_st4(uint32_t taddr, const float* v) {
                "r"(__float_as_uint(v[3]))
                : "memory");
 }
-__device__ __forceinline__ void tmem_ld4_issue(uint32_t taddr, uint32_t* r) {
+__device__ __forceinline__ void tmem_ld4_wait(uint32_t taddr, float* v) {
+  uint32_t r[4];
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                : "r"(taddr)
                : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int q = 0; q < 4; ++q) v[q] = __uint_as_float(r[q]);
 }
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_st4() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// 32 lanes x 8 columns of tensor memory <-> 8 registers per thread
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const float* v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+               "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+               "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+               "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7]))
+               : "memory");
+}
+__device__ __forceinline__ void tmem_ld8_wait(uint32_t taddr, float* v) {
+  uint32_t r[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr)
+               : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int q = 0; q < 8; ++q) v[q] = __uint_as_float(r[q]);
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// the running sums of one tile (DL_TSTRIDE columns)
+__device__ __forceinline__ void tmem_st_tile(uint32_t taddr, const float* v) {
+  if (DL_RPL == 2) tmem_st8(taddr, v);
+  else tmem_st4(taddr, v);
+}
+__device__ __forceinline__ void tmem_ld_tile(uint32_t taddr, float* v) {
+  if (DL_RPL == 2) tmem_ld8_wait(taddr, v);
+  else tmem_ld4_wait(taddr, v);
+}
 
 __device__ __forceinline__ float ldg_scale(const void* s, bool f16, int64_t i) {
   return f16 ? __half2float(reinterpret_cast<const __half*>(s)[i]) : reinterpret_cast<const float*>(s)[i];
 }
 
 // ------------------------------------------------------------------------------------
-// the lookups of one row-window: 8 sign words, NT tokens
+// the walk over this CTA's (group, tile) units
 // ------------------------------------------------------------------------------------
-// wd[i]: sign word (i + sigma) % 8 of the row; sc[i]: its scale; K[i] byte j: 4 * chunk of
-// (slot i, step j); sel[j]: PRMT selector -> byte 0 = K byte j, byte 1 = the sign byte of
-// step j, bytes 2-3 = 0 (sign replicate of K byte j, which is < 128). The table entry of
-// token t sits at tbase + v * 256 + 4 * chunk + (t & 1) * 128 + (t >> 1) * 65536.
+struct DlPiece {
+  bd_tenant T;
+  int item, tile0, P, nt, u, skind, ssrc, lg;
+  int tok[4];
+};
+
+struct DlWalk {
+  int64_t r0, r1, Ck, j, j1, cbase;
+  int k, Sk, sbase, wk, tiles;
+};
+
+__device__ __forceinline__ void walk_init(DlWalk& w, const int32_t* seg_base, int tiles) {
+  int64_t W = 0;
+  for (int k = 0; k < kLutClasses; ++k) W += (int64_t)seg_base[2 + k] * tiles * lut_class_weight(k);
+  w.r0 = W * (int64_t)blockIdx.x / gridDim.x;
+  w.r1 = W * ((int64_t)blockIdx.x + 1) / gridDim.x;
+  w.Ck = 0;
+  w.Sk = 0;
+  w.k = -1;
+  w.j = w.j1 = 0;
+  w.cbase = 0;
+  w.sbase = 0;
+  w.wk = 1;
+  w.tiles = tiles;
+}
+
+// Next piece of this CTA's share; false when there is none. Deterministic: the producer
+// and every consumer thread get the same sequence. *bad is set for an invalid record.
+__device__ __forceinline__ bool walk_next(DlWalk& w, const int32_t* __restrict__ seg_base, const int32_t* __restrict__ grp_tenant,
+                          const int32_t* __restrict__ grp_start, const int32_t* __restrict__ grp_len,
+                          const int32_t* __restrict__ perm, const bd_tenant* __restrict__ tenants,
+                          int64_t d_in, DlPiece& pc, bool* bad) {
+  while (w.j >= w.j1) {
+    if (++w.k >= kLutClasses) return false;
+    const int nk = seg_base[2 + w.k];
+    w.wk = lut_class_weight(w.k);
+    const int64_t Ck1 = w.Ck + (int64_t)nk * w.tiles * w.wk;
+    const int64_t lo = w.r0 > w.Ck ? w.r0 : w.Ck, hi = w.r1 < Ck1 ? w.r1 : Ck1;
+    w.cbase = w.Ck;
+    w.sbase = w.Sk;
+    w.Ck = Ck1;
+    w.Sk += nk;
+    if (lo < hi) {
+      // the units whose start offset cbase + j * wk lies in [lo, hi)
+      w.j = (lo - w.cbase + w.wk - 1) / w.wk;
+      w.j1 = (hi - w.cbase + w.wk - 1) / w.wk;
+    } else {
+      w.j = w.j1 = 0;
+    }
+  }
+  pc.item = w.sbase + (int)(w.j / w.tiles);
+  pc.tile0 = (int)(w.j % w.tiles);
+  int P = w.tiles - pc.tile0;
+  if (P > DL_PMAX) P = DL_PMAX;
+  if ((int64_t)P > w.j1 - w.j) P = (int)(w.j1 - w.j);
+  pc.P = P;
+  w.j += P;
+  pc.nt = grp_len[pc.item];
+  const int gs = grp_start[pc.item];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) pc.tok[q] = q < pc.nt ? perm[gs + q] : 0;
+  pc.u = grp_tenant[pc.item];
+  *bad = false;
+  if (pc.u >= 0) {
+    pc.T = tenants[pc.u];
+    const bd_tenant& T = pc.T;
+    const bool ok_mode = T.mode >= BD_SCALE_GROUP && T.mode <= BD_SCALE_TENSOR;
+    const bool ok_group = T.mode != BD_SCALE_GROUP ||
+                          (T.group_size >= 32 && (T.group_size & (T.group_size - 1)) == 0 && (d_in % T.group_size) == 0);
+    const bool ok_ptr = T.signs != nullptr && T.scales != nullptr &&
+                        ((reinterpret_cast<uintptr_t>(T.signs) | reinterpret_cast<uintptr_t>(T.scales)) & 15u) == 0;
+    const bool ok_layout = (T.layout == BD_LAYOUT_ROWMAJOR || T.layout == BD_LAYOUT_TILED) && T.reserved == 0;
+    if (!(ok_mode && ok_group && ok_ptr && ok_layout)) {
+      *bad = true;
+      pc.u = -1;
+    }
+  }
+  pc.lg = 0;
+  pc.skind = SK_NONE;
+  pc.ssrc = SS_STAGED;
+  if (pc.u >= 0) {
+    const bd_tenant& T = pc.T;
+    if (T.mode == BD_SCALE_GROUP)
+      while ((1 << pc.lg) < T.group_size) ++pc.lg;
+    const bool tiled = T.layout == BD_LAYOUT_TILED;
+    pc.skind = T.mode != BD_SCALE_GROUP ? SK_NONE : ((T.group_size == 128 && tiled) ? SK_STAGED : SK_GLOBAL);
+    pc.ssrc = (tiled || (d_in % DL_W) == 0) ? SS_STAGED : SS_DIRECT;
+  }
+  return true;
+}
+
+// ------------------------------------------------------------------------------------
+// tables and lookups
+// ------------------------------------------------------------------------------------
+// Table entry of (sign byte v, chunk c, token t), offset from the table base:
+//   NT = 1 : v * 256 + 8 * (c & 15) + 4 * (c >> 4)              (32 chunks on 32 banks)
+//   NT >= 2: (t >> 1) * 65536 + v * 256 + 8 * c + 4 * (t & 1)   (token pairs side by side)
+__host__ __device__ __forceinline__ uint32_t dl_chunk_off(int c, bool single) {
+  return single ? (uint32_t)(8 * (c & 15) + 4 * (c >> 4)) : (uint32_t)(8 * c);
+}
+
+// The lookups of one row-window: wd[i] = sign word (i + sigma) % 8 of the row, sc[i] its
+// scale. part[t] += sum over the window of sc * (table entry), token t.
 template <int NT>
-__device__ __forceinline__ void lut_row_window(const uint32_t (&wd)[8], const float (&sc)[8],
-                                               const uint32_t (&K)[8], const uint32_t (&sel)[4],
-                                               uint32_t tbase, float (&part)[4]) {
+__device__ __forceinline__ void lut_row(const uint32_t (&wd)[8], const float (&sc)[8], const uint32_t (&K)[8][2],
+                                        const uint32_t (&sel)[4], float* part) {
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    float a[NT];
-#pragma unroll
-    for (int t = 0; t < NT; ++t) a[t] = 0.f;
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const uint32_t addr = tbase + prmt(wd[i], K[i], sel[j]);
-      a[0] += lds_off<0>(addr);
-      if (NT > 1) a[NT > 1 ? 1 : 0] += lds_off<128>(addr);
-      if (NT > 2) a[NT > 2 ? 2 : 0] += lds_off<65536>(addr);
-      if (NT > 3) a[NT > 3 ? 3 : 0] += lds_off<65536 + 128>(addr);
+      const uint32_t addr = prmt(wd[i], K[i][j >> 1], sel[j]);
+      if (NT == 1) {
+        a0 += lds_off<0>(addr);
+      } else {
+        const float2 e = lds2_off<0>(addr);
+        a0 += e.x;
+        a1 += e.y;
+        if (NT == 3) a2 += lds_off<(int)DL_PAGE>(addr);
+        if (NT == 4) {
+          const float2 f = lds2_off<(int)DL_PAGE>(addr);
+          a2 += f.x;
+          a3 += f.y;
+        }
+      }
     }
-#pragma unroll
-    for (int t = 0; t < NT; ++t) part[t] = fmaf(sc[i], a[t], part[t]);
+    part[0] = fmaf(sc[i], a0, part[0]);
+    if (NT > 1) part[1] = fmaf(sc[i], a1, part[1]);
+    if (NT > 2) part[2] = fmaf(sc[i], a2, part[2]);
+    if (NT > 3) part[3] = fmaf(sc[i], a3, part[3]);
   }
 }
 
 // Tables of one window for the group's tokens, from the x slice (and column scales) in
-// slot xs. Thread (warp h, lane c): chunk c, sign patterns with high nibble h.
+// slot xs. Thread (warp h8, lane c): chunk c, the sign patterns whose high nibble is
+// h8 + DL_CWARPS * k, k < DL_NIB.
 template <bool XBF16>
-__device__ __forceinline__ void lut_build(uint32_t tbase, uint32_t xs, int nt, bool col_mode,
-                                          bool cs_f16, int64_t col0, int64_t d_in) {
-  const int c = threadIdx.x & 31, h = threadIdx.x >> 5;
+__device__ __forceinline__ void lut_build(uint32_t tbase, uint32_t xs, int nt, bool col_mode, bool cs_f16,
+                                          int64_t col0, int64_t d_in) {
+  const int c = threadIdx.x & 31, h8 = threadIdx.x >> 5;
   const bool valid = col0 + 8 * c < d_in;  // d_in % 32 == 0: a chunk is all in or all out
   float cs[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) cs[k] = 1.f;
   if (col_mode && valid) {
     if (cs_f16) {
-      uint4 v;
-      asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                   : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                   : "r"(xs + DL_XCS_OFF + 16u * c));
+      const uint4 v = lds128(xs + dl_xcs_off(XBF16) + 16u * c);
       const uint32_t a[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
@@ -185,46 +365,155 @@ __device__ __forceinline__ void lut_build(uint32_t tbase, uint32_t xs, int nt, b
       }
     } else {
 #pragma unroll
-      for (int k = 0; k < 8; ++k) cs[k] = __uint_as_float(lds32(xs + DL_XCS_OFF + 32u * c + 4u * k));
+      for (int k = 0; k < 8; ++k) cs[k] = __uint_as_float(lds32(xs + dl_xcs_off(XBF16) + 32u * c + 4u * k));
     }
   }
-  for (int t = 0; t < nt; ++t) {
-    float xv[8];
-    if (valid) {
-      const uint32_t xa = xs + (uint32_t)t * DL_XTOK_BYTES;
-      if (XBF16) {
-        uint4 v;
-        asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                     : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                     : "r"(xa + 16u * c));
-        const uint32_t a[4] = {v.x, v.y, v.z, v.w};
+  const bool single = nt == 1;
+  const uint32_t coff = dl_chunk_off(c, single);
+  for (int t0 = 0; t0 < nt; t0 += 2) {
+    // tokens t0 and t0 + 1 (the second one absent for an odd count: zero entries)
+    float lo16[2][16], hi[2][DL_NIB];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          xv[2 * k] = bf16lo(a[k]);
-          xv[2 * k + 1] = bf16hi(a[k]);
+    for (int q = 0; q < 2; ++q) {
+      float xv[8];
+      if (valid && t0 + q < nt) {
+        const uint32_t xa = xs + (uint32_t)(t0 + q) * dl_xtok_bytes(XBF16);
+        if (XBF16) {
+          const uint4 v = lds128(xa + 16u * c);
+          const uint32_t a[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            xv[2 * k] = bf16lo(a[k]);
+            xv[2 * k + 1] = bf16hi(a[k]);
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) xv[k] = __uint_as_float(lds32(xa + 32u * c + 4u * k));
         }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) xv[k] *= cs[k];
       } else {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) xv[k] = __uint_as_float(lds32(xa + 32u * c + 4u * k));
+        for (int k = 0; k < 8; ++k) xv[k] = 0.f;
+      }
+      float p01[4], p23[4];
+#pragma unroll
+      for (int n = 0; n < 4; ++n) {
+        p01[n] = ((n & 1) ? xv[0] : -xv[0]) + ((n & 2) ? xv[1] : -xv[1]);
+        p23[n] = ((n & 1) ? xv[2] : -xv[2]) + ((n & 2) ? xv[3] : -xv[3]);
       }
 #pragma unroll
-      for (int k = 0; k < 8; ++k) xv[k] *= cs[k];
+      for (int lo = 0; lo < 16; ++lo) lo16[q][lo] = p01[lo & 3] + p23[lo >> 2];
+#pragma unroll
+      for (int hh = 0; hh < DL_NIB; ++hh) {
+        const int h = h8 + DL_CWARPS * hh;
+        hi[q][hh] = (((h & 1) ? xv[4] : -xv[4]) + ((h & 2) ? xv[5] : -xv[5])) +
+                    (((h & 4) ? xv[6] : -xv[6]) + ((h & 8) ? xv[7] : -xv[7]));
+      }
+    }
+    const uint32_t page = tbase + (uint32_t)(t0 >> 1) * DL_PAGE + coff;
+#pragma unroll
+    for (int hh = 0; hh < DL_NIB; ++hh) {
+      const uint32_t rowb = page + (uint32_t)(16 * (h8 + DL_CWARPS * hh)) * 256u;
+#pragma unroll
+      for (int lo = 0; lo < 16; ++lo) {
+        if (single)
+          sts32f(rowb + (uint32_t)lo * 256u, lo16[0][lo] + hi[0][hh]);
+        else
+          sts64f(rowb + (uint32_t)lo * 256u, lo16[0][lo] + hi[0][hh], lo16[1][lo] + hi[1][hh]);
+      }
+    }
+  }
+}
+
+// Per-lane PRMT constants for a table layout. K[i][h] bytes 0, 1: the entry offsets of
+// the chunks of (slot i, steps 2h and 2h + 1); bytes 2, 3: the table base >> 16.
+// sel[j]: byte 0 <- K byte (j & 1), byte 1 <- sign byte (j + rho) % 4 of the word,
+// bytes 2, 3 <- K bytes 2, 3.
+__device__ __forceinline__ void dl_lane_consts(int lane, uint32_t tbase, bool single, uint32_t (&K)[8][2],
+                                               uint32_t (&sel)[4]) {
+  const int sig = lane >> 2, rho = lane & 3;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t b = (uint32_t)((j + rho) & 3);
+    sel[j] = (4u + (uint32_t)(j & 1)) | (b << 4) | (6u << 8) | (7u << 12);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int wi = (i + sig) & 7;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t o0 = dl_chunk_off(4 * wi + ((2 * h + rho) & 3), single);
+      const uint32_t o1 = dl_chunk_off(4 * wi + ((2 * h + 1 + rho) & 3), single);
+      K[i][h] = o0 | (o1 << 8) | (tbase & 0xFFFF0000u);
+    }
+  }
+}
+
+// What the consumers need of a piece; written by the producer into a small ring.
+struct DlDesc {
+  const uint32_t* signs;
+  const void* scales;
+  int32_t tile0, P, nt, u;  // u: tenant, -1 base only, -2 end of this CTA's work
+  int32_t mode, skind, ssrc, lg;
+  int32_t tok[4];
+};
+static_assert(sizeof(DlDesc) == 64, "descriptor slot size");
+constexpr int DL_DSLOTS = 4;
+
+// One row-window of a stage: its sign words, their scales, the lookups into part[0..3].
+__device__ __forceinline__ void dl_row_window(const DlDesc& D, uint32_t st, int r_in, int tile, int win, int nt,
+                                              int sig, uint32_t hi_slots, bool scale_f16, int64_t d_out,
+                                              int64_t d_in, int64_t wpr, const uint32_t (&K)[8][2],
+                                              const uint32_t (&sel)[4], float* part) {
+  const int64_t row = (int64_t)tile * DL_ROWS + r_in;
+  const bool live = row < d_out;
+  uint32_t wd[8];
+  if (D.ssrc == SS_STAGED) {
+    const uint32_t wrow = st + (uint32_t)r_in * 32u;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) wd[i] = lds32(wrow + 4u * (uint32_t)((i + sig) & 7));
+  } else {
+    const uint32_t* signs = D.signs;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int64_t wi = (int64_t)win * 8 + ((i + sig) & 7);
+      wd[i] = (live && wi < wpr) ? signs[row * wpr + wi] : 0u;
+    }
+  }
+  float sc[8];
+  const int skind = D.skind;
+  if (skind == SK_STAGED) {
+    const uint32_t sa = st + DL_SC_OFF + (uint32_t)r_in * (scale_f16 ? 4u : 8u);
+    float s0, s1;
+    if (scale_f16) {
+      const uint32_t v = lds32(sa);
+      s0 = __half2float(__ushort_as_half((unsigned short)(v & 0xFFFFu)));
+      s1 = __half2float(__ushort_as_half((unsigned short)(v >> 16)));
     } else {
-#pragma unroll
-      for (int k = 0; k < 8; ++k) xv[k] = 0.f;
+      s0 = __uint_as_float(lds32(sa));
+      s1 = __uint_as_float(lds32(sa + 4u));
     }
-    float p01[4], p23[4];
 #pragma unroll
-    for (int n = 0; n < 4; ++n) {
-      p01[n] = ((n & 1) ? xv[0] : -xv[0]) + ((n & 2) ? xv[1] : -xv[1]);
-      p23[n] = ((n & 1) ? xv[2] : -xv[2]) + ((n & 2) ? xv[3] : -xv[3]);
+    for (int i = 0; i < 8; ++i) sc[i] = ((hi_slots >> i) & 1u) ? s1 : s0;
+  } else if (skind == SK_GLOBAL) {
+    const int lg = D.lg;
+    const void* scales = D.scales;
+    const int64_t gpr = d_in >> lg;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int64_t col = (int64_t)win * DL_W + 32 * ((i + sig) & 7);
+      sc[i] = (live && col < d_in) ? ldg_scale(scales, scale_f16, row * gpr + (col >> lg)) : 0.f;
     }
-    const float hi = (((h & 1) ? xv[4] : -xv[4]) + ((h & 2) ? xv[5] : -xv[5])) +
-                     (((h & 4) ? xv[6] : -xv[6]) + ((h & 8) ? xv[7] : -xv[7]));
-    const uint32_t base = tbase + (uint32_t)(t >> 1) * 65536u + (uint32_t)(t & 1) * 128u +
-                          (uint32_t)(16 * h) * 256u + 4u * (uint32_t)c;
+  } else {
 #pragma unroll
-    for (int lo = 0; lo < 16; ++lo) sts32f(base + (uint32_t)lo * 256u, (p01[lo & 3] + p23[lo >> 2]) + hi);
+    for (int i = 0; i < 8; ++i) sc[i] = 1.f;
+  }
+  switch (nt) {
+    case 1: lut_row<1>(wd, sc, K, sel, part); break;
+    case 2: lut_row<2>(wd, sc, K, sel, part); break;
+    case 3: lut_row<3>(wd, sc, K, sel, part); break;
+    default: lut_row<4>(wd, sc, K, sel, part); break;
   }
 }
 
@@ -250,30 +539,43 @@ __global__ void __launch_bounds__(DL_THREADS, 1) k_delta_lut(
     int max_groups, int max_tc, const void* __restrict__ x, const float* __restrict__ y_part,
     int ksplit, int64_t d_out, int64_t d_in, int batch, void* __restrict__ y, bool y_bf16,
     uint32_t* __restrict__ status) {
-  extern __shared__ uint8_t dl_smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dl_smem_raw) + 127) & ~uintptr_t(127));
-  const uint32_t tbase = smem_u32(sm);
-  uint8_t* stages = sm + DL_TABLE_BYTES;
-  uint8_t* xslots = stages + DL_STAGES * DL_STAGE_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(xslots + 2 * DL_XSLOT_BYTES);
-  uint64_t* empty = full + DL_STAGES;
-  uint64_t* xfull = empty + DL_STAGES;
-  uint64_t* xempty = xfull + 2;
-  uint64_t* cbar = xempty + 2;  // [2]: consumers before / after a table build
+  extern __shared__ __align__(16) uint8_t dl_smem_raw[];
+  const uint32_t raw = smem_u32(dl_smem_raw);
+  const DlLayout L = dl_layout(raw, DL_SMEM, XBF16);
+  constexpr uint32_t XTOK = dl_xtok_bytes(XBF16), XCS = dl_xcs_off(XBF16), XSLOT = dl_xslot_bytes(XBF16);
+  if (L.stages < 2) {  // checked on the host before the launch
+    if (threadIdx.x == 0) atomicOr(status, BD_DEV_INTERNAL);
+    return;
+  }
+  uint8_t* gen = dl_smem_raw - raw;  // generic pointer of shared address 0
+  const uint32_t xslot0 = L.fixed;
+  DlDesc* desc = reinterpret_cast<DlDesc*>(gen + L.fixed + DL_XSLOTS * XSLOT);
+  uint64_t* full = reinterpret_cast<uint64_t*>(desc + DL_DSLOTS);
+  uint64_t* empty = full + DL_MAX_STAGES;
+  uint64_t* xfull = empty + DL_MAX_STAGES;
+  uint64_t* xempty = xfull + DL_XSLOTS;
+  uint64_t* dfull = xempty + DL_XSLOTS;
+  uint64_t* dempty = dfull + DL_DSLOTS;
+  uint64_t* cbar = dempty + DL_DSLOTS;  // [2]: consumers before / after a table build
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cbar + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int NS = L.stages;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
-    for (int i = 0; i < DL_STAGES; ++i) {
+    for (int i = 0; i < DL_MAX_STAGES; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], DL_CWARPS);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < DL_XSLOTS; ++i) {
       mbar_init(&xfull[i], 1);
       mbar_init(&xempty[i], DL_CWARPS);
-      mbar_init(&cbar[i], DL_CWARPS);
     }
+    for (int i = 0; i < DL_DSLOTS; ++i) {
+      mbar_init(&dfull[i], 1);
+      mbar_init(&dempty[i], DL_CWARPS);
+    }
+    for (int i = 0; i < 2; ++i) mbar_init(&cbar[i], DL_CWARPS);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -283,395 +585,293 @@ __global__ void __launch_bounds__(DL_THREADS, 1) k_delta_lut(
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int32_t* grp_tenant = seg_base + kSegHeader;
-  const int32_t* grp_start = grp_tenant + max_groups;
-  const int32_t* grp_len = grp_start + max_groups;
-  const int32_t* perm = grp_len + max_groups + 4 * max_tc;
   const int nwin = (int)((d_in + DL_W - 1) / DL_W);
   const int tiles = (int)((d_out + DL_ROWS - 1) / DL_ROWS);
   const int64_t wpr = d_in >> 5;
+  const int ssz = scale_f16 ? 2 : 4;
 
   if (warp == DL_CWARPS) {
     // ================================ producer ================================
-    // class k: lookup groups of 4, 3, 2, 1 tokens of a tenant, then base-only groups;
-    // a (group, tile) unit weighs about its shared-memory reads
-    int64_t W = 0;
-    for (int k = 0; k < kLutClasses; ++k) W += (int64_t)seg_base[2 + k] * tiles * lut_class_weight(k);
-    const int64_t r0 = W * (int64_t)blockIdx.x / gridDim.x;
-    const int64_t r1 = W * ((int64_t)blockIdx.x + 1) / gridDim.x;
-    const int ssz = scale_f16 ? 2 : 4;
+    const int32_t* grp_tenant = seg_base + kSegHeader;
+    const int32_t* grp_start = grp_tenant + max_groups;
+    const int32_t* grp_len = grp_start + max_groups;
+    const int32_t* perm = grp_len + max_groups + 4 * max_tc;
+    DlWalk walk;
+    walk_init(walk, seg_base, tiles);
+    DlPiece pc;
+    bool bad = false;
     const int xb = XBF16 ? 2 : 4;
-    DlRing S, X;
+    DlRing S, X, Dr;
     bool stop = false;
-
-    // wait for a free stage; false on abort / timeout (warp-uniform)
-    auto acquire = [&]() -> bool {
+    // a free descriptor slot (warp-uniform; false on abort / timeout)
+    auto take_desc = [&]() -> bool {
       bool ok = true;
-      if (lane == 0 && S.n >= DL_STAGES) ok = mbar_wait(&empty[S.slot], S.phase ^ 1u, abort_flag);
+      if (lane == 0 && Dr.n >= DL_DSLOTS) ok = mbar_wait(&dempty[Dr.slot], Dr.phase ^ 1u, abort_flag);
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (!ok && lane == 0) *abort_flag = 1;
       return ok;
     };
-
-    int64_t Ck = 0;  // weight before class k
-    int Sk = 0;      // first group of class k
-    for (int k = 0; k < kLutClasses && !stop; ++k) {
-      const int nk = seg_base[2 + k];
-      const int wk = lut_class_weight(k);
-      const int64_t Ck1 = Ck + (int64_t)nk * tiles * wk;
-      const int64_t lo = r0 > Ck ? r0 : Ck, hi = r1 < Ck1 ? r1 : Ck1;
-      const int64_t cbase = Ck;
-      const int sbase = Sk;
-      Ck = Ck1;
-      Sk += nk;
-      if (lo >= hi) continue;
-      // units whose start offset cbase + j * wk lies in [lo, hi)
-      const int64_t j1 = (hi - cbase + wk - 1) / wk;
-      int64_t j = (lo - cbase + wk - 1) / wk;
-      while (j < j1 && !stop) {
-        const int item = sbase + (int)(j / tiles);
-        const int tile0 = (int)(j % tiles);
-        int P = tiles - tile0;
-        if (P > DL_PMAX) P = DL_PMAX;
-        if ((int64_t)P > j1 - j) P = (int)(j1 - j);
-        j += P;
-        // ---- the group and its tenant record
-        const int u0 = grp_tenant[item];
-        const int nt = grp_len[item];
-        int tok[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) tok[q] = q < nt ? perm[grp_start[item] + q] : 0;
-        bd_tenant T{};
-        int u = u0;
-        if (u >= 0) {
-          T = tenants[u];
-          const bool ok_mode = T.mode >= BD_SCALE_GROUP && T.mode <= BD_SCALE_TENSOR;
-          const bool ok_group = T.mode != BD_SCALE_GROUP ||
-                                (T.group_size >= 32 && (T.group_size & (T.group_size - 1)) == 0 &&
-                                 (d_in % T.group_size) == 0);
-          const bool ok_ptr = T.signs != nullptr && T.scales != nullptr &&
-                              ((reinterpret_cast<uintptr_t>(T.signs) |
-                                reinterpret_cast<uintptr_t>(T.scales)) & 15u) == 0;
-          const bool ok_layout = (T.layout == BD_LAYOUT_ROWMAJOR || T.layout == BD_LAYOUT_TILED) &&
-                                 T.reserved == 0;
-          if (!(ok_mode && ok_group && ok_ptr && ok_layout)) {
-            if (lane == 0) atomicOr(status, BD_DEV_TENANT_RECORD);
-            u = -1;
-          }
-        }
-        if (u < 0) {
-          // base-only piece: one header-only stage
-          if (!acquire()) { stop = true; break; }
-          if (lane == 0) {
-            DlHdr* H = reinterpret_cast<DlHdr*>(stages + S.slot * DL_STAGE_BYTES + DL_HDR_OFF);
-            H->flags = F_BASE | F_LAST;
-            H->nt = nt;
-            H->p = 0;
-            H->P = P;
-            H->tile0 = tile0;
-            H->win = 0;
-            H->mode = BD_SCALE_GROUP;
-            H->skind = SK_NONE;
-            H->lg = 0;
-            H->ssrc = SS_STAGED;
-            H->scales = nullptr;
-            H->signs = nullptr;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) H->tok[q] = tok[q];
-            mbar_arrive(&full[S.slot]);
-          }
-          __syncwarp();
-          S.next(DL_STAGES);
-          continue;
-        }
-        int lg = 0;
-        if (T.mode == BD_SCALE_GROUP)
-          while ((1 << lg) < T.group_size) ++lg;
-        const bool tiled = T.layout == BD_LAYOUT_TILED;
-        const int skind = T.mode != BD_SCALE_GROUP ? SK_NONE
-                          : ((T.group_size == 128 && tiled) ? SK_STAGED : SK_GLOBAL);
-        const int ssrc = (tiled || (d_in % DL_W) == 0) ? SS_STAGED : SS_DIRECT;
-        for (int win = 0; win < nwin && !stop; ++win) {
-          // ---- x slices (and column scales) of this window
-          const int64_t col0 = (int64_t)win * DL_W;
-          const int ncols = (int)((d_in - col0) < DL_W ? (d_in - col0) : DL_W);
-          {
-            bool ok = true;
-            if (lane == 0 && X.n >= 2) ok = mbar_wait(&xempty[X.slot], X.phase ^ 1u, abort_flag);
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            if (!ok) {
-              if (lane == 0) *abort_flag = 1;
-              stop = true;
-              break;
-            }
-            if (lane == 0) {
-              uint8_t* xs = xslots + X.slot * DL_XSLOT_BYTES;
-              const uint32_t xbytes = (uint32_t)(ncols * xb);
-              const uint32_t cbytes = T.mode == BD_SCALE_COL ? (uint32_t)(ncols * ssz) : 0u;
-              mbar_arrive_expect_tx(&xfull[X.slot], xbytes * (uint32_t)nt + cbytes);
-              for (int q = 0; q < nt; ++q)
-                bulk_load(xs + q * DL_XTOK_BYTES,
-                          reinterpret_cast<const uint8_t*>(x) + ((int64_t)tok[q] * d_in + col0) * xb,
-                          xbytes, &xfull[X.slot]);
-              if (cbytes)
-                bulk_load(xs + DL_XCS_OFF, reinterpret_cast<const uint8_t*>(T.scales) + col0 * ssz,
-                          cbytes, &xfull[X.slot]);
-            }
-            __syncwarp();
-            X.next(2);
-          }
-          for (int p = 0; p < P; ++p) {
-            if (!acquire()) { stop = true; break; }
-            const int tile = tile0 + p;
-            uint8_t* st = stages + S.slot * DL_STAGE_BYTES;
-            const int rows = (int)((d_out - (int64_t)tile * DL_ROWS) < DL_ROWS ? (d_out - (int64_t)tile * DL_ROWS)
-                                                                                : DL_ROWS);
-            uint32_t bytes = 0;
-            if (ssrc == SS_STAGED) bytes += tiled ? DL_SIGN_BYTES : (uint32_t)rows * 32u;
-            if (skind == SK_STAGED) bytes += 1024u * (uint32_t)ssz;
-            if (lane == 0) {
-              DlHdr* H = reinterpret_cast<DlHdr*>(st + DL_HDR_OFF);
-              int f = 0;
-              if (p == 0) f |= F_WIN0;
-              if (win == 0) f |= F_FIRSTWIN;
-              if (win == nwin - 1 && p == P - 1) f |= F_LAST;
-              H->flags = f;
-              H->nt = nt;
-              H->p = p;
-              H->P = P;
-              H->tile0 = tile0;
-              H->win = win;
-              H->mode = T.mode;
-              H->skind = skind;
-              H->lg = lg;
-              H->ssrc = ssrc;
-              H->scales = T.scales;
-              H->signs = T.signs;
-#pragma unroll
-              for (int q = 0; q < 4; ++q) H->tok[q] = tok[q];
-              if (bytes) mbar_arrive_expect_tx(&full[S.slot], bytes);
-              else mbar_arrive(&full[S.slot]);
-              if (ssrc == SS_STAGED && tiled)
-                bulk_load(st, T.signs + ((int64_t)tile * nwin + win) * 4096, DL_SIGN_BYTES, &full[S.slot]);
-              if (skind == SK_STAGED)
-                bulk_load(st + DL_SC_OFF,
-                          reinterpret_cast<const uint8_t*>(T.scales) + ((int64_t)tile * nwin + win) * 1024 * ssz,
-                          1024u * (uint32_t)ssz, &full[S.slot]);
-            }
-            __syncwarp();
-            if (ssrc == SS_STAGED && !tiled) {
-              // row-major, d_in % 256 == 0: one 32-byte copy per row (16-byte aligned)
-              for (int r = lane; r < rows; r += 32)
-                bulk_load(st + r * 32, T.signs + ((int64_t)tile * DL_ROWS + r) * wpr + (int64_t)win * 8, 32u,
-                          &full[S.slot]);
-            }
-            __syncwarp();
-            S.next(DL_STAGES);
-          }
-        }
+    for (;;) {
+      const bool more = walk_next(walk, seg_base, grp_tenant, grp_start, grp_len, perm, tenants, d_in, pc, &bad);
+      if (!take_desc()) {
+        stop = true;
+        break;
       }
-    }
-    // end marker; after an abort there is none: the consumers see the abort flag instead
-    if (!stop && acquire()) {
       if (lane == 0) {
-        DlHdr* H = reinterpret_cast<DlHdr*>(stages + S.slot * DL_STAGE_BYTES + DL_HDR_OFF);
-        H->flags = F_END;
-        mbar_arrive(&full[S.slot]);
+        DlDesc& D = desc[Dr.slot];
+        if (!more) {
+          D.u = -2;
+        } else {
+          if (bad) atomicOr(status, BD_DEV_TENANT_RECORD);
+          D.signs = pc.T.signs;
+          D.scales = pc.T.scales;
+          D.tile0 = pc.tile0;
+          D.P = pc.P;
+          D.nt = pc.nt;
+          D.u = pc.u;
+          D.mode = pc.u >= 0 ? pc.T.mode : (int)BD_SCALE_GROUP;
+          D.skind = pc.skind;
+          D.ssrc = pc.ssrc;
+          D.lg = pc.lg;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) D.tok[q] = pc.tok[q];
+        }
+        mbar_arrive(&dfull[Dr.slot]);
       }
       __syncwarp();
-      S.next(DL_STAGES);
+      Dr.next(DL_DSLOTS);
+      if (!more) break;
+      if (pc.u < 0) continue;  // base-only piece: the consumers write it without stages
+      const bd_tenant& T = pc.T;
+      const bool tiled = T.layout == BD_LAYOUT_TILED;
+      for (int win = 0; win < nwin && !stop; ++win) {
+        // ---- x slices (and column scales) of this window
+        const int64_t col0 = (int64_t)win * DL_W;
+        const int ncols = (int)((d_in - col0) < DL_W ? (d_in - col0) : DL_W);
+        {
+          bool ok = true;
+          if (lane == 0 && X.n >= DL_XSLOTS) ok = mbar_wait(&xempty[X.slot], X.phase ^ 1u, abort_flag);
+          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+          if (!ok) {
+            if (lane == 0) *abort_flag = 1;
+            stop = true;
+            break;
+          }
+          if (lane == 0) {
+            uint8_t* xs = gen + xslot0 + X.slot * XSLOT;
+            const uint32_t xbytes = (uint32_t)(ncols * xb);
+            const uint32_t cbytes = T.mode == BD_SCALE_COL ? (uint32_t)(ncols * ssz) : 0u;
+            mbar_arrive_expect_tx(&xfull[X.slot], xbytes * (uint32_t)pc.nt + cbytes);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              if (q < pc.nt)
+                bulk_load(xs + q * XTOK,
+                          reinterpret_cast<const uint8_t*>(x) + ((int64_t)pc.tok[q] * d_in + col0) * xb, xbytes,
+                          &xfull[X.slot]);
+            if (cbytes)
+              bulk_load(xs + XCS, reinterpret_cast<const uint8_t*>(T.scales) + col0 * ssz, cbytes, &xfull[X.slot]);
+          }
+          __syncwarp();
+          X.next(DL_XSLOTS);
+        }
+        for (int p = 0; p < pc.P; ++p) {
+          bool ok = true;
+          if (lane == 0 && S.n >= NS) ok = mbar_wait(&empty[S.slot], S.phase ^ 1u, abort_flag);
+          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+          if (!ok) {
+            if (lane == 0) *abort_flag = 1;
+            stop = true;
+            break;
+          }
+          const int tile = pc.tile0 + p;
+          uint8_t* st = gen + dl_stage_addr(L, S.slot);
+          const int rows = (int)((d_out - (int64_t)tile * DL_ROWS) < DL_ROWS ? (d_out - (int64_t)tile * DL_ROWS)
+                                                                              : DL_ROWS);
+          uint32_t bytes = 0;
+          if (pc.ssrc == SS_STAGED) bytes += tiled ? DL_SIGN_BYTES : (uint32_t)rows * 32u;
+          if (pc.skind == SK_STAGED) bytes += 1024u * (uint32_t)ssz;
+          if (lane == 0) {
+            if (bytes) mbar_arrive_expect_tx(&full[S.slot], bytes);
+            else mbar_arrive(&full[S.slot]);
+            if (pc.ssrc == SS_STAGED && tiled)
+              bulk_load(st, T.signs + ((int64_t)tile * nwin + win) * 4096, DL_SIGN_BYTES, &full[S.slot]);
+            if (pc.skind == SK_STAGED)
+              bulk_load(st + DL_SC_OFF,
+                        reinterpret_cast<const uint8_t*>(T.scales) + ((int64_t)tile * nwin + win) * 1024 * ssz,
+                        1024u * (uint32_t)ssz, &full[S.slot]);
+          }
+          __syncwarp();
+          if (pc.ssrc == SS_STAGED && !tiled) {
+            // row-major, d_in % 256 == 0: one 32-byte copy per row (16-byte aligned)
+            for (int r = lane; r < rows; r += 32)
+              bulk_load(st + r * 32, T.signs + ((int64_t)tile * DL_ROWS + r) * wpr + (int64_t)win * 8, 32u,
+                        &full[S.slot]);
+          }
+          __syncwarp();
+          S.next(NS);
+        }
+      }
+      if (stop) break;
     }
     // every copy issued must land before the CTA leaves: the last fill of each stage and
     // of each x slot completes its phase (bounded; a phase already completed returns at once)
     if (lane == 0) {
-      for (int q = 1; q <= DL_STAGES && q <= S.n; ++q) {
+      for (int q = 1; q <= NS && q <= S.n; ++q) {
         const int f = S.n - q;
-        mbar_wait(&full[f % DL_STAGES], (uint32_t)(f / DL_STAGES) & 1u, nullptr);
+        mbar_wait(&full[f % NS], (uint32_t)(f / NS) & 1u, nullptr);
       }
-      for (int q = 1; q <= 2 && q <= X.n; ++q) {
+      for (int q = 1; q <= DL_XSLOTS && q <= X.n; ++q) {
         const int f = X.n - q;
-        mbar_wait(&xfull[f % 2], (uint32_t)(f / 2) & 1u, nullptr);
+        mbar_wait(&xfull[f % DL_XSLOTS], (uint32_t)(f / DL_XSLOTS) & 1u, nullptr);
       }
     }
     __syncwarp();
   } else {
     // ================================ consumers ================================
-    const int sig = lane >> 2, rho = lane & 3;
-    uint32_t K[8], sel[4];
+    // lane constants: rotation sigma (words), which slots hold words 4-7 of a window, the
+    // PRMT constants of the table layout in use (recomputed when a piece changes it)
+    const int sig = lane >> 2;
+    uint32_t hi_slots = 0;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t b = (uint32_t)((j + rho) & 3);
-      const uint32_t kb = 4u + (uint32_t)j;
-      sel[j] = kb | (b << 4) | ((0x8u | kb) << 8) | ((0x8u | kb) << 12);
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint32_t wi = (uint32_t)((i + sig) & 7);
-      uint32_t v = 0;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) v |= (4u * (4u * wi + (uint32_t)((j + rho) & 3))) << (8 * j);
-      K[i] = v;
-    }
-    const uint32_t t_lane = tmem_base + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(warp >> 2) * 128u;
-    const int r_in = warp * 32 + lane;  // row inside a tile
-    DlRing S, X;
-    bool dead = false;
+    for (int i = 0; i < 8; ++i) hi_slots |= (((i + sig) & 7) >= 4 ? 1u : 0u) << i;
+    uint32_t K[8][2], sel[4];
+    int k_single = -1;
+    // tensor memory: lane quadrant warp % 4, column block warp / 4; tile p, row h of the
+    // lane, token t at column DL_TSTRIDE * p + 4h + t
+    const uint32_t t_lane = tmem_base + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(warp >> 2) * DL_TBLK;
+    const int r_lo = warp * 32 + lane;  // rows r_lo + 32 * DL_CWARPS * h of each tile, h < DL_RPL
+    DlRing S, X, Dr;
     for (;;) {
-      const bool got = __all_sync(0xffffffffu, mbar_wait(&full[S.slot], S.phase, abort_flag));
-      if (!got) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&dfull[Dr.slot], Dr.phase, abort_flag))) {
         if (lane == 0) *abort_flag = 1;
-        dead = true;
         break;
       }
-      const uint8_t* st = stages + S.slot * DL_STAGE_BYTES;
-      const DlHdr* H = reinterpret_cast<const DlHdr*>(st + DL_HDR_OFF);
-      const int flags = H->flags;
-      if (flags & F_END) break;
-      const int nt = H->nt, p = H->p, P = H->P, tile0 = H->tile0, win = H->win, mode = H->mode;
-      const int skind = H->skind, lg = H->lg, ssrc = H->ssrc;
-      const void* scales = H->scales;
-      const uint32_t* signs = H->signs;
-      int tok[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) tok[q] = H->tok[q];
-
-      if (!(flags & F_BASE)) {
-        if (flags & F_WIN0) {
+      const DlDesc& D = desc[Dr.slot];
+      const int u = D.u;
+      if (u == -2) break;
+      const int nt = D.nt, P = D.P, tile0 = D.tile0;
+      bool dead = false;
+      if (u >= 0) {
+        const bool single = nt == 1;
+        if ((int)single != k_single) {
+          dl_lane_consts(lane, L.tbase, single, K, sel);
+          k_single = (int)single;
+        }
+        for (int win = 0; win < nwin && !dead; ++win) {
           // new window: wait for its x, rebuild the tables once every warp is done with
           // the previous window's lookups
           const bool xok = __all_sync(0xffffffffu, mbar_wait(&xfull[X.slot], X.phase, abort_flag));
-          if (!xok) {
-            if (lane == 0) *abort_flag = 1;
+          const uint32_t cpar = (uint32_t)X.n & 1u;  // both meeting barriers flip once per window
+          if (!xok || !consumer_sync(&cbar[0], cpar, abort_flag)) {
             dead = true;
             break;
           }
-          // X.n counts the windows seen: both meeting barriers flip phase once per window
-          const uint32_t cpar = (uint32_t)X.n & 1u;
-          if (!consumer_sync(&cbar[0], cpar, abort_flag)) {
-            if (lane == 0) *abort_flag = 1;
-            dead = true;
-            break;
-          }
-          lut_build<XBF16>(tbase, smem_u32(xslots + X.slot * DL_XSLOT_BYTES), nt, mode == BD_SCALE_COL,
-                           scale_f16, (int64_t)win * DL_W, d_in);
+          lut_build<XBF16>(L.tbase, xslot0 + X.slot * XSLOT, nt, D.mode == BD_SCALE_COL, scale_f16,
+                           (int64_t)win * DL_W, d_in);
           __syncwarp();
           if (lane == 0) mbar_arrive(&xempty[X.slot]);
-          X.next(2);
+          X.next(DL_XSLOTS);
           if (!consumer_sync(&cbar[1], cpar, abort_flag)) {
-            if (lane == 0) *abort_flag = 1;
             dead = true;
             break;
           }
-        }
-        const int64_t row = (int64_t)(tile0 + p) * DL_ROWS + r_in;
-        const bool live = row < d_out;
-        // the row's 8 sign words, rotated by sigma
-        uint32_t wd[8];
-        if (ssrc == SS_STAGED) {
-          const uint32_t wrow = smem_u32(st) + (uint32_t)r_in * 32u;
+          for (int p = 0; p < P; ++p) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&full[S.slot], S.phase, abort_flag))) {
+              dead = true;
+              break;
+            }
+            const uint32_t st = dl_stage_addr(L, S.slot);
+            float part[4 * DL_RPL];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) wd[i] = lds32(wrow + 4u * (uint32_t)((i + sig) & 7));
-        } else {
+            for (int q = 0; q < 4 * DL_RPL; ++q) part[q] = 0.f;
+            const uint32_t tcol = t_lane + DL_TSTRIDE * (uint32_t)p;
+            if (win > 0) {
+              // running sums of this tile from the previous windows
+              tmem_wait_st();
+              tmem_ld_tile(tcol, part);
+            }
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int64_t wi = (int64_t)win * 8 + ((i + sig) & 7);
-            wd[i] = (live && wi < wpr) ? signs[row * wpr + wi] : 0u;
+            for (int h = 0; h < DL_RPL; ++h)
+              dl_row_window(D, st, r_lo + 32 * DL_CWARPS * h, tile0 + p, win, nt, sig, hi_slots, scale_f16, d_out,
+                            d_in, wpr, K, sel, part + 4 * h);
+            tmem_st_tile(tcol, part);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[S.slot]);
+            S.next(NS);
           }
         }
-        // the scale of each word
-        float sc[8];
-        if (skind == SK_STAGED) {
-          const uint32_t sa = smem_u32(st) + DL_SC_OFF + (uint32_t)r_in * (scale_f16 ? 4u : 8u);
-          float s0, s1;
-          if (scale_f16) {
-            const uint32_t v = lds32(sa);
-            s0 = __half2float(__ushort_as_half((unsigned short)(v & 0xFFFFu)));
-            s1 = __half2float(__ushort_as_half((unsigned short)(v >> 16)));
-          } else {
-            s0 = __uint_as_float(lds32(sa));
-            s1 = __uint_as_float(lds32(sa + 4u));
-          }
-#pragma unroll
-          for (int i = 0; i < 8; ++i) sc[i] = ((i + sig) & 7) < 4 ? s0 : s1;
-        } else if (skind == SK_GLOBAL) {
-          const int64_t gpr = d_in >> lg;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int64_t col = (int64_t)win * DL_W + 32 * ((i + sig) & 7);
-            sc[i] = (live && col < d_in) ? ldg_scale(scales, scale_f16, row * gpr + (col >> lg)) : 0.f;
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) sc[i] = 1.f;
+        if (dead) {
+          if (lane == 0) *abort_flag = 1;
+          break;
         }
-        const uint32_t tcol = t_lane + 4u * (uint32_t)p;
-        float part[4] = {0.f, 0.f, 0.f, 0.f};
-        if (!(flags & F_FIRSTWIN)) {
-          // running sums of this tile from the previous windows
-          uint32_t old[4];
-          tmem_wait_st4();
-          tmem_ld4_issue(tcol, old);
-          tmem_wait_ld();
-#pragma unroll
-          for (int q = 0; q < 4; ++q) part[q] = __uint_as_float(old[q]);
-        }
-        switch (nt) {
-          case 1: lut_row_window<1>(wd, sc, K, sel, tbase, part); break;
-          case 2: lut_row_window<2>(wd, sc, K, sel, tbase, part); break;
-          case 3: lut_row_window<3>(wd, sc, K, sel, tbase, part); break;
-          default: lut_row_window<4>(wd, sc, K, sel, tbase, part); break;
-        }
-        tmem_st4(tcol, part);
+        tmem_wait_st();
       }
-      // the stage is consumed (its header was copied to registers above)
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[S.slot]);
-      S.next(DL_STAGES);
-
-      if (flags & F_LAST) {
-        // ---- end of a piece: y = base partial sums + delta, rows of this lane
-        const bool base_only = (flags & F_BASE) != 0;
-        if (!base_only) tmem_wait_st4();
-        float rs = 1.f;
-        if (!base_only && mode == BD_SCALE_TENSOR) rs = ldg_scale(scales, scale_f16, 0);
-        for (int p0 = 0; p0 < P; p0 += 8) {
-          uint32_t acc[32];
-          if (!base_only) {
-            tmem_ld32(t_lane + 4u * (uint32_t)p0, acc);  // includes the wait
-          } else {
+      // ---- end of a piece: y = base partial sums + delta, rows of this lane. Several
+      // tiles at a time: their running sums in one tensor-memory read and all their base
+      // partial sums as independent loads before any store.
+      const bool base_only = u < 0;
+      const int mode = D.mode;
+      const void* scales = D.scales;
+      float rs = 1.f;
+      if (!base_only && mode == BD_SCALE_TENSOR) rs = ldg_scale(scales, scale_f16, 0);
+      constexpr int PT = 32 / DL_TSTRIDE;  // tiles per 32-column read
+      for (int p0 = 0; p0 < P; p0 += PT) {
+        uint32_t acc[32];  // tile p0 + pp, row h, token q at DL_TSTRIDE * pp + 4 h + q
+        if (!base_only) {
+          tmem_ld32(t_lane + DL_TSTRIDE * (uint32_t)p0, acc);
+        } else {
 #pragma unroll
-            for (int q = 0; q < 32; ++q) acc[q] = 0u;
-          }
+          for (int q = 0; q < 32; ++q) acc[q] = 0u;
+        }
+        float bsum[PT][DL_RPL][4];
 #pragma unroll
-          for (int pp = 0; pp < 8; ++pp) {
-            if (p0 + pp >= P) break;
-            const int64_t row = (int64_t)(tile0 + p0 + pp) * DL_ROWS + r_in;
-            if (row >= d_out) continue;
+        for (int pp = 0; pp < PT; ++pp)
+#pragma unroll
+          for (int h = 0; h < DL_RPL; ++h)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) bsum[pp][h][q] = 0.f;
+        for (int kz = 0; kz < ksplit; ++kz) {
+          const float* part = y_part + (int64_t)kz * batch * d_out;
+#pragma unroll
+          for (int pp = 0; pp < PT; ++pp)
+#pragma unroll
+            for (int h = 0; h < DL_RPL; ++h) {
+              const int64_t row = (int64_t)(tile0 + p0 + pp) * DL_ROWS + r_lo + 32 * DL_CWARPS * h;
+              if (p0 + pp < P && row < d_out) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                  if (q < nt) bsum[pp][h][q] += part[(int64_t)D.tok[q] * d_out + row];
+              }
+            }
+        }
+#pragma unroll
+        for (int pp = 0; pp < PT; ++pp)
+#pragma unroll
+          for (int h = 0; h < DL_RPL; ++h) {
+            const int64_t row = (int64_t)(tile0 + p0 + pp) * DL_ROWS + r_lo + 32 * DL_CWARPS * h;
+            if (p0 + pp >= P || row >= d_out) continue;
             float s_row = rs;
             if (!base_only && mode == BD_SCALE_ROW) s_row = ldg_scale(scales, scale_f16, row);
-            float bsum[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int kz = 0; kz < ksplit; ++kz) {
-              const float* part = y_part + (int64_t)kz * batch * d_out + row;
-#pragma unroll
-              for (int q = 0; q < 4; ++q)
-                if (q < nt) bsum[q] += part[(int64_t)tok[q] * d_out];
-            }
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               if (q < nt) {
-                const float v = bsum[q] + (base_only ? 0.f : s_row * __uint_as_float(acc[4 * pp + q]));
+                const float v =
+                    bsum[pp][h][q] + (base_only ? 0.f : s_row * __uint_as_float(acc[DL_TSTRIDE * pp + 4 * h + q]));
+                const int64_t t = D.tok[q];
                 if (y_bf16)
-                  reinterpret_cast<uint16_t*>(y)[(int64_t)tok[q] * d_out + row] = (uint16_t)f2bf_bits(v);
+                  reinterpret_cast<uint16_t*>(y)[t * d_out + row] = (uint16_t)f2bf_bits(v);
                 else
-                  reinterpret_cast<float*>(y)[(int64_t)tok[q] * d_out + row] = v;
+                  reinterpret_cast<float*>(y)[t * d_out + row] = v;
               }
             }
           }
-        }
       }
+      // the descriptor is no longer read
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&dempty[Dr.slot]);
+      Dr.next(DL_DSLOTS);
     }
-    (void)dead;
-    tmem_wait_st4();
+    tmem_wait_st();
   }
   tc_fence_before();
   __syncthreads();
@@ -685,7 +885,31 @@ __global__ void __launch_bounds__(DL_THREADS, 1) k_delta_lut(
 // ------------------------------------------------------------------------------------
 // host side
 // ------------------------------------------------------------------------------------
-size_t delta_lut_smem() { return DL_SMEM; }
+// The kernel's layout needs its dynamic window to start low enough that the tables (on a
+// 64 KB boundary) and at least two ring stages fit: checked once per device from the
+// kernel's static shared memory and the device's reserved shared memory per block.
+static bool dl_layout_fits(const void* fn, bool xbf16) {
+  static std::atomic<uint64_t> ok_bits[2], bad_bits[2];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return false;
+  }
+  const uint64_t bit = dev < 64 ? (1ull << dev) : 0ull;
+  if (bit && (ok_bits[xbf16].load() & bit)) return true;
+  if (bit && (bad_bits[xbf16].load() & bit)) return false;
+  cudaFuncAttributes fa;
+  int reserved = 0;
+  if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess ||
+      cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return false;
+  }
+  const uint32_t start = (uint32_t)reserved + (uint32_t)fa.sharedSizeBytes;
+  const bool fits = dl_layout(start, DL_SMEM, xbf16).stages >= 2;
+  if (bit) (fits ? ok_bits[xbf16] : bad_bits[xbf16]).fetch_or(bit);
+  return fits;
+}
 
 bd_status launch_delta_lut(bool xbf16, const bd_tenant* tenants, bool scale_f16, const int32_t* seg,
                            int max_groups, int max_tc, const void* x, const float* y_part, int ksplit,
@@ -693,7 +917,8 @@ bd_status launch_delta_lut(bool xbf16, const bd_tenant* tenants, bool scale_f16,
                            uint32_t* status, cudaStream_t s) {
   auto kfn = xbf16 ? k_delta_lut<true> : k_delta_lut<false>;
   static std::atomic<uint64_t> attr[2];
-  if (!ensure_dyn_smem(kfn, (int)DL_SMEM, attr[xbf16 ? 1 : 0])) return BD_ERR_CUDA;
+  if (!ensure_dyn_smem(kfn, DL_SMEM, attr[xbf16 ? 1 : 0])) return BD_ERR_CUDA;
+  if (!dl_layout_fits(reinterpret_cast<const void*>(kfn), xbf16)) return BD_ERR_INTERNAL;
   launch_begin(K_DELTA_LUT, s);
   kfn<<<(unsigned)sm_count(), DL_THREADS, DL_SMEM, s>>>(tenants, scale_f16, seg, max_groups, max_tc, x,
                                                        y_part, ksplit, d_out, d_in, (int)batch, y, y_bf16,
