@@ -207,7 +207,7 @@ bd_status bd_prepare_tenant(const uint32_t* signs, const void* scales, int32_t s
 /* The many-token threshold built into the library: a tenant with at least this many
  * tokens in a batch (and a record the tensor-core path supports) goes to the tensor-core
  * delta; every other tenant goes through the lookup-table delta, at most 4 of its tokens
- * per pass over its bits. */
+ * per pass over its bits (a tenant with 5 to 8 tokens is read twice). */
 int32_t bd_tc_min_tokens(void);
 
 /* Bytes of workspace bd_apply_multi needs. */
@@ -220,7 +220,7 @@ size_t bd_apply_workspace_size(int64_t d_out, int64_t d_in, int64_t batch, int32
  * The base product W_base X is computed once for the whole batch; the tokens are
  * grouped by tenant on the device (no host synchronisation). Two delta kernels share the
  * work, chosen per tenant on the device:
- *   - a tenant with at least bd_tc_min_tokens() tokens in the batch (5 as built),
+ *   - a tenant with at least bd_tc_min_tokens() tokens in the batch (9 as built),
  *     stored in the TILED layout with
  *     fp16 scales in GROUP (group_size >= 64), ROW or TENSOR mode (bf16 w_base and
  *     d_in % 64 == 0), is a dense product on the tensor cores, in segments of <= 64 of

@@ -265,16 +265,17 @@ bd_status launch_delta_lut(bool xbf16, const bd_tenant* tenants, bool scale_f16,
                            uint32_t* status, cudaStream_t s);
 
 // A tenant with at least this many tokens in a batch (and a supported record) goes to the
-// tensor-core delta kernel; below it the lookup-table kernel serves all of the tenant's
-// tokens (at most kLutTokens) in one pass over its bits. Both kernels compute the same
-// product, so a build may set another value with -DBD_TC_MIN_TOKENS=n, 1 <= n <= 5, to
-// re-tune it; bd_tc_min_tokens() reports the value built in.
+// tensor-core delta kernel; below it the lookup-table kernel serves the tenant's tokens,
+// kLutTokens of them per pass over its bits (one pass up to 4 tokens, two up to 8). 9 is
+// the crossover measured on B200 over the fused Llama-3-8B calls of the serving workload
+// (a layer took 2.36 ms with 9, 2.52 ms with 5). Both kernels compute the same product, so
+// a build may set another value with -DBD_TC_MIN_TOKENS=n, n >= 1, to re-tune it;
+// bd_tc_min_tokens() reports the value built in.
 #ifndef BD_TC_MIN_TOKENS
-#define BD_TC_MIN_TOKENS 5
+#define BD_TC_MIN_TOKENS 9
 #endif
 constexpr int kTcMinTokens = BD_TC_MIN_TOKENS;
-static_assert(kTcMinTokens >= 1 && kTcMinTokens <= kLutTokens + 1,
-              "lookup groups hold at most kLutTokens tokens of a tenant");
+static_assert(kTcMinTokens >= 1, "the many-token threshold is a token count");
 
 namespace {
 struct ApplyLayout {

@@ -327,13 +327,13 @@ def _many_token_problem(seed, d_out, d_in, counts, mode, G, zero_base=False, x_s
 @pytest.mark.parametrize("layout", [0, 1])
 @pytest.mark.parametrize("mode,G", [(0, 128), (0, 64), (0, 256), (1, 128), (3, 128), (2, 128)])
 def test_many_token_tenants_delta_only(bd, mode, G, layout):
-    """300 tokens (five tensor-core segments), 8 (the smallest many-token tenant), 7, 20 and
-    1 token; 200 rows (a partial 128-row tile), 384 columns (a partial 256-column tile of
-    the serving layout; 768 for groups of 256). Column scales (mode 2) stay on the
-    lookup-table path."""
+    """300 tokens (five tensor-core segments), 9 (the smallest many-token tenant), 8 (two
+    passes of the lookup-table kernel), 20 and 1 token; 200 rows (a partial 128-row tile),
+    384 columns (a partial 256-column tile of the serving layout; 768 for groups of 256).
+    Column scales (mode 2) stay on the lookup-table path."""
     d_out, d_in = 200, (768 if G == 256 else 384)
     wb, tenants, ids, x = _many_token_problem(mode * 7 + G + layout, d_out, d_in,
-                                              [300, 8, 7, 20, 1], mode, G, zero_base=True)
+                                              [300, 9, 8, 20, 1], mode, G, zero_base=True)
     y_ref = O.apply_multi(wb, "bf16", tenants, ids, x, "bf16")
     y, rc, flags = _run(bd, wb, tenants, ids, x, y_dtype="f32", layout=layout)
     assert rc == bd.BD_OK and flags == 0
