@@ -89,6 +89,7 @@ def parse():
     p.add_argument("--compress-layers", type=int, default=N_LAYERS)
     p.add_argument("--no-compress", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-extra", action="store_true", help="skip the decode and mixed workloads")
     p.add_argument("--cpu-seconds", type=float, default=15.0)
     return p.parse_args()
 
@@ -441,6 +442,9 @@ def bench_serving(args, rank, pg, log, peaks):
 
 
 def bench_compress(args, log, peaks):
+    """bd_compress over the 32-layer stack: group-128 scales without and with the 3-sigma
+    clip, row and column scales; each with the 224 independent calls spread over
+    COMPRESS_STREAMS CUDA streams and on a single stream (one call after another)."""
     import torch
     import tenant_serving_b200 as bd
     from workloads import device_weight_pair
@@ -456,63 +460,70 @@ def bench_compress(args, log, peaks):
     log(f"compress: {len(mats)} matrices generated in {time.time() - t0:.1f}s")
     params = sum(d_out * d_in for d_out, d_in, _, _ in mats)
     out = {}
-    for label, clip in (("group128", False), ("group128_clip3", True)):
-        cfg = bd.compress_cfg(mode=bd.BD_SCALE_GROUP, group_size=GROUP, clip=clip, clip_k=3.0)
+    main_s = torch.cuda.current_stream()
+    variants = (("group128", bd.BD_SCALE_GROUP, False), ("group128_clip3", bd.BD_SCALE_GROUP, True),
+                ("row", bd.BD_SCALE_ROW, False), ("col", bd.BD_SCALE_COL, False))
+    for label, mode, clip in variants:
+        cfg = bd.compress_cfg(mode=mode, group_size=GROUP, clip=clip, clip_k=3.0)
         bufs = []
         for d_out, d_in, wb, wf in mats:
             signs = torch.empty((d_out, d_in // 32), dtype=torch.int32, device="cuda")
-            scales = torch.empty((d_out, d_in // GROUP), dtype=torch.float32, device="cuda")
+            scales = torch.empty(bd.scales_shape(mode, d_out, d_in, GROUP), dtype=torch.float32,
+                                 device="cuda")
             ws = torch.empty(max(bd.bd_compress_workspace_size(d_out, d_in, cfg), 16),
                              dtype=torch.uint8, device="cuda")
             bufs.append((signs, scales, ws))
+        # algorithmic bytes: bf16 W_base + W_fine read once, sign bits and fp32 scales written
+        # (the clip's statistics pass is a second read, not counted)
+        scale_bytes = sum((d_out * d_in // GROUP if mode == bd.BD_SCALE_GROUP else
+                           d_out if mode == bd.BD_SCALE_ROW else d_in) * 4 for d_out, d_in, _, _ in mats)
+        alg = params * (4 + 1 / 8) + scale_bytes
+        res = {}
+        for nstreams in (COMPRESS_STREAMS, 1):
+            streams = [torch.cuda.Stream() for _ in range(nstreams)]
 
-        # the matrices are independent: calls go round-robin to COMPRESS_STREAMS streams
-        # (each with its own workspace), so a small matrix's launch ramp and tail overlap
-        # another matrix's kernels; the main stream waits for all of them
-        main_s = torch.cuda.current_stream()
-        streams = [torch.cuda.Stream() for _ in range(COMPRESS_STREAMS)]
+            def one_pass():
+                start = torch.cuda.Event()
+                start.record(main_s)
+                for st in streams:
+                    st.wait_event(start)
+                for i, ((d_out, d_in, wb, wf), (signs, scales, ws)) in enumerate(zip(mats, bufs)):
+                    bd.bd_compress(wb, wf, cfg, signs=signs, scales=scales, workspace=ws,
+                                   stream=streams[i % nstreams])
+                for st in streams:
+                    done = torch.cuda.Event()
+                    done.record(st)
+                    main_s.wait_event(done)
 
-        def one_pass():
-            start = torch.cuda.Event()
-            start.record(main_s)
-            for st in streams:
-                st.wait_event(start)
-            for i, ((d_out, d_in, wb, wf), (signs, scales, ws)) in enumerate(zip(mats, bufs)):
-                st = streams[i % len(streams)]
-                bd.bd_compress(wb, wf, cfg, signs=signs, scales=scales, workspace=ws,
-                               stream=st)
-            for st in streams:
-                done = torch.cuda.Event()
-                done.record(st)
-                main_s.wait_event(done)
-
-        for _ in range(2):
-            one_pass()
-        torch.cuda.synchronize()
-        reps = 3
-        bd.bd_profile_enable(True, capacity=len(mats) * reps * 8 + 16)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(main_s)
-        for _ in range(reps):
-            one_pass()
-        e1.record(main_s)
-        torch.cuda.synchronize()
-        prof = bd.bd_profile_collect()
-        bd.bd_profile_enable(False)
-        ms = e0.elapsed_time(e1) / reps
-        alg = params * (4 + 1 / 8 + 4 / GROUP)  # bf16 W_base + W_fine, sign bits, fp32 scales
-        gbs = alg / (ms / 1e3) / 1e9
-        main = prof.get("scale_signpack", (0, 0.0))
-        main_gbs = alg * reps / (main[1] / 1e3) / 1e9 if main[1] else None
-        out[label] = {"ms_per_stack": ms, "params": params, "gbs": gbs, "frac": gbs / peaks[0],
-                      "streams": COMPRESS_STREAMS,
-                      "tparams_per_s": params / (ms / 1e3) / 1e12,
-                      "kernels": {k: {"launches": v[0], "total_ms": v[1] / reps} for k, v in prof.items()},
-                      "signpack_kernel_gbs": main_gbs}
-        if not clip:
-            out["reconstruct_merged"] = _bench_reconstruct(bd, mats, bufs, streams, main_s,
-                                                           params, peaks)
+            for _ in range(2):
+                one_pass()
+            torch.cuda.synchronize()
+            reps = 3
+            if nstreams == 1:
+                bd.bd_profile_enable(True, capacity=len(mats) * reps * 4 + 16)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(main_s)
+            for _ in range(reps):
+                one_pass()
+            e1.record(main_s)
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / reps
+            key = "streams4" if nstreams > 1 else "stream1"
+            res[key] = {"ms_per_stack": ms, "gbs": alg / (ms / 1e3) / 1e9,
+                        "frac": alg / (ms / 1e3) / 1e9 / peaks[0], "streams": nstreams}
+            if nstreams == 1:
+                # per-kernel device time of the single-stream run (kernels do not overlap)
+                prof = bd.bd_profile_collect()
+                bd.bd_profile_enable(False)
+                res[key]["kernels"] = {k: {"launches": v[0] // reps, "ms_per_stack": v[1] / reps}
+                                       for k, v in prof.items()}
+        out[label] = {"params": params, "bytes_per_stack": alg,
+                      "tparams_per_s": params / (res["streams4"]["ms_per_stack"] / 1e3) / 1e12, **res}
+        if label == "group128":
+            out["reconstruct_merged"] = _bench_reconstruct(
+                bd, mats, bufs, [torch.cuda.Stream() for _ in range(COMPRESS_STREAMS)], main_s, params,
+                peaks)
         del bufs
     del mats
     torch.cuda.empty_cache()
@@ -559,6 +570,116 @@ def _bench_reconstruct(bd, mats, bufs, streams, main_s, params, peaks):
     return {"ms_per_stack": ms, "gbs": gbs, "frac": gbs / peaks[0], "streams": len(streams)}
 
 
+def _time_calls(run, iters, warmup, stream):
+    """Device time of `iters` runs of run() after `warmup` runs, plus the library's
+    per-kernel times of a second timed pass (ms)."""
+    import torch
+    import tenant_serving_b200 as bd
+    for _ in range(warmup):
+        run()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(iters):
+        run()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / iters
+    bd.bd_profile_enable(True, capacity=iters * 64 + 16)
+    for _ in range(iters):
+        run()
+    torch.cuda.synchronize()
+    prof = bd.bd_profile_collect()
+    bd.bd_profile_enable(False)
+    return ms, {k: {"launches": v[0] // iters, "us_per_run": v[1] / iters * 1e3} for k, v in prof.items()}
+
+
+def bench_decode(args, log, peaks):
+    """Decode GEMV: the up_proj shape 14336 x 4096 with a bf16 base, 64 resident tenants
+    (sign words + fp16 group-128 scales, tiled serving layout), 64 tokens, one per tenant
+    (a seeded permutation), x ~ N(0, 1) bf16. The ~646 MB read per call is far larger than
+    L2, so no flush is needed between calls."""
+    import torch
+    import tenant_serving_b200 as bd
+    d_out, d_in, T, B = 14336, 4096, 64, 64
+    g = torch.Generator(device="cuda")
+    g.manual_seed(2000)
+    wb = (torch.randn((d_out, d_in), generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+    recs = []
+    for u in range(T):
+        words = torch.randint(-(2 ** 31), 2 ** 31 - 1, (d_out, d_in // 32), generator=g, device="cuda",
+                              dtype=torch.int32)
+        sc = (0.001 * math.sqrt(2.0 / math.pi) *
+              torch.exp(0.1 * torch.randn((d_out, d_in // GROUP), generator=g, device="cuda"))).to(torch.float16)
+        tw, ts = bd.bd_prepare_tenant(words, sc, bd.BD_SCALE_GROUP, GROUP, d_out, d_in)
+        recs.append((tw, ts, bd.BD_SCALE_GROUP, GROUP, bd.BD_LAYOUT_TILED))
+    table = bd.TenantTable(recs, "cuda")
+    ids = torch.from_numpy(np.random.default_rng(2000).permutation(T).astype(np.int32)).cuda()
+    x = (torch.randn((B, d_in), generator=g, device="cuda")).to(torch.bfloat16)
+    y = torch.empty((B, d_out), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(bd.bd_apply_workspace_size(d_out, d_in, B, T), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    ms, kern = _time_calls(lambda: bd.bd_apply_multi(wb, table, ids, x, y=y, workspace=ws), 20, 3, stream)
+    alg = d_out * d_in * 2 + T * (d_out * d_in // 8 + d_out * (d_in // GROUP) * 2) + B * (d_in + d_out) * 2
+    del recs, table
+    return {"workload": "decode: up_proj 14336x4096 bf16 base, 64 tenants (group-128 fp16 scales), "
+                        "64 tokens one per tenant",
+            "us_per_call": ms * 1e3, "tokens_per_s": B / (ms / 1e3), "bytes_per_call": alg,
+            "gbs": alg / (ms / 1e3) / 1e9, "frac": alg / (ms / 1e3) / 1e9 / peaks[0], "kernels": kern}
+
+
+def bench_mixed(args, log, peaks):
+    """Mixed batch: one Llama-3-8B-shaped layer applied as its 7 projections, 32 resident
+    tenants with per-axis fp16 scale vectors (row or column per (tenant, projection),
+    Bernoulli(1/2) from the seed), 256 tokens with Zipf(1.1) ids over the 32 tenants,
+    bf16 base product on the tensor cores. One run = the 7 calls (~1.25 GB read, far
+    larger than L2)."""
+    import torch
+    import tenant_serving_b200 as bd
+    B, T = 256, 32
+    rng = np.random.default_rng(3000)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(3000)
+    ids_host = zipf_ids_host(rng, B, T, ZIPF_S)
+    ids = torch.from_numpy(ids_host).cuda()
+    distinct = np.unique(ids_host)
+    calls, alg = [], 0
+    for name, d_out, d_in in LLAMA3_8B_PROJECTIONS:
+        wb = (torch.randn((d_out, d_in), generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+        recs, scale_bytes = [], []
+        for u in range(T):
+            mode = bd.BD_SCALE_ROW if rng.random() < 0.5 else bd.BD_SCALE_COL
+            words = torch.randint(-(2 ** 31), 2 ** 31 - 1, (d_out, d_in // 32), generator=g, device="cuda",
+                                  dtype=torch.int32)
+            n = d_out if mode == bd.BD_SCALE_ROW else d_in
+            sc = (0.001 * math.sqrt(2.0 / math.pi) *
+                  torch.exp(0.1 * torch.randn((n,), generator=g, device="cuda"))).to(torch.float16)
+            tw, ts = bd.bd_prepare_tenant(words, sc, mode, GROUP, d_out, d_in)
+            recs.append((tw, ts, mode, GROUP, bd.BD_LAYOUT_TILED))
+            scale_bytes.append(n * 2)
+        table = bd.TenantTable(recs, "cuda")
+        x = torch.randn((B, d_in), generator=g, device="cuda").to(torch.bfloat16)
+        y = torch.empty((B, d_out), dtype=torch.bfloat16, device="cuda")
+        ws = torch.empty(bd.bd_apply_workspace_size(d_out, d_in, B, T), dtype=torch.uint8, device="cuda")
+        calls.append((wb, table, x, y, ws, recs))
+        alg += d_out * d_in * 2 + sum(d_out * d_in // 8 + scale_bytes[u] for u in distinct) + B * (d_in + d_out) * 2
+    stream = torch.cuda.current_stream()
+
+    def run():
+        for wb, table, x, y, ws, _ in calls:
+            bd.bd_apply_multi(wb, table, ids, x, y=y, workspace=ws)
+
+    ms, kern = _time_calls(run, 20, 3, stream)
+    del calls
+    torch.cuda.empty_cache()
+    return {"workload": "mixed: one Llama-3-8B-shaped layer (7 projections), 32 tenants with per-axis "
+                        "fp16 scales (row or column per tenant and projection), 256 tokens, Zipf(1.1) ids",
+            "us_per_layer": ms * 1e3, "tokens_per_s": B / (ms / 1e3), "bytes_per_layer": alg,
+            "distinct_tenants": int(len(distinct)), "gbs": alg / (ms / 1e3) / 1e9,
+            "frac": alg / (ms / 1e3) / 1e9 / peaks[0], "kernels": kern}
+
+
 # ------------------------------------------------------------------------------------
 # oracle on host cores (cpu_baseline and the reference arm)
 # ------------------------------------------------------------------------------------
@@ -573,7 +694,7 @@ def oracle_sample(seconds: float):
         from threadpoolctl import threadpool_info
         threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     except Exception:
-        threads = os.cpu_count() or 1
+        threads = 1
     rng = np.random.default_rng(11)
     B = BATCH
     ids = zipf_ids_host(rng, B, N_TENANTS, ZIPF_S)
@@ -596,6 +717,22 @@ def oracle_sample(seconds: float):
             f"{rows_per} output rows each, batch {B}, {N_TENANTS} tenants, Zipf(1.1) ids; "
             f"time scaled by output rows to the 32-layer step")
     return B / step_seconds, threads, desc
+
+
+def cpu_baseline(seconds: float) -> dict:
+    """The oracle's serving sample on the host: with the BLAS pool as configured (the
+    reported value) and with one thread. cores = the host's logical CPUs; blas_threads =
+    the threads the multi-threaded run could use."""
+    value, threads, desc = oracle_sample(seconds)
+    one = None
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            one, _, _ = oracle_sample(max(2.0, seconds / 3))
+    except Exception:
+        pass
+    return {"value": value, "unit": "tokens/s", "cores": threads, "host_cpus": os.cpu_count(),
+            "blas_threads": threads, "single_thread_value": one, "kind": "oracle", "sample": desc}
 
 
 def reference_arm(args):
@@ -650,9 +787,12 @@ def main():
         barrier(pg)
     res = bench_serving(args, rank, pg, log, peaks)
     cpu = None
+    dec = mix = None
+    if rank == 0 and world == 1 and not args.no_extra:
+        dec = bench_decode(args, log, peaks)
+        mix = bench_mixed(args, log, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, cores, desc = oracle_sample(args.cpu_seconds)
-        cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc}
+        cpu = cpu_baseline(args.cpu_seconds)
     if rank == 0:
         line = {
             "metric": METRIC, "value": res["value"], "unit": "tokens/s", "n_gpus": world,
@@ -666,6 +806,7 @@ def main():
             "ms_per_step_profiled": res["ms_per_step_profiled"],
             "distinct_tenants_mean": res["distinct_tenants_mean"],
             "kernels": res["kernels"], "kernel_rates": res["kernel_rates"], "compress": comp,
+            "decode": dec, "mixed": mix,
         }
         print(json.dumps(line))
     if pg is not None:

@@ -11,7 +11,7 @@ namespace bd {
 static const char* const kKernelNames[K_KIND_COUNT] = {
     "delta_stats",       "scale_signpack", "col_scale_signpack",
     "scale_final",       "reconstruct",  "tenant_bucket",  "base_gemv",
-    "base_tc",           "delta_lut",    "clip_fixup",     "prepare",
+    "base_tc",           "delta_lut",    "prepare",
     "tc_gather",         "delta_tc",     "selftest_wait",
 };
 

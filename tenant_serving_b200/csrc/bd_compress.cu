@@ -7,7 +7,7 @@
 //   sign bit = !(delta_c < 0), packed LSB-first along d_in into uint32 words.
 //
 // Kernels (all HBM-bound streams; 16-byte coalesced loads of both inputs):
-//   k_delta_stats      clip statistics (ROW / COL / TENSOR modes): sums of the shifted
+//   k_delta_stats      clip statistics: sums of the shifted
 //                      delta and of its square, in fp64 per element, one pair per block;
 //                      the last block merges the pairs in a fixed order -> mean, std, lo,
 //                      hi and the fp32 thresholds the main pass compares with.
@@ -19,11 +19,6 @@
 //                      keeping fp64 column sums in registers; fp64 partials per tile.
 //   k_scale_final      fixed-order reduction of the partials into row / column / tensor
 //                      scales (deterministic, no atomics).
-//   GROUP mode with the clip reads the matrices once: k_scale_signpack writes the
-//   unclipped signs and scales, the fp64 statistics (finished by its last block) and each
-//   group's smallest and largest delta; k_clip_fixup then re-reads only the groups with a
-//   delta outside [lo, hi] and rewrites their signs and scales. The result is the same as
-//   clipping first: a group inside the bounds is not changed by the clamp.
 #include "bd_internal.cuh"
 
 #include <math.h>
@@ -249,37 +244,21 @@ __global__ void __launch_bounds__(256) k_delta_stats(const uint4* __restrict__ w
 // A task is (row, segment of seg_chunks chunks); a chunk is 32 lanes x 16 bytes. Column
 // arithmetic is 32-bit (d_in < 2^31 is checked on the host) and the group size is a power
 // of two, so group indices are shifts.
-// STATS (GROUP mode, no clip applied yet): the first pass of the clip. Besides the
-// unclipped signs and scales it accumulates the fp64 shifted sums of the exact deltas
-// (finished by the last block into the clip parameters) and writes every group's smallest
-// and largest fp32 delta, so that the fix-up pass re-reads only the groups the clip changes.
-template <bool BF16, int SEGC, bool CLIP, bool GROUP, bool STATS>
+template <bool BF16, int SEGC, bool CLIP, bool GROUP>
 __global__ void __launch_bounds__(256, 4) k_scale_signpack(
     const uint8_t* __restrict__ wb, const uint8_t* __restrict__ wf, int64_t d_out, int d_in,
     int lg, int seg_chunks, int nseg, const ClipParams* __restrict__ clipp,
-    uint32_t* __restrict__ signs, float* __restrict__ scales, double* __restrict__ partials,
-    float2* __restrict__ minmax, double* __restrict__ stat_parts, unsigned int* __restrict__ counter,
-    double clip_k, ClipParams* __restrict__ clip_out, double* __restrict__ stats_out) {
-  static_assert(!STATS || (GROUP && !CLIP), "the statistics variant is the unclipped group pass");
+    uint32_t* __restrict__ signs, float* __restrict__ scales, double* __restrict__ partials) {
   using V = Vec<BF16>;
   constexpr int VEC = V::N;
   constexpr int CHUNK = 32 * VEC;             // columns per chunk
   constexpr int LPW = 32 / VEC;               // lanes per 32-bit sign word
   constexpr int ESZ = BF16 ? 2 : 4;
   const int lane = threadIdx.x & 31;
-  const int64_t task0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const bool have_task = task0 < d_out * (int64_t)nseg;
-  if (!STATS && !have_task) return;
-  // the statistics variant keeps idle warps to the end: the block reduction needs them
-  const int64_t task = have_task ? task0 : 0;
+  const int64_t task = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (task >= d_out * (int64_t)nseg) return;
   const int64_t row = task / nseg;
   const int seg = (int)(task - row * nseg);
-  double shift = 0.0, st1 = 0.0, st2 = 0.0;
-  if (STATS) {
-    double d0[VEC];
-    V::delta64(reinterpret_cast<const uint4*>(wb)[0], reinterpret_cast<const uint4*>(wf)[0], d0);
-    shift = d0[0];
-  }
 
   ClipF cp{0.f, 0.f, 0.f, 0.f};
   if (CLIP) cp = load_clip(clipp);
@@ -296,8 +275,7 @@ __global__ void __launch_bounds__(256, 4) k_scale_signpack(
   double acc_row = 0.0;   // ROW / TENSOR: this lane's share of the segment sum
   double acc_grp = 0.0;   // GROUP with G > CHUNK: running group sum (all lanes equal)
 
-  float gmin = 3.4e38f, gmax = -3.4e38f;  // GROUP with G > CHUNK: running extremes
-  for (int c0 = 0; c0 < seg_chunks && have_task; c0 += SEGC) {
+  for (int c0 = 0; c0 < seg_chunks; c0 += SEGC) {
     uint4 b[SEGC], f[SEGC];
     bool valid[SEGC];
 #pragma unroll
@@ -316,7 +294,6 @@ __global__ void __launch_bounds__(256, 4) k_scale_signpack(
       const int col = chunk_col0 + lane * VEC;
       uint32_t m = 0;
       float a = 0.f;
-      float lmin = 3.4e38f, lmax = -3.4e38f;
       if (valid[u]) {
         float d[VEC];
         V::delta(b[u], f[u], d);
@@ -325,20 +302,6 @@ __global__ void __launch_bounds__(256, 4) k_scale_signpack(
           const float dc = CLIP ? clamp_delta(d[k], cp) : d[k];
           m |= (dc < 0.f ? 0u : 1u) << k;
           a += fabsf(dc);
-          if (STATS) {
-            lmin = fminf(lmin, d[k]);
-            lmax = fmaxf(lmax, d[k]);
-          }
-        }
-        if (STATS) {
-          double d64[VEC];
-          V::delta64(b[u], f[u], d64);  // exact difference of the stored values
-#pragma unroll
-          for (int k = 0; k < VEC; ++k) {
-            const double t = d64[k] - shift;
-            st1 += t;
-            st2 = fma(t, t, st2);
-          }
         }
       }
       // pack: LPW lanes x VEC bits -> one word, lane order = column order (LSB first)
@@ -351,36 +314,13 @@ __global__ void __launch_bounds__(256, 4) k_scale_signpack(
         if (G <= CHUNK) {
           float s = a;
           for (int o = 1; o < lpg; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-          if (STATS) {
-            for (int o = 1; o < lpg; o <<= 1) {
-              lmin = fminf(lmin, __shfl_xor_sync(0xffffffffu, lmin, o));
-              lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
-            }
-          }
-          if (valid[u] && (lane & (lpg - 1)) == 0) {
-            srow_s[col >> lg] = s * invG;
-            if (STATS) minmax[row * (int64_t)(d_in >> lg) + (col >> lg)] = make_float2(lmin, lmax);
-          }
+          if (valid[u] && (lane & (lpg - 1)) == 0) srow_s[col >> lg] = s * invG;
         } else {
           const float s = warp_sum_f(a);
           acc_grp += (double)s;
-          if (STATS) {
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-              lmin = fminf(lmin, __shfl_xor_sync(0xffffffffu, lmin, o));
-              lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
-            }
-            gmin = fminf(gmin, lmin);
-            gmax = fmaxf(gmax, lmax);
-          }
           if (((chunk_col0 + CHUNK) & (G - 1)) == 0 || chunk_col0 + CHUNK >= d_in) {
-            if (lane == 0) {
-              srow_s[chunk_col0 >> lg] = (float)(acc_grp * (double)invG);
-              if (STATS) minmax[row * (int64_t)(d_in >> lg) + (chunk_col0 >> lg)] = make_float2(gmin, gmax);
-            }
+            if (lane == 0) srow_s[chunk_col0 >> lg] = (float)(acc_grp * (double)invG);
             acc_grp = 0.0;
-            gmin = 3.4e38f;
-            gmax = -3.4e38f;
           }
         }
       } else {
@@ -391,76 +331,6 @@ __global__ void __launch_bounds__(256, 4) k_scale_signpack(
   if (!GROUP) {
     acc_row = warp_sum_d(acc_row);
     if (lane == 0) partials[row * nseg + seg] = acc_row;
-  }
-  if (STATS)
-    stats_block_finish(st1, st2, stat_parts, counter, shift, d_out * (int64_t)d_in, clip_k, clip_out,
-                       stats_out);
-}
-
-// ------------------------------------------------------------------------------------
-// clip fix-up for GROUP mode: re-read only the groups the clip changes
-// ------------------------------------------------------------------------------------
-// A group whose fp32 deltas all satisfy lo_up <= d <= hi_dn is left as it is by the clamp,
-// so the unclipped pass already wrote its final signs and scale. Every other group is read
-// again, clamped, and its signs and scale are rewritten. A warp checks 32 groups at a time
-// (one per lane) and then recomputes the flagged ones together.
-template <bool BF16>
-__global__ void __launch_bounds__(256) k_clip_fixup(const uint8_t* __restrict__ wb,
-                                                    const uint8_t* __restrict__ wf, int64_t d_out,
-                                                    int d_in, int lg,
-                                                    const ClipParams* __restrict__ clipp,
-                                                    const float2* __restrict__ minmax,
-                                                    uint32_t* __restrict__ signs,
-                                                    float* __restrict__ scales) {
-  using V = Vec<BF16>;
-  constexpr int VEC = V::N;
-  constexpr int CHUNK = 32 * VEC;
-  constexpr int LPW = 32 / VEC;
-  constexpr int ESZ = BF16 ? 2 : 4;
-  const int lane = threadIdx.x & 31;
-  const ClipF cp = load_clip(clipp);
-  const int G = 1 << lg;
-  const int64_t gpr = d_in >> lg;
-  const int64_t ngroups = d_out * gpr;
-  const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  for (int64_t g0 = (((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5) * 32; g0 < ngroups;
-       g0 += warps * 32) {
-    bool flag = false;
-    if (g0 + lane < ngroups) {
-      const float2 mm = minmax[g0 + lane];
-      flag = mm.x < cp.lo_up || mm.y > cp.hi_dn;
-    }
-    uint32_t mask = __ballot_sync(0xffffffffu, flag);
-    while (mask) {
-      const int64_t g = g0 + (__ffs(mask) - 1);
-      mask &= mask - 1;
-      const int64_t row = g / gpr;
-      const int gc0 = (int)(g - row * gpr) << lg;
-      const uint8_t* rb = wb + row * (int64_t)d_in * ESZ;
-      const uint8_t* rf = wf + row * (int64_t)d_in * ESZ;
-      float a = 0.f;
-      for (int c0 = 0; c0 < G; c0 += CHUNK) {
-        const int colg = c0 + lane * VEC;  // column inside the group
-        uint32_t m = 0;
-        if (colg < G) {
-          const int col = gc0 + colg;
-          float d[VEC];
-          V::delta(ldg_stream(rb + (int64_t)col * ESZ), ldg_stream(rf + (int64_t)col * ESZ), d);
-#pragma unroll
-          for (int k = 0; k < VEC; ++k) {
-            const float dc = clamp_delta(d[k], cp);
-            m |= (dc < 0.f ? 0u : 1u) << k;
-            a += fabsf(dc);
-          }
-        }
-        uint32_t v = m << (VEC * (lane & (LPW - 1)));
-#pragma unroll
-        for (int o = 1; o < LPW; o <<= 1) v |= __shfl_xor_sync(0xffffffffu, v, o);
-        if (colg < G && (lane & (LPW - 1)) == 0) signs[row * (int64_t)(d_in >> 5) + ((gc0 + colg) >> 5)] = v;
-      }
-      const float sum = warp_sum_f(a);
-      if (lane == 0) scales[g] = sum * (1.0f / (float)G);
-    }
   }
 }
 
@@ -578,7 +448,6 @@ namespace {
 
 struct CompressPlan {
   bool bf16;
-  bool selective;     // GROUP + clip: one pass + fix-up of the groups the clip changes
   int chunk;          // columns per warp chunk
   int seg_chunks;     // chunks per task (GROUP / ROW / TENSOR)
   int nseg;           // tasks per row
@@ -587,13 +456,11 @@ struct CompressPlan {
   int col_tile;       // rows per tile (COL)
   int64_t nchunks;    // chunks per row
   int64_t ntile;      // row tiles (COL)
-  size_t off_clip, off_cnt, off_stats, off_part, off_mm, total;
+  size_t off_clip, off_cnt, off_stats, off_part, total;
 };
 
-// selective: plan the one-pass clip of GROUP mode (it needs a min / max pair per group);
-// otherwise a clip takes a statistics pass over both matrices first
 bd_status plan_compress(int32_t dtype, int64_t d_out, int64_t d_in, const bd_compress_cfg* cfg,
-                        bool selective, CompressPlan* p) {
+                        CompressPlan* p) {
   if (!cfg) return BD_ERR_NULL;
   if (dtype != BD_F32 && dtype != BD_BF16) return BD_ERR_DTYPE;
   if (d_out < 1 || d_in < 32 || (d_in % 32) != 0) return BD_ERR_SHAPE;
@@ -606,7 +473,6 @@ bd_status plan_compress(int32_t dtype, int64_t d_out, int64_t d_in, const bd_com
     if (G < 32 || !is_pow2(G) || (d_in % G) != 0) return BD_ERR_CONFIG;
   }
   p->bf16 = dtype == BD_BF16;
-  p->selective = selective && cfg->clip && cfg->mode == BD_SCALE_GROUP;
   p->chunk = p->bf16 ? 256 : 128;
   p->nchunks = (d_in + p->chunk - 1) / p->chunk;
   const int sms = sm_count();
@@ -632,8 +498,7 @@ bd_status plan_compress(int32_t dtype, int64_t d_out, int64_t d_in, const bd_com
   p->off_cnt = off;
   off = align_up(off + sizeof(unsigned int), 256);
   p->off_stats = off;
-  const int parts = p->selective ? p->main_blocks : p->stats_blocks;
-  off = align_up(off + (size_t)parts * 2 * sizeof(double), 256);
+  off = align_up(off + (size_t)p->stats_blocks * 2 * sizeof(double), 256);
   p->off_part = off;
   size_t part = 0;
   if (cfg->mode == BD_SCALE_ROW || cfg->mode == BD_SCALE_TENSOR)
@@ -641,8 +506,6 @@ bd_status plan_compress(int32_t dtype, int64_t d_out, int64_t d_in, const bd_com
   else if (cfg->mode == BD_SCALE_COL)
     part = (size_t)p->ntile * d_in * sizeof(double);
   off = align_up(off + part, 256);
-  p->off_mm = off;
-  if (p->selective) off = align_up(off + (size_t)d_out * (size_t)(d_in / G) * sizeof(float2), 256);
   p->total = off;
   return BD_OK;
 }
@@ -662,7 +525,7 @@ bd_status launch_compress(const CompressPlan& p, const void* w_base, const void*
     // the last-block ticket of the statistics starts from zero in every call
     BD_CUDA_TRY(cudaMemsetAsync(counter, 0, sizeof(unsigned int), s));
   }
-  if (clip && !p.selective) {
+  if (clip) {
     launch_begin(K_DELTA_STATS, s);
     k_delta_stats<BF16><<<p.stats_blocks, 256, 0, s>>>((const uint4*)w_base, (const uint4*)w_fine,
                                                        nvec, d_out * d_in, (double)cfg->clip_k,
@@ -692,36 +555,21 @@ bd_status launch_compress(const CompressPlan& p, const void* w_base, const void*
   if (group)
     while ((1 << lg) < cfg->group_size) ++lg;
   const int din = (int)d_in;
-  float2* minmax = reinterpret_cast<float2*>(ws + p.off_mm);
-#define BD_SIGNPACK(SEGC, CLIP, GRP, STATS)                                                     \
-  k_scale_signpack<BF16, SEGC, CLIP, GRP, STATS><<<blocks, 256, 0, s>>>(                        \
-      (const uint8_t*)w_base, (const uint8_t*)w_fine, d_out, din, lg, p.seg_chunks, p.nseg,      \
-      clipp, signs, scales, part, minmax, stat_parts, counter, (double)cfg->clip_k, clipp, stats_out)
+#define BD_SIGNPACK(SEGC, CLIP, GRP)                                                           \
+  k_scale_signpack<BF16, SEGC, CLIP, GRP><<<blocks, 256, 0, s>>>(                              \
+      (const uint8_t*)w_base, (const uint8_t*)w_fine, d_out, din, lg, p.seg_chunks, p.nseg,    \
+      clipp, signs, scales, part)
   launch_begin(K_SCALE_SIGNPACK, s);
-  if (p.selective) {
-    if (p.seg_chunks >= 4) BD_SIGNPACK(4, false, true, true);
-    else BD_SIGNPACK(2, false, true, true);
-  } else if (p.seg_chunks >= 4) {
-    if (clip) { if (group) BD_SIGNPACK(4, true, true, false); else BD_SIGNPACK(4, true, false, false); }
-    else { if (group) BD_SIGNPACK(4, false, true, false); else BD_SIGNPACK(4, false, false, false); }
+  if (p.seg_chunks >= 4) {
+    if (clip) { if (group) BD_SIGNPACK(4, true, true); else BD_SIGNPACK(4, true, false); }
+    else { if (group) BD_SIGNPACK(4, false, true); else BD_SIGNPACK(4, false, false); }
   } else {
-    if (clip) { if (group) BD_SIGNPACK(2, true, true, false); else BD_SIGNPACK(2, true, false, false); }
-    else { if (group) BD_SIGNPACK(2, false, true, false); else BD_SIGNPACK(2, false, false, false); }
+    if (clip) { if (group) BD_SIGNPACK(2, true, true); else BD_SIGNPACK(2, true, false); }
+    else { if (group) BD_SIGNPACK(2, false, true); else BD_SIGNPACK(2, false, false); }
   }
 #undef BD_SIGNPACK
   launch_end(K_SCALE_SIGNPACK, s);
   BD_LAUNCH_CHECK();
-  if (p.selective) {
-    const int64_t ngroups = d_out * (d_in >> lg);
-    int64_t fblocks = (ngroups + 255) / 256;  // one group per thread for the check
-    const int64_t cap = (int64_t)sm_count() * 8;
-    if (fblocks > cap) fblocks = cap;
-    launch_begin(K_CLIP_FIXUP, s);
-    k_clip_fixup<BF16><<<(unsigned)fblocks, 256, 0, s>>>((const uint8_t*)w_base, (const uint8_t*)w_fine,
-                                                         d_out, din, lg, clipp, minmax, signs, scales);
-    launch_end(K_CLIP_FIXUP, s);
-    BD_LAUNCH_CHECK();
-  }
   if (cfg->mode == BD_SCALE_ROW) {
     launch_begin(K_SCALE_FINAL, s);
     k_row_final<<<(unsigned)((d_out + 255) / 256), 256, 0, s>>>(part, p.nseg, d_out, d_in, scales);
@@ -740,9 +588,8 @@ bd_status launch_compress(const CompressPlan& p, const void* w_base, const void*
 // Host-side checks of a compress call (nothing is launched); fills the plan.
 bd_status compress_check(const void* w_base, const void* w_fine, int32_t dtype, int64_t d_out,
                          int64_t d_in, const bd_compress_cfg* cfg, const uint32_t* signs_out,
-                         const float* scales_out, const double* stats_out, bool selective,
-                         CompressPlan* p) {
-  bd_status st = plan_compress(dtype, d_out, d_in, cfg, selective, p);
+                         const float* scales_out, const double* stats_out, CompressPlan* p) {
+  bd_status st = plan_compress(dtype, d_out, d_in, cfg, p);
   if (st != BD_OK) return st;
   if (!w_base || !w_fine || !signs_out || !scales_out) return BD_ERR_NULL;
   if (!aligned16(w_base) || !aligned16(w_fine) || !aligned16(signs_out) || !aligned16(scales_out))
@@ -772,7 +619,7 @@ bd_status compress_impl(const void* w_base, const void* w_fine, int32_t dtype, i
                         cudaStream_t s) {
   CompressPlan p;
   bd_status st = compress_check(w_base, w_fine, dtype, d_out, d_in, cfg, signs_out, scales_out,
-                                stats_out, true, &p);
+                                stats_out, &p);
   if (st != BD_OK) return st;
   return compress_run(p, w_base, w_fine, d_out, d_in, cfg, signs_out, scales_out, stats_out,
                       workspace, ws_bytes, s);
@@ -780,9 +627,9 @@ bd_status compress_impl(const void* w_base, const void* w_fine, int32_t dtype, i
 
 size_t compress_workspace_size(int64_t d_out, int64_t d_in, const bd_compress_cfg* cfg) {
   CompressPlan p;
-  if (plan_compress(BD_BF16, d_out, d_in, cfg, true, &p) != BD_OK) return 0;
+  if (plan_compress(BD_BF16, d_out, d_in, cfg, &p) != BD_OK) return 0;
   CompressPlan q;
-  plan_compress(BD_F32, d_out, d_in, cfg, true, &q);
+  plan_compress(BD_F32, d_out, d_in, cfg, &q);
   return p.total > q.total ? p.total : q.total;
 }
 
@@ -844,11 +691,10 @@ extern "C" bd_status bd_compress_noalloc(const void* w_base, const void* w_fine,
                                          int64_t d_out, int64_t d_in, const bd_compress_cfg* cfg,
                                          uint32_t* signs_out, float* scales_out,
                                          double* stats_out, void* stream) {
-  // the arguments first, as for bd_compress; the clip takes the statistics-pass route,
-  // whose scratch stays small for GROUP mode at any size
+  // the arguments first, as for bd_compress
   bd::CompressPlan p;
   bd_status st = bd::compress_check(w_base, w_fine, dtype, d_out, d_in, cfg, signs_out, scales_out,
-                                    stats_out, false, &p);
+                                    stats_out, &p);
   if (st != BD_OK) return st;
   if (p.total > bd::kNoAllocScratchBytes) return BD_ERR_WORKSPACE;
   void* scratch = nullptr;

@@ -36,7 +36,6 @@ enum KernelKind : int32_t {
   K_BASE_GEMV,           // CUDA-core base product for small batches / fp32
   K_BASE_TC,             // tcgen05 base product (bf16, fp32 accumulation in TMEM)
   K_DELTA_LUT,           // per-tenant sign-LUT delta product + combine
-  K_CLIP_FIXUP,          // compress: re-read of the groups the clip changes
   K_PREPARE,             // re-tiling of a tenant into the serving layout
   K_TC_GATHER,           // gather + fp16 scaling of the tensor-core segments' tokens
   K_DELTA_TC,            // tcgen05 delta product of many-token tenants + combine

@@ -263,7 +263,8 @@ def test_launches_are_counted(bd):
     wb, tenants, ids, x = _problem(1, 128, 256, 4, 2, (0,))
     _run(bd, wb, tenants, ids, x)
     assert bd.bd_launch_count() - n0 == 3  # bucket, base product, lookup-table delta
-    # from 6 tokens in a batch on the tensor-core delta (gather + product) is launched too
+    # a tenant with at least bd_tc_min_tokens() tokens in the batch takes the tensor-core
+    # delta (gather + product): two launches more
     n0 = bd.bd_launch_count()
     wb, tenants, ids, x = _problem(1, 128, 256, 16, 2, (0,))
     _run(bd, wb, tenants, ids, x)
