@@ -570,6 +570,78 @@ def _bench_reconstruct(bd, mats, bufs, streams, main_s, params, peaks):
     return {"ms_per_stack": ms, "gbs": gbs, "frac": gbs / peaks[0], "streams": len(streams)}
 
 
+def bench_cold_start(args, log, peaks):
+    """Cold start of one tenant, as the per-axis delta page measures it: all 224 modules of
+    the 32-layer Llama-3-8B stack (group-128 fp16 scales, 981 MB of packed records in
+    pinned host memory) loaded by the tenant cache with one transfer per module, against
+    loading the dense bf16 merged weights of the same stack (13.96 GB: 32 transfers of one
+    layer's 436 MB from pinned host memory). Device time on the copy stream."""
+    import torch
+    import tenant_serving_b200 as bd
+    mods = [(d_out, d_in, GROUP) for _ in range(N_LAYERS) for _, d_out, d_in in LLAMA3_8B_PROJECTIONS]
+    rng = np.random.default_rng(4000)
+    t0 = time.time()
+    records = []
+    for d_out, d_in, g in mods:
+        words = rng.integers(0, 2 ** 32, size=(d_out, d_in // 32), dtype=np.uint32)
+        sc = (0.001 * math.sqrt(2.0 / math.pi) * np.exp(0.1 * rng.standard_normal((d_out, d_in // g)))
+              ).astype(np.float16)
+        records.append(bd.bd_prepare_record_host(words, sc, bd.BD_SCALE_GROUP, g, d_out, d_in, pin=True))
+    log(f"cold start: {len(records)} records packed in {time.time() - t0:.1f}s")
+    rec_bytes = sum(r.numel() for r in records)
+    # two host tenants with the same records and one slot: every prefetch is a full load
+    cache = bd.TenantCache(mods, n_host_tenants=2, n_slots=1)
+    for u in range(2):
+        for m, r in enumerate(records):
+            cache.register(u, m, r, bd.BD_SCALE_GROUP, GROUP)
+    cs = torch.cuda.Stream()
+    times = []
+    for k in range(6):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(cs)
+        _, n, ticket = cache.prefetch(np.array([k % 2], dtype=np.int32), stream=cs)
+        e1.record(cs)
+        cache.acquire(ticket, stream=cs)
+        cache.release(ticket, stream=cs)
+        torch.cuda.synchronize()
+        if k >= 2:
+            times.append(e0.elapsed_time(e1))
+        assert n == 1
+    delta_ms = statistics.median(times)
+    stats = cache.resident()[1]
+    cache.close()
+    del records
+    # dense merged weights: one layer's bf16 weights, pinned, moved 32 times
+    layer_elems = sum(d_out * d_in for _, d_out, d_in in LLAMA3_8B_PROJECTIONS)
+    host_layer = torch.empty(layer_elems, dtype=torch.bfloat16).pin_memory()
+    host_layer.view(torch.int16).copy_(torch.from_numpy(
+        rng.integers(-2 ** 15, 2 ** 15, size=layer_elems, dtype=np.int16)))
+    dev_layer = torch.empty(layer_elems, dtype=torch.bfloat16, device="cuda")
+    dtimes = []
+    for k in range(3):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(cs)
+        with torch.cuda.stream(cs):
+            for _ in range(N_LAYERS):
+                dev_layer.copy_(host_layer, non_blocking=True)
+        e1.record(cs)
+        torch.cuda.synchronize()
+        if k >= 1:
+            dtimes.append(e0.elapsed_time(e1))
+    dense_ms = statistics.median(dtimes)
+    dense_bytes = layer_elems * 2 * N_LAYERS
+    del host_layer, dev_layer
+    torch.cuda.empty_cache()
+    return {"workload": "one tenant of the 32-layer Llama-3-8B stack, group-128 fp16 scales, pinned host "
+                        "memory -> HBM",
+            "delta_ms": delta_ms, "delta_bytes": rec_bytes, "delta_gbs": rec_bytes / (delta_ms / 1e3) / 1e9,
+            "delta_transfers": len(mods) + 1, "dense_bf16_ms": dense_ms, "dense_bytes": dense_bytes,
+            "dense_gbs": dense_bytes / (dense_ms / 1e3) / 1e9, "speedup": dense_ms / delta_ms,
+            "cache_stats": stats}
+
+
 def _time_calls(run, iters, warmup, stream):
     """Device time of `iters` runs of run() after `warmup` runs, plus the library's
     per-kernel times of a second timed pass (ms)."""
@@ -788,9 +860,11 @@ def main():
     res = bench_serving(args, rank, pg, log, peaks)
     cpu = None
     dec = mix = None
+    cold = None
     if rank == 0 and world == 1 and not args.no_extra:
         dec = bench_decode(args, log, peaks)
         mix = bench_mixed(args, log, peaks)
+        cold = bench_cold_start(args, log, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(args.cpu_seconds)
     if rank == 0:
@@ -806,7 +880,7 @@ def main():
             "ms_per_step_profiled": res["ms_per_step_profiled"],
             "distinct_tenants_mean": res["distinct_tenants_mean"],
             "kernels": res["kernels"], "kernel_rates": res["kernel_rates"], "compress": comp,
-            "decode": dec, "mixed": mix,
+            "decode": dec, "mixed": mix, "cold_start": cold,
         }
         print(json.dumps(line))
     if pg is not None:

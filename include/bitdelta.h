@@ -210,6 +210,112 @@ bd_status bd_prepare_tenant(const uint32_t* signs, const void* scales, int32_t s
  * per pass over its bits (a tenant with 5 to 8 tokens is read twice). */
 int32_t bd_tc_min_tokens(void);
 
+/* ---------------------------------------------------------------------------------- */
+/* host-resident tenant cache and packed-delta loader                                  */
+/* ---------------------------------------------------------------------------------- */
+/* "Per-Axis Weight Deltas", Key Contributions item 4 and Implementation details: packed
+ * deltas (1-bit signs along the input axis + fp16 scale vectors) go to the GPU in a single
+ * non-blocking transfer per module, with no dense reconstruction. "BitDelta Guide",
+ * "3. Dynamic Model Hot-Swapping and Multi-Tenant Batching": deltas are pre-cached in GPU
+ * memory or streamed from host CPU memory.
+ *
+ * A module is one projection of one layer. Every tenant is kept in host memory as one
+ * packed RECORD per module: the TILED sign words (bd_prepared_signs_bytes bytes), then its
+ * scales in the TILED layout (bd_prepared_scales_bytes bytes), i.e. the two outputs of
+ * bd_prepare_tenant placed back to back. The GPU holds n_slots tenant slots; the cache maps
+ * the tenants of each batch onto slots (least recently used slot evicted first) and loads
+ * a missing tenant with one cudaMemcpyAsync per module. The caller allocates every buffer
+ * (a device pool and pinned host staging); the cache object itself is host memory that
+ * bd_cache_create allocates and bd_cache_destroy frees. Not thread-safe: one host thread
+ * per cache. */
+typedef struct {
+  int64_t d_out, d_in;     /* the module's shape: d_out >= 1, d_in >= 32, d_in % 32 == 0    */
+  int32_t min_group_size;  /* smallest GROUP size a record may use (power of two >= 32 that
+                              divides d_in), or 0 when no record uses GROUP scales          */
+  int32_t reserved;        /* 0 */
+} bd_cache_module;
+
+typedef struct bd_cache bd_cache;  /* opaque */
+
+/* Bytes of one packed record (0 for an invalid shape, mode, group size or dtype). */
+size_t bd_cache_record_bytes(int64_t d_out, int64_t d_in, int32_t mode, int32_t group_size,
+                             int32_t scale_dtype);
+
+/* bd_prepare_record_host — host-side packing of one module of one tenant: sign words
+ * uint32[d_out][d_in/32] (as bd_compress writes them) and scales (BD_F16 / BD_F32, plain
+ * layout) into a packed record of bd_cache_record_bytes bytes at `record` (host memory).
+ * The bytes are those bd_prepare_tenant writes on the device. Pure host code, no CUDA.
+ * BD_ERR_WORKSPACE when record_bytes is too small. */
+bd_status bd_prepare_record_host(const uint32_t* signs, const void* scales, int32_t scale_dtype,
+                                 int32_t mode, int32_t group_size, int64_t d_out, int64_t d_in,
+                                 void* record, size_t record_bytes);
+
+/* Device pool bytes for n_slots slots of these modules (tables first, then the slots);
+ * pinned host staging bytes (two copies of the tables). 0 for invalid arguments. */
+size_t bd_cache_pool_bytes(const bd_cache_module* modules, int32_t n_modules, int32_t n_slots,
+                           int32_t scale_dtype);
+size_t bd_cache_staging_bytes(int32_t n_modules, int32_t n_slots);
+
+/* bd_cache_create — a cache for n_host_tenants tenants (ids 0 .. n_host_tenants-1) over
+ * n_modules modules, every tenant's scales of dtype scale_dtype.
+ *   pool    : device, >= bd_cache_pool_bytes, 256-byte aligned; owned by the caller and
+ *             written only by the cache's copies.
+ *   staging : host, pinned (cudaHostAlloc / pin_memory), >= bd_cache_staging_bytes,
+ *             16-byte aligned.
+ * Makes no CUDA call (events are created on the first bd_cache_prefetch).
+ * Errors: BD_ERR_NULL, BD_ERR_SHAPE, BD_ERR_DTYPE, BD_ERR_ALIGN, BD_ERR_WORKSPACE. */
+bd_status bd_cache_create(const bd_cache_module* modules, int32_t n_modules, int32_t scale_dtype,
+                          int32_t n_host_tenants, int32_t n_slots, void* pool, size_t pool_bytes,
+                          void* staging, size_t staging_bytes, bd_cache** out);
+/* Waits for the cache's copies in flight, then frees the host object. */
+bd_status bd_cache_destroy(bd_cache* cache);
+
+/* bd_cache_register — the packed record of (tenant, module) in host memory, with its scale
+ * mode and group size. The memory must stay valid and unchanged while the cache exists;
+ * pinned memory makes the copies asynchronous. A tenant that is resident on the GPU cannot
+ * be re-registered (BD_ERR_CONFIG). */
+bd_status bd_cache_register(bd_cache* cache, int32_t tenant, int32_t module, const void* record_host,
+                            int32_t mode, int32_t group_size);
+
+/* The device table of `module`: bd_cache_slots() bd_tenant records, one per slot, to pass
+ * to bd_apply_multi as `tenants` (n_tenants = bd_cache_slots()) with the slot ids from
+ * bd_cache_prefetch as `tenant_ids`. NULL for a bad module. */
+const bd_tenant* bd_cache_table(const bd_cache* cache, int32_t module);
+int32_t bd_cache_slots(const bd_cache* cache);
+
+/* bd_cache_assign — host part of a prefetch, no CUDA call: maps the batch's tenant ids
+ * (host int32[batch], -1 = base only) onto slots. Resident tenants are hits; every other
+ * distinct tenant takes the least recently used slot not held by an unreleased batch
+ * (empty slots first, then the lowest slot index among equals) and is listed in
+ * loads[2k] = tenant, loads[2k+1] = slot (host, room for 2 * n_slots ints, may be NULL).
+ * Writes slot_ids[t] (host int32[batch]; -1 for -1) and a ticket for the batch, which
+ * holds its slots until bd_cache_release. At most 4 batches may be held at once. The
+ * loads are left to the caller (bd_cache_prefetch is assign + loads).
+ * Errors (nothing changed): BD_ERR_TENANT_RANGE (an id outside [-1, n_host_tenants)),
+ * BD_ERR_TENANT_RECORD (a tenant without a record for every module), BD_ERR_CONFIG (not
+ * enough free slots for the batch's missing tenants, or 4 batches held). */
+bd_status bd_cache_assign(bd_cache* cache, const int32_t* tenant_ids, int64_t batch, int32_t* slot_ids,
+                          int32_t* loads, int32_t* n_loads, int64_t* ticket);
+
+/* bd_cache_prefetch — bd_cache_assign, then the loads on copy_stream: for each missing
+ * tenant, after the last batch that read its slot has been released, one cudaMemcpyAsync
+ * per module from its host record into the slot; then one copy of the changed tables.
+ * The batch's ticket records when its copies are done. Issue it for the next batch while
+ * the current one computes. A CUDA error returns BD_ERR_CUDA; the batch's new slots are
+ * then marked empty and its ticket is closed. */
+bd_status bd_cache_prefetch(bd_cache* cache, const int32_t* tenant_ids, int64_t batch, int32_t* slot_ids,
+                            int32_t* n_loads, int64_t* ticket, void* copy_stream);
+/* Makes compute_stream wait for the ticket's copies (no host wait). acquire and release
+ * of a cache's batches go to one compute stream. BD_ERR_CONFIG for a ticket not held. */
+bd_status bd_cache_acquire(bd_cache* cache, int64_t ticket, void* compute_stream);
+/* Marks the end of the ticket's use on compute_stream (after its bd_apply_multi calls):
+ * its slots may be refilled once compute_stream has passed this point. */
+bd_status bd_cache_release(bd_cache* cache, int64_t ticket, void* compute_stream);
+
+/* slot_tenant (host int32[n_slots], may be NULL): the tenant in each slot (-1 empty);
+ * stats (host int64[4], may be NULL): hits, misses, bytes copied, copies issued. */
+bd_status bd_cache_resident(const bd_cache* cache, int32_t* slot_tenant, int64_t* stats);
+
 /* Bytes of workspace bd_apply_multi needs. */
 size_t bd_apply_workspace_size(int64_t d_out, int64_t d_in, int64_t batch, int32_t n_tenants);
 

@@ -17,4 +17,5 @@ from ._lib import (  # noqa: F401
     bd_compress, bd_compress_noalloc, bd_compress_workspace_size, bd_reconstruct, bd_apply_multi,
     bd_apply_workspace_size, bd_get_status, bd_launch_count, bd_profile_enable,
     bd_profile_collect, bd_selftest_wait_timeout, bd_tc_min_tokens,
+    bd_cache_module, bd_cache_record_bytes, bd_prepare_record_host, CacheTable, TenantCache,
 )

@@ -39,7 +39,10 @@ EXPORTS = (
     "bd_apply_multi", "bd_prepared_signs_bytes", "bd_prepared_scales_bytes", "bd_prepare_tenant",
     "bd_apply_workspace_size", "bd_get_status", "bd_status_string", "bd_launch_count",
     "bd_profile_enable", "bd_profile_collect", "bd_kernel_name", "bd_selftest_wait_timeout",
-    "bd_tc_min_tokens",
+    "bd_tc_min_tokens", "bd_cache_record_bytes", "bd_prepare_record_host", "bd_cache_pool_bytes",
+    "bd_cache_staging_bytes", "bd_cache_create", "bd_cache_destroy", "bd_cache_register",
+    "bd_cache_table", "bd_cache_slots", "bd_cache_assign", "bd_cache_prefetch", "bd_cache_acquire",
+    "bd_cache_release", "bd_cache_resident",
 )
 
 
@@ -50,6 +53,11 @@ class bd_compress_cfg(ctypes.Structure):
 class bd_tenant(ctypes.Structure):
     _fields_ = [("signs", c_void_p), ("scales", c_void_p), ("mode", c_int32),
                 ("group_size", c_int32), ("layout", c_int32), ("reserved", c_int32)]
+
+
+class bd_cache_module(ctypes.Structure):
+    _fields_ = [("d_out", c_int64), ("d_in", c_int64), ("min_group_size", c_int32),
+                ("reserved", c_int32)]
 
 
 class BitDeltaError(RuntimeError):
@@ -112,6 +120,38 @@ def lib():
     L.bd_selftest_wait_timeout.restype = c_int32
     L.bd_tc_min_tokens.argtypes = []
     L.bd_tc_min_tokens.restype = c_int32
+    L.bd_cache_record_bytes.argtypes = [c_int64, c_int64, c_int32, c_int32, c_int32]
+    L.bd_cache_record_bytes.restype = c_size_t
+    L.bd_prepare_record_host.argtypes = [c_void_p, c_void_p, c_int32, c_int32, c_int32, c_int64,
+                                         c_int64, c_void_p, c_size_t]
+    L.bd_prepare_record_host.restype = c_int32
+    L.bd_cache_pool_bytes.argtypes = [POINTER(bd_cache_module), c_int32, c_int32, c_int32]
+    L.bd_cache_pool_bytes.restype = c_size_t
+    L.bd_cache_staging_bytes.argtypes = [c_int32, c_int32]
+    L.bd_cache_staging_bytes.restype = c_size_t
+    L.bd_cache_create.argtypes = [POINTER(bd_cache_module), c_int32, c_int32, c_int32, c_int32,
+                                  c_void_p, c_size_t, c_void_p, c_size_t, POINTER(c_void_p)]
+    L.bd_cache_create.restype = c_int32
+    L.bd_cache_destroy.argtypes = [c_void_p]
+    L.bd_cache_destroy.restype = c_int32
+    L.bd_cache_register.argtypes = [c_void_p, c_int32, c_int32, c_void_p, c_int32, c_int32]
+    L.bd_cache_register.restype = c_int32
+    L.bd_cache_table.argtypes = [c_void_p, c_int32]
+    L.bd_cache_table.restype = c_void_p
+    L.bd_cache_slots.argtypes = [c_void_p]
+    L.bd_cache_slots.restype = c_int32
+    L.bd_cache_assign.argtypes = [c_void_p, c_void_p, c_int64, c_void_p, c_void_p,
+                                  POINTER(c_int32), POINTER(c_int64)]
+    L.bd_cache_assign.restype = c_int32
+    L.bd_cache_prefetch.argtypes = [c_void_p, c_void_p, c_int64, c_void_p, POINTER(c_int32),
+                                    POINTER(c_int64), c_void_p]
+    L.bd_cache_prefetch.restype = c_int32
+    L.bd_cache_acquire.argtypes = [c_void_p, c_int64, c_void_p]
+    L.bd_cache_acquire.restype = c_int32
+    L.bd_cache_release.argtypes = [c_void_p, c_int64, c_void_p]
+    L.bd_cache_release.restype = c_int32
+    L.bd_cache_resident.argtypes = [c_void_p, c_void_p, c_void_p]
+    L.bd_cache_resident.restype = c_int32
     _LIB = L
     return L
 
@@ -347,3 +387,150 @@ def bd_profile_collect():
         if la[i]:
             out[lib().bd_kernel_name(i).decode()] = (int(la[i]), float(ms[i]))
     return out
+
+
+# ----------------------------------------------------------------------------------
+# host-resident tenant cache
+# ----------------------------------------------------------------------------------
+def bd_cache_record_bytes(d_out, d_in, mode, group_size, scale_dtype=BD_F16) -> int:
+    return int(lib().bd_cache_record_bytes(int(d_out), int(d_in), int(mode), int(group_size),
+                                           int(scale_dtype)))
+
+
+def bd_prepare_record_host(signs, scales, mode, group_size, d_out, d_in, out=None, pin=False):
+    """Wrap ``bd_prepare_record_host``. signs: host int32/uint32 array [d_out, d_in//32];
+    scales: host fp16/fp32 array (plain layout). Returns a host uint8 torch tensor holding
+    the packed record (pinned if ``pin``)."""
+    import numpy as np
+    torch = _torch()
+    sg = np.ascontiguousarray(np.asarray(signs).view(np.uint32))
+    sc = np.ascontiguousarray(np.asarray(scales))
+    sdt = {np.dtype(np.float16): BD_F16, np.dtype(np.float32): BD_F32}.get(sc.dtype)
+    if sdt is None:
+        raise TypeError(f"unsupported scale dtype {sc.dtype}")
+    n = bd_cache_record_bytes(d_out, d_in, mode, group_size, sdt)
+    if n == 0:
+        raise BitDeltaError(BD_ERR_CONFIG, "bd_prepare_record_host")
+    if out is None:
+        out = torch.empty(n, dtype=torch.uint8)
+        if pin:
+            out = out.pin_memory()
+    rc = lib().bd_prepare_record_host(sg.ctypes.data, sc.ctypes.data, sdt, int(mode), int(group_size),
+                                      int(d_out), int(d_in), c_void_p(out.data_ptr()), out.numel())
+    check(rc, "bd_prepare_record_host")
+    return out
+
+
+class CacheTable:
+    """The device table of one module of a TenantCache, accepted by bd_apply_multi."""
+
+    def __init__(self, ptr, n, scale_dtype):
+        self._p, self.n, self.scale_dtype = ptr, n, scale_dtype
+
+    def ptr(self):
+        return c_void_p(self._p)
+
+
+class TenantCache:
+    """Wrap ``bd_cache_*``: modules = [(d_out, d_in, min_group_size)]. The device pool and
+    the pinned staging are torch allocations kept by this object. ``device=None`` builds
+    the cache over host buffers; only ``assign`` (no CUDA) may be used then."""
+
+    def __init__(self, modules, n_host_tenants, n_slots, scale_dtype=BD_F16, device="cuda"):
+        torch = _torch()
+        L = lib()
+        self.n_modules = len(modules)
+        arr = (bd_cache_module * self.n_modules)()
+        for i, (d_out, d_in, g) in enumerate(modules):
+            arr[i] = bd_cache_module(int(d_out), int(d_in), int(g), 0)
+        self._mods = arr
+        self.scale_dtype = scale_dtype
+        pb = int(L.bd_cache_pool_bytes(arr, self.n_modules, int(n_slots), int(scale_dtype)))
+        sb = int(L.bd_cache_staging_bytes(self.n_modules, int(n_slots)))
+        if pb == 0 or sb == 0:
+            raise BitDeltaError(BD_ERR_SHAPE, "bd_cache_pool_bytes")
+        if device is None:
+            self.pool = torch.empty(pb + 256, dtype=torch.uint8)
+            off = (-self.pool.data_ptr()) % 256
+            self.pool = self.pool[off:off + pb]
+            self.staging = torch.empty(sb, dtype=torch.uint8)
+        else:
+            self.pool = torch.empty(pb, dtype=torch.uint8, device=device)
+            self.staging = torch.empty(sb, dtype=torch.uint8).pin_memory()
+        h = c_void_p()
+        rc = L.bd_cache_create(arr, self.n_modules, int(scale_dtype), int(n_host_tenants), int(n_slots),
+                               c_void_p(self.pool.data_ptr()), pb, c_void_p(self.staging.data_ptr()), sb,
+                               ctypes.byref(h))
+        check(rc, "bd_cache_create")
+        self._h = h
+        self._host_only = device is None
+        self.n_slots = int(n_slots)
+        self.n_host = int(n_host_tenants)
+        self._records = {}
+
+    def register(self, tenant, module, record, mode, group_size):
+        rc = lib().bd_cache_register(self._h, int(tenant), int(module), c_void_p(record.data_ptr()),
+                                     int(mode), int(group_size))
+        check(rc, "bd_cache_register")
+        self._records[(int(tenant), int(module))] = record
+
+    def table(self, module) -> CacheTable:
+        p = lib().bd_cache_table(self._h, int(module))
+        if not p:
+            raise BitDeltaError(BD_ERR_SHAPE, "bd_cache_table")
+        return CacheTable(p, self.n_slots, self.scale_dtype)
+
+    def assign(self, tenant_ids):
+        """Host-only slot assignment: (slot_ids int32 array, [(tenant, slot)] loads, ticket)."""
+        import numpy as np
+        ids = np.ascontiguousarray(np.asarray(tenant_ids, dtype=np.int32))
+        slots = np.empty_like(ids)
+        loads = np.empty(2 * self.n_slots, dtype=np.int32)
+        n = c_int32(0)
+        t = c_int64(-1)
+        rc = lib().bd_cache_assign(self._h, ids.ctypes.data, ids.size, slots.ctypes.data, loads.ctypes.data,
+                                   ctypes.byref(n), ctypes.byref(t))
+        check(rc, "bd_cache_assign")
+        return slots, [(int(loads[2 * k]), int(loads[2 * k + 1])) for k in range(n.value)], int(t.value)
+
+    def prefetch(self, tenant_ids, stream=None):
+        """Assign + loads on ``stream``: (slot_ids int32 array, number of loads, ticket)."""
+        import numpy as np
+        ids = np.ascontiguousarray(np.asarray(tenant_ids, dtype=np.int32))
+        slots = np.empty_like(ids)
+        n = c_int32(0)
+        t = c_int64(-1)
+        rc = lib().bd_cache_prefetch(self._h, ids.ctypes.data, ids.size, slots.ctypes.data, ctypes.byref(n),
+                                     ctypes.byref(t), _stream(stream))
+        check(rc, "bd_cache_prefetch")
+        return slots, int(n.value), int(t.value)
+
+    def _s(self, stream):
+        # a host-only cache never issued a copy: its acquire / release touch no stream
+        return c_void_p(None) if self._host_only else _stream(stream)
+
+    def acquire(self, ticket, stream=None):
+        check(lib().bd_cache_acquire(self._h, int(ticket), self._s(stream)), "bd_cache_acquire")
+
+    def release(self, ticket, stream=None):
+        check(lib().bd_cache_release(self._h, int(ticket), self._s(stream)), "bd_cache_release")
+
+    def resident(self):
+        """(tenant per slot, {hits, misses, bytes, copies})."""
+        import numpy as np
+        st = np.zeros(self.n_slots, dtype=np.int32)
+        stats = np.zeros(4, dtype=np.int64)
+        check(lib().bd_cache_resident(self._h, st.ctypes.data, stats.ctypes.data), "bd_cache_resident")
+        return st.tolist(), dict(zip(("hits", "misses", "bytes", "copies"), stats.tolist()))
+
+    def close(self):
+        if getattr(self, "_h", None):
+            rc = lib().bd_cache_destroy(self._h)
+            self._h = None
+            check(rc, "bd_cache_destroy")
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
