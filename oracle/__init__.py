@@ -18,6 +18,9 @@ source pages state it:
   "Systems Mechanics: 1. Decoupled Forward Pass".
 * "Per-Axis Weight Deltas for Frequent Model Updates", "Key Contributions" item 1
   (row / column scale vectors, mask packed along the input axis).
+* ``oracle.fp8``: an e4m3 base with per-row scales under the same delta path ("BitDelta
+  Guide", "3. Quantized Base Model Compatibility"; "Per-Axis Weight Deltas", Future
+  Directions, FP8 co-design).
 
 Every function here is pinned by ``tests/test_oracle.py`` against the pages' worked
 examples, closed forms, invariants or brute force; none is "parity unpinned".
@@ -41,4 +44,12 @@ from .bitdelta import (  # noqa: F401
     reconstruct,
     apply_multi,
     apply_rows,
+)
+from .fp8 import (  # noqa: F401
+    E4M3_MAX,
+    e4m3_value,
+    e4m3_round,
+    quantize_base,
+    dequantize_base,
+    apply_multi_fp8,
 )
