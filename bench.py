@@ -667,11 +667,12 @@ def _time_calls(run, iters, warmup, stream):
     return ms, {k: {"launches": v[0] // iters, "us_per_run": v[1] / iters * 1e3} for k, v in prof.items()}
 
 
-def bench_decode(args, log, peaks):
-    """Decode GEMV: the up_proj shape 14336 x 4096 with a bf16 base, 64 resident tenants
-    (sign words + fp16 group-128 scales, tiled serving layout), 64 tokens, one per tenant
-    (a seeded permutation), x ~ N(0, 1) bf16. The ~646 MB read per call is far larger than
-    L2, so no flush is needed between calls."""
+def bench_decode(args, log, peaks, fp8=False):
+    """Decode GEMV: the up_proj shape 14336 x 4096 with a bf16 base (or, with fp8, the same
+    base quantized to e4m3 with per-row scales), 64 resident tenants (sign words + fp16
+    group-128 scales, tiled serving layout), 64 tokens, one per tenant (a seeded
+    permutation), x ~ N(0, 1) bf16. The ~646 MB (fp8: ~587 MB) read per call is far larger
+    than L2, so no flush is needed between calls."""
     import torch
     import tenant_serving_b200 as bd
     d_out, d_in, T, B = 14336, 4096, 64, 64
@@ -690,15 +691,29 @@ def bench_decode(args, log, peaks):
     ids = torch.from_numpy(np.random.default_rng(2000).permutation(T).astype(np.int32)).cuda()
     x = (torch.randn((B, d_in), generator=g, device="cuda")).to(torch.bfloat16)
     y = torch.empty((B, d_out), dtype=torch.bfloat16, device="cuda")
-    ws = torch.empty(bd.bd_apply_workspace_size(d_out, d_in, B, T), dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
-    ms, kern = _time_calls(lambda: bd.bd_apply_multi(wb, table, ids, x, y=y, workspace=ws), 20, 3, stream)
-    alg = d_out * d_in * 2 + T * (d_out * d_in // 8 + d_out * (d_in // GROUP) * 2) + B * (d_in + d_out) * 2
+    if fp8:
+        codes, wsc = bd.bd_quantize_base_fp8(wb)
+        del wb
+        ws = torch.empty(bd.bd_apply_fp8_workspace_size(d_out, d_in, B, T), dtype=torch.uint8, device="cuda")
+        run = lambda: bd.bd_apply_multi_fp8(codes, wsc, table, ids, x, y=y, workspace=ws)  # noqa: E731
+        base_bytes = d_out * d_in + d_out * 4
+    else:
+        ws = torch.empty(bd.bd_apply_workspace_size(d_out, d_in, B, T), dtype=torch.uint8, device="cuda")
+        run = lambda: bd.bd_apply_multi(wb, table, ids, x, y=y, workspace=ws)  # noqa: E731
+        base_bytes = d_out * d_in * 2
+    ms, kern = _time_calls(run, 20, 3, stream)
+    alg = base_bytes + T * (d_out * d_in // 8 + d_out * (d_in // GROUP) * 2) + B * (d_in + d_out) * 2
     del recs, table
-    return {"workload": "decode: up_proj 14336x4096 bf16 base, 64 tenants (group-128 fp16 scales), "
-                        "64 tokens one per tenant",
-            "us_per_call": ms * 1e3, "tokens_per_s": B / (ms / 1e3), "bytes_per_call": alg,
-            "gbs": alg / (ms / 1e3) / 1e9, "frac": alg / (ms / 1e3) / 1e9 / peaks[0], "kernels": kern}
+    torch.cuda.empty_cache()
+    base_k = "base_fp8" if fp8 else "base_tc"
+    out = {"workload": "decode: up_proj 14336x4096 %s base, 64 tenants (group-128 fp16 scales), "
+                       "64 tokens one per tenant" % ("e4m3 (per-row fp32 scales)" if fp8 else "bf16"),
+           "us_per_call": ms * 1e3, "tokens_per_s": B / (ms / 1e3), "bytes_per_call": alg,
+           "gbs": alg / (ms / 1e3) / 1e9, "frac": alg / (ms / 1e3) / 1e9 / peaks[0], "kernels": kern}
+    if base_k in kern and kern[base_k]["us_per_run"] > 0:
+        out["base_gbs"] = base_bytes / (kern[base_k]["us_per_run"] / 1e6) / 1e9
+    return out
 
 
 def bench_mixed(args, log, peaks):
@@ -859,10 +874,11 @@ def main():
         barrier(pg)
     res = bench_serving(args, rank, pg, log, peaks)
     cpu = None
-    dec = mix = None
+    dec = dec8 = mix = None
     cold = None
     if rank == 0 and world == 1 and not args.no_extra:
         dec = bench_decode(args, log, peaks)
+        dec8 = bench_decode(args, log, peaks, fp8=True)
         mix = bench_mixed(args, log, peaks)
         cold = bench_cold_start(args, log, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -880,7 +896,7 @@ def main():
             "ms_per_step_profiled": res["ms_per_step_profiled"],
             "distinct_tenants_mean": res["distinct_tenants_mean"],
             "kernels": res["kernels"], "kernel_rates": res["kernel_rates"], "compress": comp,
-            "decode": dec, "mixed": mix, "cold_start": cold,
+            "decode": dec, "decode_fp8_base": dec8, "mixed": mix, "cold_start": cold,
         }
         print(json.dumps(line))
     if pg is not None:

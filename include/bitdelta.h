@@ -355,6 +355,42 @@ bd_status bd_apply_multi(const void* w_base, int32_t w_dtype, int64_t d_out, int
                          int32_t y_dtype, void* workspace, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------- */
+/* e4m3 base weights                                                                   */
+/* ---------------------------------------------------------------------------------- */
+/* "BitDelta Guide", "3. Quantized Base Model Compatibility (BitDelta + GPTQ / QuIP#)":
+ * the 1-bit delta is applied on top of quantized base weights; "Per-Axis Weight Deltas",
+ * Future Directions: FP8 co-design. The base is held as OCP E4M3 codes (1 sign, 4
+ * exponent bits with bias 7, 3 mantissa bits; largest finite 448; S.1111.111 NaN) with one
+ * fp32 scale per output row: W_hat[o][i] = scales[o] * e4m3(codes[o][i]).
+ *
+ * bd_quantize_base_fp8 — scales[o] = max_i |w[o][i]| / 448 and codes[o][i] = e4m3 of
+ * w[o][i] / scales[o], both quotients IEEE fp32 divisions, the rounding to nearest even
+ * with saturation at +-448 and the sign kept; a row of zeros gets scale 0 and codes 0.
+ *   w      : device [d_out][d_in], w_dtype BD_BF16 or BD_F32, 16-byte aligned.
+ *   codes  : device uint8 [d_out][d_in], 16-byte aligned.  scales : device fp32 [d_out].
+ * d_in % 32 == 0. Asynchronous on `stream`. */
+bd_status bd_quantize_base_fp8(const void* w, int32_t w_dtype, int64_t d_out, int64_t d_in,
+                               uint8_t* codes, float* scales, void* stream);
+
+/* Bytes of workspace bd_apply_multi_fp8 needs. */
+size_t bd_apply_fp8_workspace_size(int64_t d_out, int64_t d_in, int64_t batch, int32_t n_tenants);
+
+/* bd_apply_multi_fp8 — bd_apply_multi with an e4m3 base:
+ *     y[t] = W_hat x[t] + Delta_hat_{u(t)} x[t].
+ * Same tenants, ids, output and status rules as bd_apply_multi; x is bf16 [batch][d_in].
+ * The base product runs on the tensor cores in e4m3 x e4m3 with fp32 accumulation: each
+ * x[t] is written as 2^e_t (hi + lo), hi and lo e4m3 and 2^e_t the power of two that puts
+ * max|x[t]| in [128, 256). This is exact for bf16 values down to about max|x[t]| / 2^16;
+ * smaller ones carry an error of at most 2^-10 * 2^e_t.
+ *   w_codes  : device uint8 [d_out][d_in] (bd_quantize_base_fp8), 16-byte aligned.
+ *   w_scales : device fp32 [d_out], 4-byte aligned.
+ *   workspace: bd_apply_fp8_workspace_size() bytes. */
+bd_status bd_apply_multi_fp8(const uint8_t* w_codes, const float* w_scales, int64_t d_out, int64_t d_in,
+                             const bd_tenant* tenants, int32_t n_tenants, int32_t scale_dtype,
+                             const int32_t* tenant_ids, const void* x, int64_t batch, void* y,
+                             int32_t y_dtype, void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------- */
 /* status, diagnostics                                                                 */
 /* ---------------------------------------------------------------------------------- */
 /* Copies the device status word of a workspace (compress or apply) to *flags (host)

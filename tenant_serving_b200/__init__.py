@@ -18,4 +18,5 @@ from ._lib import (  # noqa: F401
     bd_apply_workspace_size, bd_get_status, bd_launch_count, bd_profile_enable,
     bd_profile_collect, bd_selftest_wait_timeout, bd_tc_min_tokens,
     bd_cache_module, bd_cache_record_bytes, bd_prepare_record_host, CacheTable, TenantCache,
+    bd_quantize_base_fp8, bd_apply_fp8_workspace_size, bd_apply_multi_fp8,
 )

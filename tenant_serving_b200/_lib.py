@@ -42,7 +42,8 @@ EXPORTS = (
     "bd_tc_min_tokens", "bd_cache_record_bytes", "bd_prepare_record_host", "bd_cache_pool_bytes",
     "bd_cache_staging_bytes", "bd_cache_create", "bd_cache_destroy", "bd_cache_register",
     "bd_cache_table", "bd_cache_slots", "bd_cache_assign", "bd_cache_prefetch", "bd_cache_acquire",
-    "bd_cache_release", "bd_cache_resident",
+    "bd_cache_release", "bd_cache_resident", "bd_quantize_base_fp8", "bd_apply_fp8_workspace_size",
+    "bd_apply_multi_fp8",
 )
 
 
@@ -152,6 +153,14 @@ def lib():
     L.bd_cache_release.restype = c_int32
     L.bd_cache_resident.argtypes = [c_void_p, c_void_p, c_void_p]
     L.bd_cache_resident.restype = c_int32
+    L.bd_quantize_base_fp8.argtypes = [c_void_p, c_int32, c_int64, c_int64, c_void_p, c_void_p, c_void_p]
+    L.bd_quantize_base_fp8.restype = c_int32
+    L.bd_apply_fp8_workspace_size.argtypes = [c_int64, c_int64, c_int64, c_int32]
+    L.bd_apply_fp8_workspace_size.restype = c_size_t
+    L.bd_apply_multi_fp8.argtypes = [c_void_p, c_void_p, c_int64, c_int64, c_void_p, c_int32, c_int32,
+                                     c_void_p, c_void_p, c_int64, c_void_p, c_int32, c_void_p, c_size_t,
+                                     c_void_p]
+    L.bd_apply_multi_fp8.restype = c_int32
     _LIB = L
     return L
 
@@ -345,6 +354,44 @@ def bd_apply_multi(w_base, table: TenantTable, tenant_ids, x, y=None, y_dtype=No
                               table.scale_dtype, _ptr(tenant_ids), _ptr(x), batch, _ptr(y),
                               dtype_code(y), _ptr(workspace), workspace.numel(), _stream(stream))
     check(rc, "bd_apply_multi")
+    return y, workspace
+
+
+def bd_quantize_base_fp8(w, codes=None, scales=None, stream=None):
+    """Wrap ``bd_quantize_base_fp8``: (codes uint8 [d_out, d_in], scales fp32 [d_out])."""
+    torch = _torch()
+    _require_cuda(w)
+    d_out, d_in = w.shape
+    if codes is None:
+        codes = torch.empty((d_out, d_in), dtype=torch.uint8, device=w.device)
+    if scales is None:
+        scales = torch.empty(d_out, dtype=torch.float32, device=w.device)
+    rc = lib().bd_quantize_base_fp8(_ptr(w), dtype_code(w), d_out, d_in, _ptr(codes), _ptr(scales), _stream(stream))
+    check(rc, "bd_quantize_base_fp8")
+    return codes, scales
+
+
+def bd_apply_fp8_workspace_size(d_out, d_in, batch, n_tenants) -> int:
+    return int(lib().bd_apply_fp8_workspace_size(int(d_out), int(d_in), int(batch), int(n_tenants)))
+
+
+def bd_apply_multi_fp8(w_codes, w_scales, table, tenant_ids, x, y=None, y_dtype=None, workspace=None,
+                       stream=None):
+    """Wrap ``bd_apply_multi_fp8``: y[t] = W_hat x[t] + Delta_hat_{ids[t]} x[t], W_hat the
+    e4m3 base with per-row scales."""
+    torch = _torch()
+    _require_cuda(w_codes, w_scales, tenant_ids, x)
+    d_out, d_in = w_codes.shape
+    batch = x.shape[0]
+    if y is None:
+        y = torch.empty((batch, d_out), dtype=y_dtype or torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(max(bd_apply_fp8_workspace_size(d_out, d_in, batch, table.n), 16),
+                                dtype=torch.uint8, device=x.device)
+    rc = lib().bd_apply_multi_fp8(_ptr(w_codes), _ptr(w_scales), d_out, d_in, table.ptr(), table.n,
+                                  table.scale_dtype, _ptr(tenant_ids), _ptr(x), batch, _ptr(y), dtype_code(y),
+                                  _ptr(workspace), workspace.numel(), _stream(stream))
+    check(rc, "bd_apply_multi_fp8")
     return y, workspace
 
 

@@ -15,7 +15,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 OUT = os.path.join(HERE, "libbitdelta.so")
 SOURCES = ["bd_abi.cu", "bd_compress.cu", "bd_reconstruct.cu", "bd_apply.cu", "bd_base_tc.cu",
-           "bd_prepare.cu", "bd_delta_tc.cu", "bd_delta_lut.cu", "bd_cache.cu"]
+           "bd_prepare.cu", "bd_delta_tc.cu", "bd_delta_lut.cu", "bd_cache.cu",
+           "bd_base_fp8.cu"]
 HEADERS = ["bd_internal.cuh", "bd_tc.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

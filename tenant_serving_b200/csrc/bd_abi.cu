@@ -13,6 +13,7 @@ static const char* const kKernelNames[K_KIND_COUNT] = {
     "scale_final",       "reconstruct",  "tenant_bucket",  "base_gemv",
     "base_tc",           "delta_lut",    "prepare",
     "tc_gather",         "delta_tc",     "selftest_wait",
+    "quant_fp8",         "x_limbs",      "base_fp8",
 };
 
 const char* kernel_name(int32_t kind) {

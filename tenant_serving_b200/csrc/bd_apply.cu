@@ -23,15 +23,6 @@
 
 namespace bd {
 
-struct TcPlan {
-  int n_tile, tiles_n, tiles_m, kblocks, kb_per_split, ksplit, stages;
-  size_t smem;
-};
-TcPlan plan_base_tc(int64_t d_out, int64_t d_in, int64_t batch);
-bd_status launch_base_tc(const TcPlan& p, const void* w_base, const void* x, int64_t d_out,
-                         int64_t d_in, int64_t batch, float* y_part, uint32_t* status,
-                         cudaStream_t s);
-
 constexpr int kMaxTenants = 16384;
 constexpr int kMaxBatch = 65536;
 
@@ -281,13 +272,15 @@ namespace {
 struct ApplyLayout {
   int max_groups, max_tc;
   TcPlan tc;
+  Fp8Plan f8;
   int ksplit;
   int64_t xg_rows;
-  size_t off_seg, off_tcrec, off_part, off_xg, off_xinv, total;
+  size_t off_seg, off_tcrec, off_part, off_xg, off_xinv, off_x8, off_xmul, total;
 };
 
+// tc: the base product on the tensor cores (bf16 weights, or e4m3 ones when fp8)
 ApplyLayout layout_apply(int64_t d_out, int64_t d_in, int64_t batch, int32_t n_tenants, bool tc,
-                         bool tc_delta) {
+                         bool tc_delta, bool fp8 = false) {
   ApplyLayout L;
   L.max_groups = max_groups_for(batch, n_tenants);
   if (L.max_groups < 1) L.max_groups = 1;
@@ -301,7 +294,10 @@ ApplyLayout layout_apply(int64_t d_out, int64_t d_in, int64_t batch, int32_t n_t
   }
   L.xg_rows = tc_delta ? batch + 15 * (int64_t)L.max_tc : 0;
   L.ksplit = 1;
-  if (tc) {
+  if (fp8) {
+    L.f8 = plan_base_fp8(d_out, d_in, batch);
+    L.ksplit = L.f8.ksplit;
+  } else if (tc) {
     L.tc = plan_base_tc(d_out, d_in, batch);
     L.ksplit = L.tc.ksplit;
   }
@@ -316,6 +312,10 @@ ApplyLayout layout_apply(int64_t d_out, int64_t d_in, int64_t batch, int32_t n_t
   off = align_up(off + (size_t)L.xg_rows * d_in * 2, 256);
   L.off_xinv = off;
   off = align_up(off + (size_t)L.xg_rows * sizeof(float), 256);
+  L.off_x8 = off;
+  off = align_up(off + (fp8 ? L.f8.x8_bytes : 0), 256);
+  L.off_xmul = off;
+  off = align_up(off + (fp8 ? (size_t)L.f8.xmul_count * sizeof(float) : 0), 256);
   L.total = off;
   return L;
 }
@@ -329,10 +329,18 @@ size_t apply_workspace_size(int64_t d_out, int64_t d_in, int64_t batch, int32_t 
   return a > b ? a : b;
 }
 
+size_t apply_fp8_workspace_size(int64_t d_out, int64_t d_in, int64_t batch, int32_t n_tenants) {
+  if (d_out < 1 || d_in < 32 || batch < 0 || n_tenants < 0) return 0;
+  return layout_apply(d_out, d_in, batch, n_tenants, true, (d_in % 64) == 0, true).total;
+}
+
+// w_scales != nullptr: w_base holds e4m3 codes with per-row fp32 scales w_scales (x bf16)
 bd_status apply_impl(const void* w_base, int32_t w_dtype, int64_t d_out, int64_t d_in,
                      const bd_tenant* tenants, int32_t n_tenants, int32_t scale_dtype,
                      const int32_t* tenant_ids, const void* x, int64_t batch, void* y,
-                     int32_t y_dtype, void* workspace, size_t ws_bytes, cudaStream_t s) {
+                     int32_t y_dtype, void* workspace, size_t ws_bytes, cudaStream_t s,
+                     const float* w_scales = nullptr) {
+  const bool fp8 = w_scales != nullptr;
   if (w_dtype != BD_BF16 && w_dtype != BD_F32) return BD_ERR_DTYPE;
   if (scale_dtype != BD_F16 && scale_dtype != BD_F32) return BD_ERR_DTYPE;
   if (y_dtype != BD_BF16 && y_dtype != BD_F32) return BD_ERR_DTYPE;
@@ -342,12 +350,13 @@ bd_status apply_impl(const void* w_base, int32_t w_dtype, int64_t d_out, int64_t
   if (!w_base || !x || !y || !tenant_ids) return BD_ERR_NULL;
   if (n_tenants > 0 && !tenants) return BD_ERR_NULL;
   if (!aligned16(w_base) || !aligned16(x) || !aligned16(y) || !aligned16(tenant_ids) ||
-      (tenants && (reinterpret_cast<uintptr_t>(tenants) & 7u)))
+      (tenants && (reinterpret_cast<uintptr_t>(tenants) & 7u)) ||
+      (fp8 && (reinterpret_cast<uintptr_t>(w_scales) & 3u)))
     return BD_ERR_ALIGN;
-  const bool tc = w_dtype == BD_BF16;
+  const bool tc = w_dtype == BD_BF16;  // with an e4m3 base, w_dtype is the activations' bf16
   // the tensor-core delta path needs bf16 activations, fp16 scales and 64-column stages
   const bool tc_delta = tc && scale_dtype == BD_F16 && (d_in % 64) == 0;
-  ApplyLayout L = layout_apply(d_out, d_in, batch, n_tenants, tc, tc_delta);
+  ApplyLayout L = layout_apply(d_out, d_in, batch, n_tenants, tc, tc_delta, fp8);
   if (!workspace || ws_bytes < L.total) return BD_ERR_WORKSPACE;
   if (!aligned16(workspace)) return BD_ERR_ALIGN;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -368,7 +377,11 @@ bd_status apply_impl(const void* w_base, int32_t w_dtype, int64_t d_out, int64_t
   BD_LAUNCH_CHECK();
 
   // 2. base product (fp32 partial sums)
-  if (tc) {
+  if (fp8) {
+    bd_status st = launch_base_fp8(L.f8, static_cast<const uint8_t*>(w_base), w_scales, x, d_out, d_in, batch,
+                                   ws + L.off_x8, reinterpret_cast<float*>(ws + L.off_xmul), y_part, status, s);
+    if (st != BD_OK) return st;
+  } else if (tc) {
     bd_status st = launch_base_tc(L.tc, w_base, x, d_out, d_in, batch, y_part, status, s);
     if (st != BD_OK) return st;
   } else {
@@ -402,6 +415,21 @@ extern "C" int32_t bd_tc_min_tokens(void) { return bd::kTcMinTokens; }
 extern "C" size_t bd_apply_workspace_size(int64_t d_out, int64_t d_in, int64_t batch,
                                           int32_t n_tenants) {
   return bd::apply_workspace_size(d_out, d_in, batch, n_tenants);
+}
+
+extern "C" size_t bd_apply_fp8_workspace_size(int64_t d_out, int64_t d_in, int64_t batch,
+                                              int32_t n_tenants) {
+  return bd::apply_fp8_workspace_size(d_out, d_in, batch, n_tenants);
+}
+
+extern "C" bd_status bd_apply_multi_fp8(const uint8_t* w_codes, const float* w_scales, int64_t d_out,
+                                        int64_t d_in, const bd_tenant* tenants, int32_t n_tenants,
+                                        int32_t scale_dtype, const int32_t* tenant_ids, const void* x,
+                                        int64_t batch, void* y, int32_t y_dtype, void* workspace,
+                                        size_t ws_bytes, void* stream) {
+  if (batch > 0 && !w_scales) return BD_ERR_NULL;  // (batch 0: shapes checked, nothing launched)
+  return bd::apply_impl(w_codes, BD_BF16, d_out, d_in, tenants, n_tenants, scale_dtype, tenant_ids, x, batch, y,
+                        y_dtype, workspace, ws_bytes, static_cast<cudaStream_t>(stream), w_scales);
 }
 
 extern "C" bd_status bd_apply_multi(const void* w_base, int32_t w_dtype, int64_t d_out,

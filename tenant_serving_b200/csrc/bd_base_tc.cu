@@ -156,31 +156,10 @@ __global__ void __launch_bounds__(128, 1) k_base_tc(const __grid_constant__ CUte
 // ------------------------------------------------------------------------------------
 // host side
 // ------------------------------------------------------------------------------------
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn get_encoder() {
-  static EncodeTiledFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-    else
-      (void)cudaGetLastError();
-  }
-  return fn;
-}
-
 // bf16 row-major [rows][cols] tensor, box [box_rows][64 cols], 128-byte swizzle
 static bool encode_bf16_2d(CUtensorMap* m, const void* base, int64_t rows, int64_t cols,
                            int box_rows) {
-  EncodeTiledFn enc = get_encoder();
+  TensorMapEncodeFn enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
@@ -191,11 +170,6 @@ static bool encode_bf16_2d(CUtensorMap* m, const void* base, int64_t rows, int64
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
-
-struct TcPlan {
-  int n_tile, tiles_n, tiles_m, kblocks, kb_per_split, ksplit, stages;
-  size_t smem;
-};
 
 TcPlan plan_base_tc(int64_t d_out, int64_t d_in, int64_t batch) {
   TcPlan p;

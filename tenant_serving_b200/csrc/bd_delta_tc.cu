@@ -584,26 +584,6 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_delta_tc(
 // ------------------------------------------------------------------------------------
 // host side
 // ------------------------------------------------------------------------------------
-typedef CUresult (*EncodeTiledFn2)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn2 get_encoder2() {
-  static EncodeTiledFn2 fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn2>(p);
-    else
-      (void)cudaGetLastError();
-  }
-  return fn;
-}
 
 size_t delta_tc_smem(int nmax, int xwin) {
   size_t need = 1024 + (size_t)xwin * DT_KPW * nmax * DT_BK * 2 +
@@ -633,7 +613,7 @@ bd_status launch_delta_tc(const bd_tenant* tc_rec, const int32_t* seg, int max_g
   launch_end(K_TC_GATHER, s);
   BD_LAUNCH_CHECK();
   // 2. tensor-core delta + combine
-  EncodeTiledFn2 enc = get_encoder2();
+  TensorMapEncodeFn enc = tensor_map_encoder();
   if (!enc) return BD_ERR_CUDA;
   CUtensorMap tm;
   cuuint64_t dims[2] = {(cuuint64_t)d_in, (cuuint64_t)xg_rows};

@@ -40,10 +40,33 @@ enum KernelKind : int32_t {
   K_TC_GATHER,           // gather + fp16 scaling of the tensor-core segments' tokens
   K_DELTA_TC,            // tcgen05 delta product of many-token tenants + combine
   K_SELFTEST_WAIT,       // failure-detection self test: a bounded wait that runs out
+  K_QUANT_FP8,           // per-row e4m3 quantization of a base matrix
+  K_X_LIMBS,             // activations -> two e4m3 limbs per value + a power-of-two per token
+  K_BASE_FP8,            // tcgen05 base product from e4m3 weights (fp32 accumulation in TMEM)
   K_KIND_COUNT
 };
 
 const char* kernel_name(int32_t kind);
+
+// Launch plans of the two base products (bd_base_tc.cu, bd_base_fp8.cu), used by the
+// apply call to size its workspace and launch them.
+struct TcPlan {
+  int n_tile, tiles_n, tiles_m, kblocks, kb_per_split, ksplit, stages;
+  size_t smem;
+};
+struct Fp8Plan {
+  int h, n_tile, tiles_n, tiles_m, kblocks, kb_per_split, ksplit, stages;  // h tokens per N tile
+  size_t smem, x8_bytes;
+  int xmul_count;
+};
+TcPlan plan_base_tc(int64_t d_out, int64_t d_in, int64_t batch);
+bd_status launch_base_tc(const TcPlan& p, const void* w_base, const void* x, int64_t d_out,
+                         int64_t d_in, int64_t batch, float* y_part, uint32_t* status,
+                         cudaStream_t s);
+Fp8Plan plan_base_fp8(int64_t d_out, int64_t d_in, int64_t batch);
+bd_status launch_base_fp8(const Fp8Plan& p, const uint8_t* codes, const float* w_scales, const void* x,
+                          int64_t d_out, int64_t d_in, int64_t batch, uint8_t* x8, float* xmul, float* y_part,
+                          uint32_t* status, cudaStream_t s);
 
 // Called around every kernel launch of the library (bd_abi.cu).
 void launch_begin(int32_t kind, cudaStream_t s);

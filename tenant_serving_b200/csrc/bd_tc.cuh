@@ -4,9 +4,32 @@
 #pragma once
 
 #include <cuda.h>  // CUtensorMap (type only; the encoder is fetched at run time)
+#include <cuda_runtime.h>
 #include <stdint.h>
 
 namespace bd {
+
+// cuTensorMapEncodeTiled, fetched from the driver at run time (the library does not link
+// libcuda); nullptr when unavailable.
+typedef CUresult (*TensorMapEncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                      const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                      CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                      CUtensorMapFloatOOBfill);
+inline TensorMapEncodeFn tensor_map_encoder() {
+  static TensorMapEncodeFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<TensorMapEncodeFn>(p);
+    else
+      (void)cudaGetLastError();
+  }
+  return fn;
+}
 
 // About 2 s at the B200's ~1.9 GHz SM clock: every wait on an mbarrier gives up after
 // this many cycles, sets BD_DEV_TIMEOUT and lets the kernel leave cleanly.
@@ -117,6 +140,17 @@ __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64
       : "memory");
 }
 
+// D[tmem] (+)= A[smem desc] * B[smem desc], kind::f8f6f4 (8-bit float in, fp32 accumulate)
+__device__ __forceinline__ void umma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                        uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive (once) on `bar` when every tcgen05.mma issued so far by this thread is done.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -159,6 +193,15 @@ __host__ __device__ constexpr uint32_t umma_idesc_f16(int m, int n, bool bf16) {
   return (1u << 4)                              // D format: fp32
          | ((bf16 ? 1u : 0u) << 7)              // A format
          | ((bf16 ? 1u : 0u) << 10)             // B format
+         | ((uint32_t)(n >> 3) << 17)           // N / 8
+         | ((uint32_t)(m >> 4) << 24);          // M / 16
+}
+
+// Instruction descriptor, kind::f8f6f4: D fp32, A and B both e4m3 (format code 0), K-major.
+__host__ __device__ constexpr uint32_t umma_idesc_e4m3(int m, int n) {
+  return (1u << 4)                              // D format: fp32
+         | (0u << 7)                            // A format: e4m3
+         | (0u << 10)                           // B format: e4m3
          | ((uint32_t)(n >> 3) << 17)           // N / 8
          | ((uint32_t)(m >> 4) << 24);          // M / 16
 }
