@@ -31,6 +31,7 @@ from .bitdelta import (  # noqa: F401
     MODE_ROW,
     MODE_COL,
     MODE_TENSOR,
+    MODE_BLOCK,
     decode,
     delta,
     clip_stats,

@@ -30,8 +30,9 @@ MODE_GROUP = 0   # one scale per contiguous run of G entries along d_in
 MODE_ROW = 1     # one scale per output row (a 1 x d_out vector)
 MODE_COL = 2     # one scale per input column (a d_in x 1 vector)
 MODE_TENSOR = 3  # one scalar for the whole matrix (the original per-matrix alpha)
+MODE_BLOCK = 4   # one scale per square block of G rows x G columns
 
-_MODES = (MODE_GROUP, MODE_ROW, MODE_COL, MODE_TENSOR)
+_MODES = (MODE_GROUP, MODE_ROW, MODE_COL, MODE_TENSOR, MODE_BLOCK)
 
 
 # ----------------------------------------------------------------------------------
@@ -122,6 +123,12 @@ def abs_mean_scales(dc: np.ndarray, mode: int, group_size: int = 128) -> np.ndar
       slice, the L2-optimal value for fixed signs ("BitDelta Guide",
       "2. Optimal L2 Norm Initialization", applied per slice).
     * tensor: one scalar, ``alpha = (1 / (n m)) sum |delta_ij|`` (same section).
+    * block: "Per-Axis Weight Deltas", Future Directions, names blockwise per-group
+      scaling without defining the block. Reading: the group of G entries along a row
+      extended to a square block of G rows x G columns (rows ``G rb .. G rb + G - 1``,
+      columns ``G g .. G g + G - 1``), one abs-mean per block; the last row block holds
+      the ``d_out % G`` remaining rows when G does not divide d_out. Shape
+      ``[ceil(d_out / G), d_in // G]``.
     """
     dc = np.asarray(dc, dtype=np.float64)
     a = np.abs(dc)
@@ -140,6 +147,17 @@ def abs_mean_scales(dc: np.ndarray, mode: int, group_size: int = 128) -> np.ndar
         return a.mean(axis=0)
     if mode == MODE_TENSOR:
         return np.array([a.mean()])
+    if mode == MODE_BLOCK:
+        if a.ndim != 2 or group_size <= 0 or a.shape[1] % group_size != 0:
+            raise ValueError("block scales need a [d_out, d_in] matrix with G dividing d_in")
+        d_out, d_in = a.shape
+        G = group_size
+        nrb = -(-d_out // G)
+        s = np.empty((nrb, d_in // G))
+        for rb in range(nrb):
+            blk = a[rb * G:(rb + 1) * G]
+            s[rb] = blk.reshape(blk.shape[0], d_in // G, G).mean(axis=(0, 2))
+        return s
     raise ValueError(f"unknown scale mode {mode}")
 
 
@@ -213,6 +231,9 @@ def expand_scales(scales: np.ndarray, mode: int, group_size: int, d_out: int, d_
         return np.repeat(s.reshape(1, d_in), len(r), axis=0)
     if mode == MODE_TENSOR:
         return np.full((len(r), d_in), float(s.reshape(-1)[0]))
+    if mode == MODE_BLOCK:
+        s = s.reshape(-(-d_out // group_size), d_in // group_size)[r // group_size]
+        return np.repeat(s, group_size, axis=1)
     raise ValueError(f"unknown scale mode {mode}")
 
 

@@ -158,6 +158,46 @@ def test_row_col_group_by_loops():
 
 
 # --------------------------------------------------------------------------------
+# blockwise scales ("Per-Axis Weight Deltas", Future Directions: blockwise per-group
+# scaling), square G x G blocks, by pure-Python loops with a ragged last row block
+# --------------------------------------------------------------------------------
+def test_block_by_loops():
+    rng = np.random.default_rng(12)
+    d_out, d_in, G = 70, 96, 32
+    d = rng.normal(size=(d_out, d_in))
+    blk = O.abs_mean_scales(d, O.MODE_BLOCK, G)
+    assert blk.shape == (3, 3)
+    for rb in range(3):
+        for g in range(3):
+            acc, n = 0.0, 0
+            for o in range(rb * G, min((rb + 1) * G, d_out)):
+                for i in range(g * G, (g + 1) * G):
+                    acc += abs(d[o, i])
+                    n += 1
+            assert n == (G * G if rb < 2 else 6 * G)
+            assert abs(blk[rb, g] - acc / n) < 1e-14
+
+
+def test_block_special_cases():
+    rng = np.random.default_rng(13)
+    G = 32
+    # one row: a block is a group
+    d = rng.normal(size=(1, 128))
+    assert np.array_equal(O.abs_mean_scales(d, O.MODE_BLOCK, G), O.abs_mean_scales(d, O.MODE_GROUP, G))
+    # rows repeated within each block: the block scale is the group scale of any row
+    base = rng.normal(size=(2, 64))
+    d = np.repeat(base, G, axis=0)
+    blk = O.abs_mean_scales(d, O.MODE_BLOCK, G)
+    grp = O.abs_mean_scales(base, O.MODE_GROUP, G)
+    np.testing.assert_allclose(blk, grp, rtol=1e-14, atol=0)
+    # expand: entry (o, i) takes block (o // G, i // G)
+    e = O.expand_scales(blk, O.MODE_BLOCK, G, 2 * G, 64)
+    for o in (0, G - 1, G, 2 * G - 1):
+        for i in (0, G - 1, G, 63):
+            assert e[o, i] == blk[o // G, i // G]
+
+
+# --------------------------------------------------------------------------------
 # clip ("bitdelta" page, "Safety Benefits: 1. Outlier Clipping")
 # --------------------------------------------------------------------------------
 @pytest.mark.parametrize("n,k", [(16, 1.0), (100, 3.0), (9, 2.0)])
@@ -190,10 +230,10 @@ def test_clip_single_entry_is_identity():
 # --------------------------------------------------------------------------------
 # invariants of sign x abs-mean reconstruction, per group
 # --------------------------------------------------------------------------------
-@pytest.mark.parametrize("mode", [O.MODE_GROUP, O.MODE_ROW, O.MODE_COL, O.MODE_TENSOR])
+@pytest.mark.parametrize("mode", [O.MODE_GROUP, O.MODE_ROW, O.MODE_COL, O.MODE_TENSOR, O.MODE_BLOCK])
 def test_reconstruction_invariants(mode):
     rng = np.random.default_rng(21 + mode)
-    d_out, d_in, G = 6, 256, 64
+    d_out, d_in, G = (6, 256, 64) if mode != O.MODE_BLOCK else (40, 128, 16)
     wb = rng.normal(0, 0.02, size=(d_out, d_in)).astype(np.float32)
     wf = (wb + rng.normal(0, 0.002, size=(d_out, d_in))).astype(np.float32)
     out = O.compress(wb, wf, "f32", mode, G)
@@ -206,6 +246,9 @@ def test_reconstruction_invariants(mode):
         slices = [(slice(o, o + 1), slice(None)) for o in range(d_out)]
     elif mode == O.MODE_COL:
         slices = [(slice(None), slice(i, i + 1)) for i in range(d_in)]
+    elif mode == O.MODE_BLOCK:
+        slices = [(slice(rb * G, (rb + 1) * G), slice(g * G, (g + 1) * G))
+                  for rb in range(-(-d_out // G)) for g in range(d_in // G)]
     else:
         slices = [(slice(None), slice(None))]
     for sl in slices:

@@ -44,8 +44,13 @@ def _clip_pins():
 
 def _reconstruction_pins():
     T.test_worked_reconstruction()
-    for mode in (O.MODE_GROUP, O.MODE_ROW, O.MODE_COL, O.MODE_TENSOR):
+    for mode in (O.MODE_GROUP, O.MODE_ROW, O.MODE_COL, O.MODE_TENSOR, O.MODE_BLOCK):
         T.test_reconstruction_invariants(mode)
+
+
+def _block_pins():
+    T.test_block_by_loops()
+    T.test_block_special_cases()
 
 
 def _apply_pins():
@@ -57,7 +62,8 @@ def _apply_pins():
 def test_pins_pass_on_the_real_oracle():
     for pins in (T.test_worked_delta, T.test_worked_group_scale, _all_worked_signs,
                  T.test_sign_of_zero_is_plus_one, T.test_pack_bit_positions, _l2_pins,
-                 T.test_row_col_group_by_loops, _clip_pins, _reconstruction_pins, _apply_pins):
+                 T.test_row_col_group_by_loops, _clip_pins, _reconstruction_pins, _apply_pins,
+                 _block_pins):
         pins()
 
 
@@ -168,3 +174,38 @@ def test_apply_uses_the_wrong_tenant(monkeypatch):
         return orig(w_base, w_dtype, tenants, shifted, x, x_dtype, rows=rows)
     _patch(monkeypatch, "apply_multi", apply)
     assert _caught(_apply_pins)
+
+
+def test_block_rows_off_by_one(monkeypatch):
+    real = OB.abs_mean_scales
+
+    def scales(dc, mode, group_size=128):
+        if mode != O.MODE_BLOCK:
+            return real(dc, mode, group_size)
+        a = np.abs(np.asarray(dc, dtype=np.float64))
+        G = group_size
+        nrb = -(-a.shape[0] // G)
+        out = np.empty((nrb, a.shape[1] // G))
+        for rb in range(nrb):
+            blk = a[rb * G:(rb + 1) * G - 1] if rb * G + 1 < a.shape[0] else a[rb * G:]
+            out[rb] = blk.reshape(blk.shape[0], -1, G).mean(axis=(0, 2))
+        return out
+    _patch(monkeypatch, "abs_mean_scales", scales)
+    assert _caught(_block_pins, _reconstruction_pins)
+
+
+def test_block_index_transposed(monkeypatch):
+    real = OB.expand_scales
+
+    def expand(scales, mode, group_size, d_out, d_in, rows=None):
+        if mode != O.MODE_BLOCK:
+            return real(scales, mode, group_size, d_out, d_in, rows)
+        nrb, ngc = -(-d_out // group_size), d_in // group_size
+        s = np.asarray(scales, dtype=np.float64).reshape(nrb, ngc)
+        r = np.arange(d_out) if rows is None else np.asarray(rows)
+        # block row taken from the column and block column from the row
+        bi = np.minimum(np.arange(d_in)[None, :] // group_size, nrb - 1) + 0 * r[:, None]
+        bj = np.minimum(r[:, None] // group_size, ngc - 1) + 0 * np.arange(d_in)[None, :]
+        return s[bi, bj]
+    _patch(monkeypatch, "expand_scales", expand)
+    assert _caught(_block_pins, _reconstruction_pins)
