@@ -443,7 +443,7 @@ def bench_serving(args, rank, pg, log, peaks):
 
 def bench_compress(args, log, peaks):
     """bd_compress over the 32-layer stack: group-128 scales without and with the 3-sigma
-    clip, row and column scales; each with the 224 independent calls spread over
+    clip, row, column and 128 x 128 block scales; each with the 224 independent calls spread over
     COMPRESS_STREAMS CUDA streams and on a single stream (one call after another)."""
     import torch
     import tenant_serving_b200 as bd
@@ -462,7 +462,8 @@ def bench_compress(args, log, peaks):
     out = {}
     main_s = torch.cuda.current_stream()
     variants = (("group128", bd.BD_SCALE_GROUP, False), ("group128_clip3", bd.BD_SCALE_GROUP, True),
-                ("row", bd.BD_SCALE_ROW, False), ("col", bd.BD_SCALE_COL, False))
+                ("row", bd.BD_SCALE_ROW, False), ("col", bd.BD_SCALE_COL, False),
+                ("block128", bd.BD_SCALE_BLOCK, False))
     for label, mode, clip in variants:
         cfg = bd.compress_cfg(mode=mode, group_size=GROUP, clip=clip, clip_k=3.0)
         bufs = []
@@ -475,8 +476,7 @@ def bench_compress(args, log, peaks):
             bufs.append((signs, scales, ws))
         # algorithmic bytes: bf16 W_base + W_fine read once, sign bits and fp32 scales written
         # (the clip's statistics pass is a second read, not counted)
-        scale_bytes = sum((d_out * d_in // GROUP if mode == bd.BD_SCALE_GROUP else
-                           d_out if mode == bd.BD_SCALE_ROW else d_in) * 4 for d_out, d_in, _, _ in mats)
+        scale_bytes = sum(math.prod(bd.scales_shape(mode, d_out, d_in, GROUP)) * 4 for d_out, d_in, _, _ in mats)
         alg = params * (4 + 1 / 8) + scale_bytes
         res = {}
         for nstreams in (COMPRESS_STREAMS, 1):

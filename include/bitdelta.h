@@ -69,9 +69,16 @@ typedef enum { BD_F32 = 0, BD_BF16 = 1, BD_F16 = 2 } bd_dtype;
  *  COL   : one scale per input column, scales[d_in] (the d_in x 1 vector).
  *  TENSOR: one scalar alpha for the whole matrix, scales[1] ("BitDelta Guide",
  *          "2. Optimal L2 Norm Initialization").
+ *  BLOCK : one scale per square block of group_size rows x group_size columns,
+ *          scales[ceil(d_out/group_size)][d_in/group_size]; the last row block holds
+ *          the remaining d_out % group_size rows ("Per-Axis Weight Deltas", Future
+ *          Directions: blockwise per-group scaling, read as the row group extended to a
+ *          square block).
  * Every scale is the abs-mean of its slice of the clipped delta, the L2-optimal
- * value for fixed signs. */
-typedef enum { BD_SCALE_GROUP = 0, BD_SCALE_ROW = 1, BD_SCALE_COL = 2, BD_SCALE_TENSOR = 3 } bd_scale_mode;
+ * value for fixed signs. GROUP and BLOCK need group_size a power of two >= 32 that
+ * divides d_in. */
+typedef enum { BD_SCALE_GROUP = 0, BD_SCALE_ROW = 1, BD_SCALE_COL = 2, BD_SCALE_TENSOR = 3,
+               BD_SCALE_BLOCK = 4 } bd_scale_mode;
 
 /* Device status bits (bd_get_status). */
 #define BD_DEV_TENANT_RANGE 0x1u  /* some token had a tenant id outside [-1, n_tenants) */

@@ -9,7 +9,7 @@ from ._lib import (  # noqa: F401
     BD_OK, BD_ERR_NULL, BD_ERR_SHAPE, BD_ERR_DTYPE, BD_ERR_ALIGN, BD_ERR_CONFIG, BD_ERR_CUDA,
     BD_ERR_TENANT_RANGE, BD_ERR_TIMEOUT, BD_ERR_WORKSPACE, BD_ERR_TENANT_RECORD, BD_ERR_INTERNAL,
     BD_F32, BD_BF16, BD_F16,
-    BD_SCALE_GROUP, BD_SCALE_ROW, BD_SCALE_COL, BD_SCALE_TENSOR,
+    BD_SCALE_GROUP, BD_SCALE_ROW, BD_SCALE_COL, BD_SCALE_TENSOR, BD_SCALE_BLOCK,
     BD_DEV_TENANT_RANGE, BD_DEV_TIMEOUT, BD_DEV_TENANT_RECORD, BD_DEV_INTERNAL,
     BD_LAYOUT_ROWMAJOR, BD_LAYOUT_TILED, bd_prepare_tenant,
     EXPORTS, LIB_PATH, BitDeltaError, TenantTable, bd_compress_cfg, bd_tenant,

@@ -30,7 +30,7 @@ BD_ERR_TENANT_RECORD = 10
 BD_ERR_INTERNAL = 11
 
 BD_F32, BD_BF16, BD_F16 = 0, 1, 2
-BD_SCALE_GROUP, BD_SCALE_ROW, BD_SCALE_COL, BD_SCALE_TENSOR = 0, 1, 2, 3
+BD_SCALE_GROUP, BD_SCALE_ROW, BD_SCALE_COL, BD_SCALE_TENSOR, BD_SCALE_BLOCK = 0, 1, 2, 3, 4
 BD_DEV_TENANT_RANGE, BD_DEV_TIMEOUT, BD_DEV_TENANT_RECORD, BD_DEV_INTERNAL = 0x1, 0x2, 0x4, 0x8
 BD_LAYOUT_ROWMAJOR, BD_LAYOUT_TILED = 0, 1
 
@@ -220,6 +220,8 @@ def scales_shape(mode, d_out, d_in, group_size):
         return (d_out,)
     if mode == BD_SCALE_COL:
         return (d_in,)
+    if mode == BD_SCALE_BLOCK:
+        return (-(-d_out // group_size), d_in // group_size)
     return (1,)
 
 

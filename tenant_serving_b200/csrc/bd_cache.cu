@@ -78,11 +78,7 @@ size_t record_bytes(int64_t d_out, int64_t d_in, int32_t mode, int32_t G, int32_
 
 bool shape_ok(int64_t d_out, int64_t d_in) { return d_out >= 1 && d_in >= 32 && (d_in % 32) == 0; }
 
-bool mode_ok(int64_t d_in, int32_t mode, int32_t G) {
-  if (mode < BD_SCALE_GROUP || mode > BD_SCALE_TENSOR) return false;
-  if (mode == BD_SCALE_GROUP && (G < 32 || !bd::is_pow2(G) || (d_in % G) != 0)) return false;
-  return true;
-}
+bool mode_ok(int64_t d_in, int32_t mode, int32_t G) { return bd::scale_mode_ok(mode, G, d_in); }
 
 // The largest record a tenant of this module may have: every scale mode, group sizes from
 // min_group up to d_in.
@@ -94,8 +90,10 @@ size_t region_bytes(int64_t d_out, int64_t d_in, int32_t min_group, int32_t sdt)
   }
   for (int64_t G = min_group; G <= d_in; G *= 2) {
     if (d_in % G) continue;
-    const size_t b = record_bytes(d_out, d_in, BD_SCALE_GROUP, (int32_t)G, sdt);
-    if (b > m) m = b;
+    for (int32_t mode : {(int32_t)BD_SCALE_GROUP, (int32_t)BD_SCALE_BLOCK}) {
+      const size_t b = record_bytes(d_out, d_in, mode, (int32_t)G, sdt);
+      if (b > m) m = b;
+    }
   }
   return bd::align_up(m, kRegionAlign);
 }
@@ -204,10 +202,7 @@ extern "C" bd_status bd_prepare_record_host(const uint32_t* signs, const void* s
               std::memcpy(sc_out + ((rb * nwin + w) * 1024 + r * 2 + k) * ssz, sc_in + (row * gpr + g) * ssz, ssz);
           }
   } else {
-    size_t n = 1;
-    if (mode == BD_SCALE_GROUP) n = (size_t)(d_out * (d_in / group_size));
-    else if (mode == BD_SCALE_ROW) n = (size_t)d_out;
-    else if (mode == BD_SCALE_COL) n = (size_t)d_in;
+    const size_t n = (size_t)bd::scale_count(mode, group_size, d_out, d_in);
     std::memcpy(sc_out, sc_in, n * ssz);
   }
   return BD_OK;
@@ -308,13 +303,13 @@ extern "C" bd_status bd_cache_register(bd_cache* c, int32_t tenant, int32_t modu
   if (module < 0 || module >= (int32_t)c->mods.size()) return BD_ERR_SHAPE;
   const bd_cache::Module& M = c->mods[module];
   if (!mode_ok(M.d_in, mode, group_size)) return BD_ERR_CONFIG;
-  if (mode == BD_SCALE_GROUP && group_size < M.min_group) return BD_ERR_CONFIG;
+  if ((mode == BD_SCALE_GROUP || mode == BD_SCALE_BLOCK) && group_size < M.min_group) return BD_ERR_CONFIG;
   if (!bd::aligned16(record_host)) return BD_ERR_ALIGN;
   if (c->tenant_slot[tenant] >= 0) return BD_ERR_CONFIG;  // resident: its slot still holds the old record
   bd_cache::Entry& e = c->entries[(size_t)tenant * c->mods.size() + module];
   e.host = record_host;
   e.mode = mode;
-  e.group_size = mode == BD_SCALE_GROUP ? group_size : 0;
+  e.group_size = (mode == BD_SCALE_GROUP || mode == BD_SCALE_BLOCK) ? group_size : 0;
   e.bytes = record_bytes(M.d_out, M.d_in, mode, group_size, c->scale_dtype);
   return BD_OK;
 }

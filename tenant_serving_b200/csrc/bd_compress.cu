@@ -19,6 +19,9 @@
 //                      keeping fp64 column sums in registers; fp64 partials per tile.
 //   k_scale_final      fixed-order reduction of the partials into row / column / tensor
 //                      scales (deterministic, no atomics).
+//   k_block_final      BLOCK mode: the main pass writes each row's group means; the
+//                      block scale is their mean over the block's rows, in fp64 and in
+//                      row order.
 #include "bd_internal.cuh"
 
 #include <math.h>
@@ -426,6 +429,20 @@ __global__ void k_col_final(const double* __restrict__ colpart, int64_t ntile, i
   scales[i] = (float)(s / (double)d_out);
 }
 
+// BLOCK: scales[rb][g] = mean over rows r of row block rb of rowmean[r][g] (each row mean
+// is over G entries, so this is the mean over the block's entries); fp64, row order
+__global__ void k_block_final(const float* __restrict__ rowmean, int64_t d_out, int64_t ngc, int G,
+                              float* __restrict__ scales) {
+  const int64_t nrb = (d_out + G - 1) / G;
+  const int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= nrb * ngc) return;
+  const int64_t rb = k / ngc, g = k - rb * ngc;
+  const int64_t r0 = rb * G, r1 = r0 + G < d_out ? r0 + G : d_out;
+  double s = 0.0;
+  for (int64_t r = r0; r < r1; ++r) s += (double)rowmean[r * ngc + g];
+  scales[k] = (float)(s / (double)(r1 - r0));
+}
+
 // TENSOR: one block; strided per-thread sums then a fixed tree
 __global__ void k_tensor_final(const double* __restrict__ partials, int64_t n, double count,
                                float* __restrict__ scales) {
@@ -465,13 +482,12 @@ bd_status plan_compress(int32_t dtype, int64_t d_out, int64_t d_in, const bd_com
   if (dtype != BD_F32 && dtype != BD_BF16) return BD_ERR_DTYPE;
   if (d_out < 1 || d_in < 32 || (d_in % 32) != 0) return BD_ERR_SHAPE;
   if (d_in > ((int64_t)1 << 30) || d_out > ((int64_t)1 << 40)) return BD_ERR_SHAPE;
-  if (cfg->mode < BD_SCALE_GROUP || cfg->mode > BD_SCALE_TENSOR) return BD_ERR_CONFIG;
+  if (cfg->mode < BD_SCALE_GROUP || cfg->mode > BD_SCALE_BLOCK) return BD_ERR_CONFIG;
   if (cfg->clip != 0 && cfg->clip != 1) return BD_ERR_CONFIG;
   if (cfg->clip && !(cfg->clip_k >= 0.0f)) return BD_ERR_CONFIG;
   const int64_t G = cfg->group_size;
-  if (cfg->mode == BD_SCALE_GROUP) {
-    if (G < 32 || !is_pow2(G) || (d_in % G) != 0) return BD_ERR_CONFIG;
-  }
+  const bool grouped = cfg->mode == BD_SCALE_GROUP || cfg->mode == BD_SCALE_BLOCK;
+  if (!scale_mode_ok(cfg->mode, cfg->group_size, d_in)) return BD_ERR_CONFIG;
   p->bf16 = dtype == BD_BF16;
   p->chunk = p->bf16 ? 256 : 128;
   p->nchunks = (d_in + p->chunk - 1) / p->chunk;
@@ -479,7 +495,7 @@ bd_status plan_compress(int32_t dtype, int64_t d_out, int64_t d_in, const bd_com
   const int64_t target_tasks = (int64_t)sms * 64;  // warps in flight we want
   int segc = 4;
   while (segc > 1 && d_out * ((p->nchunks + segc - 1) / segc) < target_tasks) segc >>= 1;
-  if (cfg->mode == BD_SCALE_GROUP && G > p->chunk) {
+  if (grouped && G > p->chunk) {
     const int need = (int)(G / p->chunk);
     segc = ((segc + need - 1) / need) * need;
   }
@@ -505,6 +521,8 @@ bd_status plan_compress(int32_t dtype, int64_t d_out, int64_t d_in, const bd_com
     part = (size_t)d_out * p->nseg * sizeof(double);
   else if (cfg->mode == BD_SCALE_COL)
     part = (size_t)p->ntile * d_in * sizeof(double);
+  else if (cfg->mode == BD_SCALE_BLOCK)
+    part = (size_t)d_out * (size_t)(d_in / G) * sizeof(float);  // row group means
   off = align_up(off + part, 256);
   p->total = off;
   return BD_OK;
@@ -550,15 +568,17 @@ bd_status launch_compress(const CompressPlan& p, const void* w_base, const void*
     return BD_OK;
   }
   const unsigned blocks = (unsigned)p.main_blocks;
-  const bool group = cfg->mode == BD_SCALE_GROUP;
+  const bool group = cfg->mode == BD_SCALE_GROUP || cfg->mode == BD_SCALE_BLOCK;
   int lg = 0;
   if (group)
     while ((1 << lg) < cfg->group_size) ++lg;
   const int din = (int)d_in;
+  // BLOCK: the per-row group means go to the workspace, the block means follow
+  float* group_out = cfg->mode == BD_SCALE_BLOCK ? reinterpret_cast<float*>(part) : scales;
 #define BD_SIGNPACK(SEGC, CLIP, GRP)                                                           \
   k_scale_signpack<BF16, SEGC, CLIP, GRP><<<blocks, 256, 0, s>>>(                              \
       (const uint8_t*)w_base, (const uint8_t*)w_fine, d_out, din, lg, p.seg_chunks, p.nseg,    \
-      clipp, signs, scales, part)
+      clipp, signs, group_out, part)
   launch_begin(K_SCALE_SIGNPACK, s);
   if (p.seg_chunks >= 4) {
     if (clip) { if (group) BD_SIGNPACK(4, true, true); else BD_SIGNPACK(4, true, false); }
@@ -573,6 +593,13 @@ bd_status launch_compress(const CompressPlan& p, const void* w_base, const void*
   if (cfg->mode == BD_SCALE_ROW) {
     launch_begin(K_SCALE_FINAL, s);
     k_row_final<<<(unsigned)((d_out + 255) / 256), 256, 0, s>>>(part, p.nseg, d_out, d_in, scales);
+    launch_end(K_SCALE_FINAL, s);
+    BD_LAUNCH_CHECK();
+  } else if (cfg->mode == BD_SCALE_BLOCK) {
+    const int64_t ngc = d_in >> lg, n = ((d_out + cfg->group_size - 1) / cfg->group_size) * ngc;
+    launch_begin(K_SCALE_FINAL, s);
+    k_block_final<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(reinterpret_cast<const float*>(part), d_out, ngc,
+                                                              cfg->group_size, scales);
     launch_end(K_SCALE_FINAL, s);
     BD_LAUNCH_CHECK();
   } else if (cfg->mode == BD_SCALE_TENSOR) {

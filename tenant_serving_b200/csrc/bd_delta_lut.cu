@@ -277,13 +277,11 @@ __device__ __forceinline__ bool walk_next(DlWalk& w, const int32_t* __restrict__
   if (pc.u >= 0) {
     pc.T = tenants[pc.u];
     const bd_tenant& T = pc.T;
-    const bool ok_mode = T.mode >= BD_SCALE_GROUP && T.mode <= BD_SCALE_TENSOR;
-    const bool ok_group = T.mode != BD_SCALE_GROUP ||
-                          (T.group_size >= 32 && (T.group_size & (T.group_size - 1)) == 0 && (d_in % T.group_size) == 0);
+    const bool ok_mode = scale_mode_ok(T.mode, T.group_size, d_in);
     const bool ok_ptr = T.signs != nullptr && T.scales != nullptr &&
                         ((reinterpret_cast<uintptr_t>(T.signs) | reinterpret_cast<uintptr_t>(T.scales)) & 15u) == 0;
     const bool ok_layout = (T.layout == BD_LAYOUT_ROWMAJOR || T.layout == BD_LAYOUT_TILED) && T.reserved == 0;
-    if (!(ok_mode && ok_group && ok_ptr && ok_layout)) {
+    if (!(ok_mode && ok_ptr && ok_layout)) {
       *bad = true;
       pc.u = -1;
     }
@@ -293,10 +291,11 @@ __device__ __forceinline__ bool walk_next(DlWalk& w, const int32_t* __restrict__
   pc.ssrc = SS_STAGED;
   if (pc.u >= 0) {
     const bd_tenant& T = pc.T;
-    if (T.mode == BD_SCALE_GROUP)
+    if (T.mode == BD_SCALE_GROUP || T.mode == BD_SCALE_BLOCK)
       while ((1 << pc.lg) < T.group_size) ++pc.lg;
     const bool tiled = T.layout == BD_LAYOUT_TILED;
-    pc.skind = T.mode != BD_SCALE_GROUP ? SK_NONE : ((T.group_size == 128 && tiled) ? SK_STAGED : SK_GLOBAL);
+    pc.skind = T.mode == BD_SCALE_BLOCK ? SK_GLOBAL
+               : T.mode != BD_SCALE_GROUP ? SK_NONE : ((T.group_size == 128 && tiled) ? SK_STAGED : SK_GLOBAL);
     pc.ssrc = (tiled || (d_in % DL_W) == 0) ? SS_STAGED : SS_DIRECT;
   }
   return true;
@@ -502,10 +501,11 @@ __device__ __forceinline__ void dl_row_window(const DlDesc& D, uint32_t st, int 
     const int lg = D.lg;
     const void* scales = D.scales;
     const int64_t gpr = d_in >> lg;
+    const int64_t srow = D.mode == BD_SCALE_BLOCK ? (row >> lg) : row;  // BLOCK: G x G blocks
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int64_t col = (int64_t)win * DL_W + 32 * ((i + sig) & 7);
-      sc[i] = (live && col < d_in) ? ldg_scale(scales, scale_f16, row * gpr + (col >> lg)) : 0.f;
+      sc[i] = (live && col < d_in) ? ldg_scale(scales, scale_f16, srow * gpr + (col >> lg)) : 0.f;
     }
   } else {
 #pragma unroll

@@ -306,14 +306,17 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_delta_tc(
       const bool live = row < d_out;
       const uint16_t* sc16 = static_cast<const uint16_t*>(T.scales);
       // scale source: 0 = tiled group-128 scales in the window ring, 1 = one load per
-      // stage (other group sizes), 2 = one value for the whole item (row / tensor)
-      const int kind = T.mode == BD_SCALE_GROUP ? (T.group_size == 128 ? 0 : 1) : 2;
-      const int gshift = T.mode == BD_SCALE_GROUP ? __ffs(T.group_size) - 1 : 0;
+      // stage (other group sizes, and G x G blocks), 2 = one value for the whole item
+      // (row / tensor)
+      const bool blockwise = T.mode == BD_SCALE_BLOCK;
+      const int kind = T.mode == BD_SCALE_GROUP ? (T.group_size == 128 ? 0 : 1) : (blockwise ? 1 : 2);
+      const int gshift = (T.mode == BD_SCALE_GROUP || blockwise) ? __ffs(T.group_size) - 1 : 0;
+      const int64_t srow = blockwise ? (row >> gshift) : row;  // BLOCK: G x G blocks
       uint32_t s_item = 0;
       if (kind == 2 && live) s_item = sc16[T.mode == BD_SCALE_ROW ? row : 0];
       auto stage_scale = [&](int kb) -> uint32_t {
         if (!live || kb >= nkb) return 0u;
-        return sc16[row * (d_in >> gshift) + (((int64_t)kb * DT_BK) >> gshift)];
+        return sc16[srow * (d_in >> gshift) + (((int64_t)kb * DT_BK) >> gshift)];
       };
       uint32_t pre[DT_KPW] = {0, 0, 0, 0};  // kind 1: scales of the next window, loaded ahead
       if (kind == 1) {

@@ -102,6 +102,25 @@ struct DevStatus {
 constexpr size_t kStatusBytes = 256;  // keeps what follows 256-byte aligned
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// A scale mode and group size valid for d_in: GROUP and BLOCK need a power of two >= 32
+// that divides d_in.
+__host__ __device__ inline bool scale_mode_ok(int32_t mode, int32_t G, int64_t d_in) {
+  if (mode < BD_SCALE_GROUP || mode > BD_SCALE_BLOCK) return false;
+  if (mode == BD_SCALE_GROUP || mode == BD_SCALE_BLOCK)
+    return G >= 32 && (G & (G - 1)) == 0 && (d_in % G) == 0;
+  return true;
+}
+// number of scales of a mode
+__host__ __device__ inline int64_t scale_count(int32_t mode, int32_t G, int64_t d_out, int64_t d_in) {
+  switch (mode) {
+    case BD_SCALE_GROUP: return d_out * (d_in / G);
+    case BD_SCALE_ROW: return d_out;
+    case BD_SCALE_COL: return d_in;
+    case BD_SCALE_BLOCK: return ((d_out + G - 1) / G) * (d_in / G);
+    default: return 1;
+  }
+}
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool is_pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
 

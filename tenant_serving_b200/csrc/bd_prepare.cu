@@ -17,12 +17,7 @@ size_t prepared_signs_bytes(int64_t d_out, int64_t d_in) {
 }
 
 static size_t plain_scale_elems(int64_t d_out, int64_t d_in, int32_t mode, int32_t G) {
-  switch (mode) {
-    case BD_SCALE_GROUP: return (size_t)(d_out * (d_in / G));
-    case BD_SCALE_ROW: return (size_t)d_out;
-    case BD_SCALE_COL: return (size_t)d_in;
-    default: return 1;
-  }
+  return (size_t)scale_count(mode, G, d_out, d_in);
 }
 
 size_t prepared_scales_bytes(int64_t d_out, int64_t d_in, int32_t mode, int32_t G, int32_t sdt) {
@@ -71,9 +66,7 @@ extern "C" size_t bd_prepared_signs_bytes(int64_t d_out, int64_t d_in) {
 extern "C" size_t bd_prepared_scales_bytes(int64_t d_out, int64_t d_in, int32_t mode,
                                            int32_t group_size, int32_t scale_dtype) {
   if (d_out < 1 || d_in < 32 || (d_in % 32) != 0) return 0;
-  if (mode < BD_SCALE_GROUP || mode > BD_SCALE_TENSOR) return 0;
-  if (mode == BD_SCALE_GROUP && (group_size < 32 || !bd::is_pow2(group_size) || d_in % group_size))
-    return 0;
+  if (!bd::scale_mode_ok(mode, group_size, d_in)) return 0;
   if (scale_dtype != BD_F16 && scale_dtype != BD_F32) return 0;
   return bd::prepared_scales_bytes(d_out, d_in, mode, group_size, scale_dtype);
 }
@@ -86,9 +79,7 @@ extern "C" bd_status bd_prepare_tenant(const uint32_t* signs, const void* scales
   if (!signs || !scales || !signs_out || !scales_out) return BD_ERR_NULL;
   if (d_out < 1 || d_in < 32 || (d_in % 32) != 0) return BD_ERR_SHAPE;
   if (scale_dtype != BD_F16 && scale_dtype != BD_F32) return BD_ERR_DTYPE;
-  if (mode < BD_SCALE_GROUP || mode > BD_SCALE_TENSOR) return BD_ERR_CONFIG;
-  if (mode == BD_SCALE_GROUP && (group_size < 32 || !is_pow2(group_size) || d_in % group_size))
-    return BD_ERR_CONFIG;
+  if (!scale_mode_ok(mode, group_size, d_in)) return BD_ERR_CONFIG;
   if (!aligned16(signs) || !aligned16(scales) || !aligned16(signs_out) || !aligned16(scales_out))
     return BD_ERR_ALIGN;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

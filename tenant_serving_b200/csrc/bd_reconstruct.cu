@@ -29,6 +29,7 @@ __global__ void __launch_bounds__(256) k_reconstruct(
     } else {
       int64_t idx = 0;
       if (mode == BD_SCALE_GROUP) idx = row * (d_in / group) + col / group;
+      else if (mode == BD_SCALE_BLOCK) idx = (row / group) * (d_in / group) + col / group;
       else if (mode == BD_SCALE_ROW) idx = row;
       const float sv = load_scale(scales, scale_f16, idx);
 #pragma unroll
@@ -81,10 +82,7 @@ extern "C" bd_status bd_reconstruct(const uint32_t* signs, const void* scales, i
   if (scale_dtype != BD_F32 && scale_dtype != BD_F16) return BD_ERR_DTYPE;
   if (out_dtype != BD_F32 && out_dtype != BD_BF16) return BD_ERR_DTYPE;
   if (w_base && w_dtype != BD_F32 && w_dtype != BD_BF16) return BD_ERR_DTYPE;
-  if (mode < BD_SCALE_GROUP || mode > BD_SCALE_TENSOR) return BD_ERR_CONFIG;
-  if (mode == BD_SCALE_GROUP &&
-      (group_size < 32 || !is_pow2(group_size) || (d_in % group_size) != 0))
-    return BD_ERR_CONFIG;
+  if (!scale_mode_ok(mode, group_size, d_in)) return BD_ERR_CONFIG;
   if (!aligned16(signs) || !aligned16(scales) || !aligned16(out) || (w_base && !aligned16(w_base)))
     return BD_ERR_ALIGN;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

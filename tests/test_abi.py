@@ -61,6 +61,10 @@ def test_compress_host_validation(lib):
     for g in (0, 16, 96, 512):
         c = _cfg(mode=bd.BD_SCALE_GROUP, group_size=g)
         assert lib.bd_compress(fake, fake, bd.BD_BF16, 4, 256, ctypes.byref(c), fake, fake, None, fake, 1 << 20, None) == bd.BD_ERR_CONFIG
+    # block sizes follow the group rules
+    for g in (16, 96, 512):
+        c = _cfg(mode=bd.BD_SCALE_BLOCK, group_size=g)
+        assert lib.bd_compress(fake, fake, bd.BD_BF16, 4, 256, ctypes.byref(c), fake, fake, None, fake, 1 << 20, None) == bd.BD_ERR_CONFIG
     # bad mode, bad clip flag
     c = bd.bd_compress_cfg(128, 9, 0, 3.0)
     assert lib.bd_compress(fake, fake, bd.BD_BF16, 4, 256, ctypes.byref(c), fake, fake, None, fake, 1 << 20, None) == bd.BD_ERR_CONFIG

@@ -87,7 +87,7 @@ def test_tiny_config_end_to_end(bd):
 
 @pytest.mark.parametrize("layout", [0, 1])
 @pytest.mark.parametrize("B", [1, 4, 16, 63, 200, 300])
-@pytest.mark.parametrize("mode", [0, 1, 2, 3])
+@pytest.mark.parametrize("mode", [0, 1, 2, 3, 4])
 def test_random_batches(bd, B, mode, layout):
     d_out, d_in = 384 + 8, 1024
     wb, tenants, ids, x = _problem(B * 10 + mode, d_out, d_in, B, 5, (mode,))
@@ -99,7 +99,7 @@ def test_random_batches(bd, B, mode, layout):
 
 
 @pytest.mark.parametrize("layout", [0, 1])
-@pytest.mark.parametrize("mode", [0, 1, 2, 3])
+@pytest.mark.parametrize("mode", [0, 1, 2, 3, 4])
 @pytest.mark.parametrize("d_out,d_in", [(1100, 544), (64, 4096), (2050, 256), (130, 96), (600, 640)])
 def test_delta_only_tight(bd, mode, d_out, d_in, layout):
     """W_base = 0: the bound now constrains the delta product by itself; with fp32
@@ -121,6 +121,7 @@ def test_mixed_modes_and_group_sizes(bd, layout):
     wb = bf16_bits(rng.normal(0, 0.02, size=(d_out, d_in)))
     tenants = [random_tenant(rng, d_out, d_in, 0, g) for g in (32, 64, 128, 256, 512, 2048)]
     tenants += [random_tenant(rng, d_out, d_in, m) for m in (1, 2, 3)]
+    tenants += [random_tenant(rng, d_out, d_in, 4, g) for g in (32, 64, 128, 512)]
     B = 40
     x = activations(rng, B, d_in)
     ids = rng.integers(-1, len(tenants), size=B).astype(np.int32)
@@ -326,7 +327,8 @@ def _many_token_problem(seed, d_out, d_in, counts, mode, G, zero_base=False, x_s
 
 
 @pytest.mark.parametrize("layout", [0, 1])
-@pytest.mark.parametrize("mode,G", [(0, 128), (0, 64), (0, 256), (1, 128), (3, 128), (2, 128)])
+@pytest.mark.parametrize("mode,G", [(0, 128), (0, 64), (0, 256), (1, 128), (3, 128), (2, 128), (4, 64),
+                                    (4, 128)])
 def test_many_token_tenants_delta_only(bd, mode, G, layout):
     """300 tokens (five tensor-core segments), 9 (the smallest many-token tenant), 8 (two
     passes of the lookup-table kernel), 20 and 1 token; 200 rows (a partial 128-row tile),

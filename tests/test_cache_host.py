@@ -39,7 +39,8 @@ def _want_record(t, d_out, d_in):
 
 
 @pytest.mark.parametrize("d_out,d_in,mode,G", [(1100, 640, 0, 128), (513, 544, 0, 32), (300, 4096, 1, 128),
-                                               (70, 256, 2, 128), (9, 128, 3, 128), (1024, 512, 0, 64)])
+                                               (70, 256, 2, 128), (9, 128, 3, 128), (1024, 512, 0, 64),
+                                               (70, 256, 4, 32)])
 @pytest.mark.parametrize("sdt", ["f16", "f32"])
 def test_record_layout(bd, d_out, d_in, mode, G, sdt):
     rng = np.random.default_rng(d_out * 7 + d_in + mode)

@@ -71,7 +71,7 @@ SHAPES = [(1, 32), (3, 96), (37, 256), (64, 544), (129, 1024), (300, 4096 + 96)]
 
 @pytest.mark.parametrize("d_out,d_in", SHAPES)
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
-@pytest.mark.parametrize("mode", [O.MODE_GROUP, O.MODE_ROW, O.MODE_COL, O.MODE_TENSOR])
+@pytest.mark.parametrize("mode", [O.MODE_GROUP, O.MODE_ROW, O.MODE_COL, O.MODE_TENSOR, O.MODE_BLOCK])
 @pytest.mark.parametrize("clip", [False, True])
 def test_random_shapes(bd, d_out, d_in, dtype, mode, clip):
     seed = d_out * 7 + d_in + mode * 1000 + int(clip) * 10000 + (dtype == "f32")
@@ -85,6 +85,14 @@ def test_random_shapes(bd, d_out, d_in, dtype, mode, clip):
 def test_group_sizes(bd, G, dtype):
     wb, wf = weight_pair(G, 40, 2048, dtype, 0.02, 0.002, 0.001, 20.0)
     _check(bd, wb, wf, dtype, O.MODE_GROUP, G, True, 2.0)
+
+
+@pytest.mark.parametrize("G", [32, 64, 128, 256, 512, 1024])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_block_sizes(bd, G, dtype):
+    """G x G blocks over 1100 rows (a ragged last row block for every G)."""
+    wb, wf = weight_pair(G + 1, 1100, 2048, dtype, 0.02, 0.002, 0.001, 20.0)
+    _check(bd, wb, wf, dtype, O.MODE_BLOCK, G, G == 128, 3.0)
 
 
 def test_zero_and_negative_zero(bd):
@@ -138,7 +146,8 @@ def test_reconstruct_matches_oracle(bd):
     d_out, d_in = 70, 768
     words = rng.integers(0, 2 ** 32, size=(d_out, d_in // 32), dtype=np.uint64).astype(np.uint32)
     wb = bf16_bits(rng.normal(0, 0.02, size=(d_out, d_in)))
-    for mode, G in ((O.MODE_GROUP, 64), (O.MODE_ROW, 128), (O.MODE_COL, 128), (O.MODE_TENSOR, 128)):
+    for mode, G in ((O.MODE_GROUP, 64), (O.MODE_ROW, 128), (O.MODE_COL, 128), (O.MODE_TENSOR, 128),
+                    (O.MODE_BLOCK, 32), (O.MODE_BLOCK, 128)):
         shape = bd.scales_shape(mode, d_out, d_in, G)
         s16 = (rng.random(shape) * 0.01).astype(np.float16)
         for sd, s in (("f16", s16), ("f32", s16.astype(np.float32) * 1.5)):

@@ -146,6 +146,8 @@ def random_tenant(rng, d_out: int, d_in: int, mode: int, group_size: int = 128,
         shape = (d_out,)
     elif mode == 2:
         shape = (d_in,)
+    elif mode == 4:
+        shape = (-(-d_out // group_size), d_in // group_size)
     else:
         shape = (1,)
     z = rng.normal(0.0, 1.0, size=shape)
@@ -190,6 +192,8 @@ def device_random_tenant(gen, d_out, d_in, mode, group_size=128, device="cuda"):
         shape = (d_out,)
     elif mode == 2:
         shape = (d_in,)
+    elif mode == 4:
+        shape = (-(-d_out // group_size), d_in // group_size)
     else:
         shape = (1,)
     z = torch.randn(shape, generator=gen, device=device)
