@@ -499,8 +499,6 @@ def bench_compress(args, log, peaks):
                 one_pass()
             torch.cuda.synchronize()
             reps = 3
-            if nstreams == 1:
-                bd.bd_profile_enable(True, capacity=len(mats) * reps * 4 + 16)
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(main_s)
@@ -513,11 +511,14 @@ def bench_compress(args, log, peaks):
             res[key] = {"ms_per_stack": ms, "gbs": alg / (ms / 1e3) / 1e9,
                         "frac": alg / (ms / 1e3) / 1e9 / peaks[0], "streams": nstreams}
             if nstreams == 1:
-                # per-kernel device time of the single-stream run (kernels do not overlap)
+                # per-kernel device time of a further single-stream pass (kernels do not
+                # overlap); the events around each launch are not in the timing above
+                bd.bd_profile_enable(True, capacity=len(mats) * 4 + 16)
+                one_pass()
+                torch.cuda.synchronize()
                 prof = bd.bd_profile_collect()
                 bd.bd_profile_enable(False)
-                res[key]["kernels"] = {k: {"launches": v[0] // reps, "ms_per_stack": v[1] / reps}
-                                       for k, v in prof.items()}
+                res[key]["kernels"] = {k: {"launches": v[0], "ms_per_stack": v[1]} for k, v in prof.items()}
         out[label] = {"params": params, "bytes_per_stack": alg,
                       "tparams_per_s": params / (res["streams4"]["ms_per_stack"] / 1e3) / 1e12, **res}
         if label == "group128":
