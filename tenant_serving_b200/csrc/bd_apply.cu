@@ -61,7 +61,8 @@ constexpr int kPlanQ = 3 + kLutClasses;  // tokens, tc segments, gathered X rows
 __global__ void __launch_bounds__(1024) k_tenant_bucket(const int32_t* __restrict__ ids, int batch,
                                                         int n_tenants, int max_groups, int max_tc,
                                                         const bd_tenant* __restrict__ tenants,
-                                                        int tc_min, int64_t d_in,
+                                                        int tc_min, int64_t d_in, int64_t lut_tiles,
+                                                        int split_cap, int32_t* __restrict__ lut_cnt,
                                                         int32_t* __restrict__ seg_base,
                                                         bd_tenant* __restrict__ tc_rec,
                                                         uint32_t* __restrict__ status) {
@@ -198,8 +199,26 @@ __global__ void __launch_bounds__(1024) k_tenant_bucket(const int32_t* __restric
     seg_base[1] = tidx;
 #pragma unroll
     for (int k = 0; k < kLutClasses; ++k) seg_base[2 + k] = wsum[3 + k][last];
-    seg_base[2 + kLutClasses] = 0;
+    // K chunks of the lookup kernel's tenant units: when there are too few (group, tile)
+    // units to keep every SM busy, each is cut into kc chunks of d_in (kc divides the
+    // windows, >= 2 windows per chunk), as many as the partial-sum budget allows
+    int64_t units = 0;
+#pragma unroll
+    for (int k = 0; k < kLutClasses - 1; ++k) units += wsum[3 + k][last];
+    units *= lut_tiles;
+    const int64_t nwin = (d_in + kLutWindow - 1) / kLutWindow;
+    int kc = 1;
+    if (units > 0)
+      for (int c = kLutMaxChunks; c >= 2; --c)
+        if (nwin % c == 0 && nwin / c >= 2 && units * c <= (int64_t)split_cap) {
+          kc = c;
+          break;
+        }
+    seg_base[2 + kLutClasses] = kc;
   }
+  // the split units' arrival counters and the lookup kernel's piece counter (the word
+  // after them) start from zero in every call
+  for (int i = threadIdx.x; i <= split_cap / 2; i += blockDim.x) lut_cnt[i] = 0;
   __syncthreads();
   for (int t = threadIdx.x; t < batch; t += blockDim.x) {
     int u = ids[t];
@@ -253,7 +272,8 @@ bd_status launch_delta_tc(const bd_tenant* tenants, const int32_t* seg, int max_
 bd_status launch_delta_lut(bool xbf16, const bd_tenant* tenants, bool scale_f16, const int32_t* seg,
                            int max_groups, int max_tc, const void* x, const float* y_part, int ksplit,
                            int64_t d_out, int64_t d_in, int64_t batch, void* y, bool y_bf16,
-                           uint32_t* status, cudaStream_t s);
+                           float* lut_part, int32_t* lut_cnt, int split_cap, uint32_t* status,
+                           cudaStream_t s);
 
 // A tenant with at least this many tokens in a batch (and a supported record) goes to the
 // tensor-core delta kernel; below it the lookup-table kernel serves the tenant's tokens,
@@ -274,8 +294,9 @@ struct ApplyLayout {
   TcPlan tc;
   Fp8Plan f8;
   int ksplit;
+  int split_cap;  // lookup units (x K chunks) that may keep partial sums
   int64_t xg_rows;
-  size_t off_seg, off_tcrec, off_part, off_xg, off_xinv, off_x8, off_xmul, total;
+  size_t off_seg, off_tcrec, off_part, off_xg, off_xinv, off_x8, off_xmul, off_lpart, off_lcnt, total;
 };
 
 // tc: the base product on the tensor cores (bf16 weights, or e4m3 ones when fp8)
@@ -316,6 +337,18 @@ ApplyLayout layout_apply(int64_t d_out, int64_t d_in, int64_t batch, int32_t n_t
   off = align_up(off + (fp8 ? L.f8.x8_bytes : 0), 256);
   L.off_xmul = off;
   off = align_up(off + (fp8 ? (size_t)L.f8.xmul_count * sizeof(float) : 0), 256);
+  // lookup-kernel K split: partial sums [unit][512 rows][4 tokens] and arrival counters
+  {
+    const int64_t tiles = (d_out + kLutTileRows - 1) / kLutTileRows;
+    int64_t cap = (int64_t)kLutSplitPerSm * sm_count();
+    const int64_t most = (int64_t)L.max_groups * tiles * kLutMaxChunks;
+    if (cap > most) cap = most;
+    L.split_cap = (int)cap;
+  }
+  L.off_lpart = off;
+  off = align_up(off + (size_t)L.split_cap * kLutTileRows * 4 * sizeof(float), 256);
+  L.off_lcnt = off;
+  off = align_up(off + (size_t)(L.split_cap / 2 + 1) * sizeof(int32_t), 256);
   L.total = off;
   return L;
 }
@@ -371,7 +404,9 @@ bd_status apply_impl(const void* w_base, int32_t w_dtype, int64_t d_out, int64_t
     return BD_ERR_CUDA;
   launch_begin(K_TENANT_BUCKET, s);
   k_tenant_bucket<<<1, 1024, bucket_smem, s>>>(tenant_ids, (int)batch, n_tenants, L.max_groups,
-                                               L.max_tc, tenants, kTcMinTokens, d_in, seg,
+                                               L.max_tc, tenants, kTcMinTokens, d_in,
+                                               (d_out + kLutTileRows - 1) / kLutTileRows, L.split_cap,
+                                               reinterpret_cast<int32_t*>(ws + L.off_lcnt), seg,
                                                reinterpret_cast<bd_tenant*>(ws + L.off_tcrec), status);
   launch_end(K_TENANT_BUCKET, s);
   BD_LAUNCH_CHECK();
@@ -405,7 +440,9 @@ bd_status apply_impl(const void* w_base, int32_t w_dtype, int64_t d_out, int64_t
 
   // 4. lookup-table delta over the (lookup group, row tile) space, fused with the combine
   return launch_delta_lut(tc, tenants, scale_dtype == BD_F16, seg, L.max_groups, L.max_tc, x, y_part,
-                          L.ksplit, d_out, d_in, batch, y, y_dtype == BD_BF16, status, s);
+                          L.ksplit, d_out, d_in, batch, y, y_dtype == BD_BF16,
+                          reinterpret_cast<float*>(ws + L.off_lpart), reinterpret_cast<int32_t*>(ws + L.off_lcnt),
+                          L.split_cap, status, s);
 }
 
 }  // namespace bd

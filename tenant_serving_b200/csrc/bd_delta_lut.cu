@@ -12,10 +12,14 @@
 // the tenant's bits.
 //
 // Organisation: persistent, one CTA per SM, 9 warps.
-//   Work: the (lookup group, 512-row tile) units are split over the CTAs by a cost model
-//     (a group of NT tokens costs about what its table reads cost); a CTA walks its share
-//     in pieces of <= DL_PMAX consecutive tiles of one group. Producer and consumers walk
-//     the same sequence, so no per-stage descriptor is exchanged.
+//   Work: (lookup group, K chunk, 512-row tile) units, split over the CTAs by a cost model
+//     (a group of NT tokens costs about what its table reads cost, times the windows of a
+//     chunk); a CTA walks its share in pieces of <= DL_PMAX consecutive tiles of one group
+//     and chunk and hands each to the consumers through a small descriptor ring. A unit
+//     covers all of d_in, or one of kc K chunks when the call has too few (group, tile)
+//     units to fill the SMs.
+//   K chunks: each chunk of a tile leaves its 512 x 4 running sums in the workspace; the
+//     CTA that completes a tile adds them in chunk order and writes y.
 //   warp 8, producer: for every (window, tile) of a piece fills one stage of a ring with
 //     the tile's 16 KB of sign words (one bulk copy from the tiled serving layout, or 512
 //     row copies of 32 bytes from the row-major layout) and its group-128 scales; per
@@ -42,7 +46,7 @@ namespace bd {
 #endif
 constexpr int DL_CWARPS = BD_LUT_CWARPS;            // consumer warps (8 or 16)
 constexpr int DL_THREADS = (DL_CWARPS + 1) * 32;    // + the producer warp
-constexpr int DL_ROWS = 512;                        // rows per tile
+constexpr int DL_ROWS = kLutTileRows;               // rows per tile (512)
 constexpr int DL_RPL = DL_ROWS / (32 * DL_CWARPS);  // rows of a tile per consumer lane
 constexpr int DL_NIB = 16 / DL_CWARPS;              // table high nibbles built per warp
 // tensor memory of a consumer warp: its lane quadrant (warp % 4) and a block of columns;
@@ -50,7 +54,7 @@ constexpr int DL_NIB = 16 / DL_CWARPS;              // table high nibbles built 
 constexpr uint32_t DL_TBLK = 512u / (DL_CWARPS / 4);
 constexpr uint32_t DL_TSTRIDE = 4u * DL_RPL;
 static_assert(DL_CWARPS == 8 || DL_CWARPS == 16, "8 or 16 consumer warps");
-constexpr int DL_W = 256;                           // columns per window (32 chunks)
+constexpr int DL_W = kLutWindow;                    // columns per window (256: 32 chunks)
 constexpr int DL_PMAX = 32;                         // tiles per piece (DL_TSTRIDE TMEM columns each)
 static_assert(DL_PMAX * 4 * DL_RPL <= (int)(512u / (DL_CWARPS / 4)), "running sums fit the warp's columns");
 constexpr int DL_MAX_STAGES = 4;
@@ -80,9 +84,9 @@ constexpr int SK_GLOBAL = 1;   // group scales loaded from global memory per wor
 constexpr int SK_NONE = 2;     // row / tensor (applied at the end) or column (folded into x)
 
 // Work weight of one (group, tile) unit of class k (groups of 4, 3, 2, 1 tokens, then
-// base-only groups): its time relative to a one-token unit, fitted to per-CTA busy time
-// measured on B200 over the four fused Llama-3-8B calls (4 tokens 1.7-2.2, 3 tokens
-// 1.5-2.0, 2 tokens 1.15-1.25; a base-only unit only writes y).
+// base-only groups) over all of d_in: its time relative to a one-token unit, fitted to
+// per-CTA busy time measured on B200 over the four fused Llama-3-8B calls (4 tokens
+// 1.7-2.2, 3 tokens 1.5-2.0, 2 tokens 1.15-1.25; a base-only unit only writes y).
 __host__ __device__ constexpr int lut_class_weight(int k) {
   return k == 0 ? 19 : (k == 1 ? 17 : (k == 2 ? 12 : (k == 3 ? 10 : 1)));
 }
@@ -214,17 +218,34 @@ __device__ __forceinline__ float ldg_scale(const void* s, bool f16, int64_t i) {
 struct DlPiece {
   bd_tenant T;
   int item, tile0, P, nt, u, skind, ssrc, lg;
+  int w0, w1, chunk, kc;  // windows [w0, w1) = K chunk `chunk` of kc
   int tok[4];
 };
 
+// Units of class k: (group, K chunk, tile), tile fastest. Tenant classes are cut into
+// kc K chunks of wpc windows each (kc from the plan); base-only groups are not cut. With
+// kc > 1 a unit weighs its class weight times the windows it covers (base-only: times all
+// of them); with kc = 1 the class weights alone (the CTA boundaries then fall where the
+// weights were fitted, which measured best).
 struct DlWalk {
   int64_t r0, r1, Ck, j, j1, cbase;
-  int k, Sk, sbase, wk, tiles;
+  int k, Sk, sbase, wk, tiles, kc, wpc, nwin, ukc;
 };
 
-__device__ __forceinline__ void walk_init(DlWalk& w, const int32_t* seg_base, int tiles) {
+__device__ __forceinline__ int dl_unit_weight(int k, int wpc, int nwin) {
+  return wpc == nwin ? lut_class_weight(k) : lut_class_weight(k) * (k < kLutClasses - 1 ? wpc : nwin);
+}
+
+// split: the launch may cut units into K chunks (else every unit covers all of d_in)
+__device__ __forceinline__ void walk_init(DlWalk& w, const int32_t* seg_base, int tiles, int nwin, bool split) {
+  int kc = split ? seg_base[2 + kLutClasses] : 1;
+  if (kc < 1 || kc > kLutMaxChunks || nwin % kc != 0) kc = 1;  // (the planner only writes valid values)
+  w.kc = kc;
+  w.nwin = nwin;
+  w.wpc = nwin / kc;
   int64_t W = 0;
-  for (int k = 0; k < kLutClasses; ++k) W += (int64_t)seg_base[2 + k] * tiles * lut_class_weight(k);
+  for (int k = 0; k < kLutClasses; ++k)
+    W += (int64_t)seg_base[2 + k] * tiles * (k < kLutClasses - 1 ? kc : 1) * dl_unit_weight(k, w.wpc, nwin);
   w.r0 = W * (int64_t)blockIdx.x / gridDim.x;
   w.r1 = W * ((int64_t)blockIdx.x + 1) / gridDim.x;
   w.Ck = 0;
@@ -234,11 +255,12 @@ __device__ __forceinline__ void walk_init(DlWalk& w, const int32_t* seg_base, in
   w.cbase = 0;
   w.sbase = 0;
   w.wk = 1;
+  w.ukc = 1;
   w.tiles = tiles;
 }
 
-// Next piece of this CTA's share; false when there is none. Deterministic: the producer
-// and every consumer thread get the same sequence. *bad is set for an invalid record.
+// Next piece of this CTA's share; false when there is none. Deterministic: every lane of
+// the producer warp gets the same sequence. *bad is set for an invalid record.
 __device__ __forceinline__ bool walk_next(DlWalk& w, const int32_t* __restrict__ seg_base, const int32_t* __restrict__ grp_tenant,
                           const int32_t* __restrict__ grp_start, const int32_t* __restrict__ grp_len,
                           const int32_t* __restrict__ perm, const bd_tenant* __restrict__ tenants,
@@ -246,8 +268,9 @@ __device__ __forceinline__ bool walk_next(DlWalk& w, const int32_t* __restrict__
   while (w.j >= w.j1) {
     if (++w.k >= kLutClasses) return false;
     const int nk = seg_base[2 + w.k];
-    w.wk = lut_class_weight(w.k);
-    const int64_t Ck1 = w.Ck + (int64_t)nk * w.tiles * w.wk;
+    w.wk = dl_unit_weight(w.k, w.wpc, w.nwin);
+    w.ukc = w.k < kLutClasses - 1 ? w.kc : 1;
+    const int64_t Ck1 = w.Ck + (int64_t)nk * w.ukc * w.tiles * w.wk;
     const int64_t lo = w.r0 > w.Ck ? w.r0 : w.Ck, hi = w.r1 < Ck1 ? w.r1 : Ck1;
     w.cbase = w.Ck;
     w.sbase = w.Sk;
@@ -261,8 +284,14 @@ __device__ __forceinline__ bool walk_next(DlWalk& w, const int32_t* __restrict__
       w.j = w.j1 = 0;
     }
   }
-  pc.item = w.sbase + (int)(w.j / w.tiles);
-  pc.tile0 = (int)(w.j % w.tiles);
+  const int64_t per_item = (int64_t)w.ukc * w.tiles;
+  pc.item = w.sbase + (int)(w.j / per_item);
+  const int64_t rem = w.j % per_item;
+  pc.chunk = (int)(rem / w.tiles);
+  pc.kc = w.ukc;
+  pc.tile0 = (int)(rem % w.tiles);
+  pc.w0 = w.ukc > 1 ? pc.chunk * w.wpc : 0;
+  pc.w1 = w.ukc > 1 ? pc.w0 + w.wpc : w.nwin;
   int P = w.tiles - pc.tile0;
   if (P > DL_PMAX) P = DL_PMAX;
   if ((int64_t)P > w.j1 - w.j) P = (int)(w.j1 - w.j);
@@ -271,7 +300,7 @@ __device__ __forceinline__ bool walk_next(DlWalk& w, const int32_t* __restrict__
   pc.nt = grp_len[pc.item];
   const int gs = grp_start[pc.item];
 #pragma unroll
-  for (int q = 0; q < 4; ++q) pc.tok[q] = q < pc.nt ? perm[gs + q] : 0;
+  for (int t = 0; t < 4; ++t) pc.tok[t] = t < pc.nt ? perm[gs + t] : 0;
   pc.u = grp_tenant[pc.item];
   *bad = false;
   if (pc.u >= 0) {
@@ -460,7 +489,19 @@ struct DlDesc {
   int32_t tok[4];
 };
 static_assert(sizeof(DlDesc) == 64, "descriptor slot size");
+// K-chunk part of a piece's descriptor (only kernels launched with K chunks use it)
+struct DlSplit {
+  int32_t w0, w1, item, kc;  // windows [w0, w1); lookup group; K chunks of its units
+  int32_t chunk, pad[3];
+};
+static_assert(sizeof(DlSplit) == 32, "split slot size");
+
 constexpr int DL_DSLOTS = 4;
+// the fixed region after the x slots: descriptors, split slots, barriers, three words
+static_assert(DL_DSLOTS * (sizeof(DlDesc) + sizeof(DlSplit)) +
+                      (2 * DL_MAX_STAGES + 2 * DL_XSLOTS + 2 * DL_DSLOTS + 4) * sizeof(uint64_t) + 12 <=
+                  dl_fixed_bytes(true) - DL_XSLOTS * dl_xslot_bytes(true),
+              "fixed shared-memory region");
 
 // One row-window of a stage: its sign words, their scales, the lookups into part[0..3].
 __device__ __forceinline__ void dl_row_window(const DlDesc& D, uint32_t st, int r_in, int tile, int win, int nt,
@@ -519,6 +560,87 @@ __device__ __forceinline__ void dl_row_window(const DlDesc& D, uint32_t st, int 
   }
 }
 
+// End of a piece whose units are K chunks (Q.kc > 1). Every consumer lane stores the
+// running sums of its rows (4 tokens, unscaled) into the unit's slot
+// lut_part[((item * tiles + tile) * kc + chunk) * 512 + row][4]; after a barrier, lane p of
+// warp 0 counts the arrival at tile p; the CTA that completes a tile's count then reads
+// the kc slots of that tile in chunk order, applies the row / tensor scale, adds the base
+// partial sums and writes y. Warp-uniform; false when a bounded barrier gave up.
+__device__ __noinline__ bool dl_split_epilogue(const DlDesc& D, const DlSplit& Q, int P, int tiles, uint32_t t_lane,
+                                               int r_lo, int lane,
+                                               int warp, float* __restrict__ lut_part, int32_t* __restrict__ lut_cnt,
+                                               int split_cap, const float* __restrict__ y_part, int ksplit, int batch,
+                                               int64_t d_out, float rs, bool scale_f16, void* __restrict__ y,
+                                               bool y_bf16, uint64_t* bars, uint32_t parity,
+                                               volatile uint32_t* last_mask, const volatile int* abort_flag,
+                                               uint32_t* __restrict__ status) {
+  constexpr int PT = 32 / DL_TSTRIDE;
+  const int kc = Q.kc, nt = D.nt;
+  const int64_t unit0 = (int64_t)Q.item * tiles + D.tile0;  // (group, tile) of the piece's first tile
+  const bool fits = (unit0 + P) * kc <= (int64_t)split_cap;  // guaranteed by the planner
+  if (!fits && lane == 0 && warp == 0) atomicOr(status, BD_DEV_INTERNAL);
+  for (int p0 = 0; p0 < P; p0 += PT) {
+    uint32_t acc[32];
+    tmem_ld32(t_lane + DL_TSTRIDE * (uint32_t)p0, acc);
+#pragma unroll
+    for (int pp = 0; pp < PT; ++pp)
+#pragma unroll
+      for (int h = 0; h < DL_RPL; ++h) {
+        if (p0 + pp >= P || !fits) continue;
+        const int r_in = r_lo + 32 * DL_CWARPS * h;
+        const int64_t slot = (unit0 + p0 + pp) * kc + Q.chunk;
+        const int b = DL_TSTRIDE * pp + 4 * h;
+        __stcg(reinterpret_cast<float4*>(lut_part + (slot * DL_ROWS + r_in) * 4),
+               make_float4(__uint_as_float(acc[b]), __uint_as_float(acc[b + 1]), __uint_as_float(acc[b + 2]),
+                           __uint_as_float(acc[b + 3])));
+      }
+  }
+  __threadfence();  // the slot is visible device-wide before this CTA's arrival is counted
+  if (!consumer_sync(&bars[0], parity, abort_flag)) return false;
+  if (warp == 0) {
+    bool last = false;
+    if (lane < P && fits) last = atomicAdd(&lut_cnt[unit0 + lane], 1) == kc - 1;
+    const uint32_t m = __ballot_sync(0xffffffffu, last);
+    if (lane == 0) *last_mask = m;
+  }
+  if (!consumer_sync(&bars[1], parity, abort_flag)) return false;
+  const uint32_t m = *last_mask;
+  if (m == 0) return true;
+  __threadfence();  // the other chunks' slots are read after their arrivals were seen
+  const int mode = D.mode;
+  for (int p = 0; p < P; ++p) {
+    if (!((m >> p) & 1u)) continue;
+#pragma unroll
+    for (int h = 0; h < DL_RPL; ++h) {
+      const int r_in = r_lo + 32 * DL_CWARPS * h;
+      const int64_t row = (int64_t)(D.tile0 + p) * DL_ROWS + r_in;
+      if (row >= d_out) continue;
+      float d[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int c = 0; c < kc; ++c) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(lut_part + (((unit0 + p) * kc + c) * DL_ROWS + r_in) * 4));
+        d[0] += v.x;
+        d[1] += v.y;
+        d[2] += v.z;
+        d[3] += v.w;
+      }
+      const float s_row = mode == BD_SCALE_ROW ? ldg_scale(D.scales, scale_f16, row) : rs;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (q >= nt) continue;
+        const int64_t t = D.tok[q];
+        float v = 0.f;
+        for (int kz = 0; kz < ksplit; ++kz) v += y_part[((int64_t)kz * batch + t) * d_out + row];
+        v += s_row * d[q];
+        if (y_bf16)
+          reinterpret_cast<uint16_t*>(y)[t * d_out + row] = (uint16_t)f2bf_bits(v);
+        else
+          reinterpret_cast<float*>(y)[t * d_out + row] = v;
+      }
+    }
+  }
+  return true;
+}
+
 // ------------------------------------------------------------------------------------
 // the kernel
 // ------------------------------------------------------------------------------------
@@ -535,11 +657,14 @@ struct DlRing {
   }
 };
 
-template <bool XBF16>
+// SPLIT: the planner may have cut units into K chunks (the launch has too few units for
+// the SMs otherwise); without it the kernel keeps the plain whole-d_in code paths.
+template <bool XBF16, bool SPLIT>
 __global__ void __launch_bounds__(DL_THREADS, 1) k_delta_lut(
     const bd_tenant* __restrict__ tenants, bool scale_f16, const int32_t* __restrict__ seg_base,
     int max_groups, int max_tc, const void* __restrict__ x, const float* __restrict__ y_part,
     int ksplit, int64_t d_out, int64_t d_in, int batch, void* __restrict__ y, bool y_bf16,
+    float* __restrict__ lut_part, int32_t* __restrict__ lut_cnt, int split_cap,
     uint32_t* __restrict__ status) {
   extern __shared__ __align__(16) uint8_t dl_smem_raw[];
   const uint32_t raw = smem_u32(dl_smem_raw);
@@ -552,15 +677,18 @@ __global__ void __launch_bounds__(DL_THREADS, 1) k_delta_lut(
   uint8_t* gen = dl_smem_raw - raw;  // generic pointer of shared address 0
   const uint32_t xslot0 = L.fixed;
   DlDesc* desc = reinterpret_cast<DlDesc*>(gen + L.fixed + DL_XSLOTS * XSLOT);
-  uint64_t* full = reinterpret_cast<uint64_t*>(desc + DL_DSLOTS);
+  DlSplit* dsplit = reinterpret_cast<DlSplit*>(desc + DL_DSLOTS);
+  uint64_t* full = reinterpret_cast<uint64_t*>(dsplit + DL_DSLOTS);
   uint64_t* empty = full + DL_MAX_STAGES;
   uint64_t* xfull = empty + DL_MAX_STAGES;
   uint64_t* xempty = xfull + DL_XSLOTS;
   uint64_t* dfull = xempty + DL_XSLOTS;
   uint64_t* dempty = dfull + DL_DSLOTS;
-  uint64_t* cbar = dempty + DL_DSLOTS;  // [2]: consumers before / after a table build
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cbar + 2);
+  // [4]: consumers before / after a table build; around the arrival counts of split units
+  uint64_t* cbar = dempty + DL_DSLOTS;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cbar + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile uint32_t* last_mask = reinterpret_cast<volatile uint32_t*>(tmem_slot + 2);
   const int NS = L.stages;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -577,7 +705,7 @@ __global__ void __launch_bounds__(DL_THREADS, 1) k_delta_lut(
       mbar_init(&dfull[i], 1);
       mbar_init(&dempty[i], DL_CWARPS);
     }
-    for (int i = 0; i < 2; ++i) mbar_init(&cbar[i], DL_CWARPS);
+    for (int i = 0; i < 4; ++i) mbar_init(&cbar[i], DL_CWARPS);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -599,7 +727,7 @@ __global__ void __launch_bounds__(DL_THREADS, 1) k_delta_lut(
     const int32_t* grp_len = grp_start + max_groups;
     const int32_t* perm = grp_len + max_groups + 4 * max_tc;
     DlWalk walk;
-    walk_init(walk, seg_base, tiles);
+    walk_init(walk, seg_base, tiles, nwin, SPLIT);
     DlPiece pc;
     bool bad = false;
     const int xb = XBF16 ? 2 : 4;
@@ -635,6 +763,14 @@ __global__ void __launch_bounds__(DL_THREADS, 1) k_delta_lut(
           D.skind = pc.skind;
           D.ssrc = pc.ssrc;
           D.lg = pc.lg;
+          if (SPLIT) {
+            DlSplit& Q = dsplit[Dr.slot];
+            Q.w0 = pc.w0;
+            Q.w1 = pc.w1;
+            Q.item = pc.item;
+            Q.kc = pc.kc;
+            Q.chunk = pc.chunk;
+          }
 #pragma unroll
           for (int q = 0; q < 4; ++q) D.tok[q] = pc.tok[q];
         }
@@ -646,7 +782,8 @@ __global__ void __launch_bounds__(DL_THREADS, 1) k_delta_lut(
       if (pc.u < 0) continue;  // base-only piece: the consumers write it without stages
       const bd_tenant& T = pc.T;
       const bool tiled = T.layout == BD_LAYOUT_TILED;
-      for (int win = 0; win < nwin && !stop; ++win) {
+      const int wbeg = SPLIT ? pc.w0 : 0, wend = SPLIT ? pc.w1 : nwin;
+      for (int win = wbeg; win < wend && !stop; ++win) {
         // ---- x slices (and column scales) of this window
         const int64_t col0 = (int64_t)win * DL_W;
         const int ncols = (int)((d_in - col0) < DL_W ? (d_in - col0) : DL_W);
@@ -743,6 +880,7 @@ __global__ void __launch_bounds__(DL_THREADS, 1) k_delta_lut(
     const uint32_t t_lane = tmem_base + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(warp >> 2) * DL_TBLK;
     const int r_lo = warp * 32 + lane;  // rows r_lo + 32 * DL_CWARPS * h of each tile, h < DL_RPL
     DlRing S, X, Dr;
+    int nsplit = 0;  // split pieces finished (phase of the two epilogue barriers)
     for (;;) {
       if (!__all_sync(0xffffffffu, mbar_wait(&dfull[Dr.slot], Dr.phase, abort_flag))) {
         if (lane == 0) *abort_flag = 1;
@@ -759,7 +897,8 @@ __global__ void __launch_bounds__(DL_THREADS, 1) k_delta_lut(
           dl_lane_consts(lane, L.tbase, single, K, sel);
           k_single = (int)single;
         }
-        for (int win = 0; win < nwin && !dead; ++win) {
+        const int wbeg = SPLIT ? dsplit[Dr.slot].w0 : 0, wend = SPLIT ? dsplit[Dr.slot].w1 : nwin;
+        for (int win = wbeg; win < wend && !dead; ++win) {
           // new window: wait for its x, rebuild the tables once every warp is done with
           // the previous window's lookups
           const bool xok = __all_sync(0xffffffffu, mbar_wait(&xfull[X.slot], X.phase, abort_flag));
@@ -787,7 +926,7 @@ __global__ void __launch_bounds__(DL_THREADS, 1) k_delta_lut(
 #pragma unroll
             for (int q = 0; q < 4 * DL_RPL; ++q) part[q] = 0.f;
             const uint32_t tcol = t_lane + DL_TSTRIDE * (uint32_t)p;
-            if (win > 0) {
+            if (win > wbeg) {
               // running sums of this tile from the previous windows
               tmem_wait_st();
               tmem_ld_tile(tcol, part);
@@ -817,56 +956,70 @@ __global__ void __launch_bounds__(DL_THREADS, 1) k_delta_lut(
       float rs = 1.f;
       if (!base_only && mode == BD_SCALE_TENSOR) rs = ldg_scale(scales, scale_f16, 0);
       constexpr int PT = 32 / DL_TSTRIDE;  // tiles per 32-column read
-      for (int p0 = 0; p0 < P; p0 += PT) {
-        uint32_t acc[32];  // tile p0 + pp, row h, token q at DL_TSTRIDE * pp + 4 h + q
-        if (!base_only) {
-          tmem_ld32(t_lane + DL_TSTRIDE * (uint32_t)p0, acc);
-        } else {
-#pragma unroll
-          for (int q = 0; q < 32; ++q) acc[q] = 0u;
+      const bool split = SPLIT && !base_only && dsplit[Dr.slot].kc > 1;
+      if (split) {
+        // ---- a K chunk of split units: its running sums go to the unit's partial slot;
+        // the last chunk to arrive at a tile adds all chunks in chunk order (the result
+        // does not depend on which CTA arrives last) and writes y
+        if (!dl_split_epilogue(D, dsplit[Dr.slot], P, tiles, t_lane, r_lo, lane, warp, lut_part, lut_cnt, split_cap, y_part, ksplit,
+                               batch, d_out, rs, scale_f16, y, y_bf16, &cbar[2], (uint32_t)(nsplit & 1), last_mask,
+                               abort_flag, status)) {
+          if (lane == 0) *abort_flag = 1;
+          break;
         }
-        float bsum[PT][DL_RPL][4];
-#pragma unroll
-        for (int pp = 0; pp < PT; ++pp)
-#pragma unroll
-          for (int h = 0; h < DL_RPL; ++h)
-#pragma unroll
-            for (int q = 0; q < 4; ++q) bsum[pp][h][q] = 0.f;
-        for (int kz = 0; kz < ksplit; ++kz) {
-          const float* part = y_part + (int64_t)kz * batch * d_out;
-#pragma unroll
+        ++nsplit;
+      } else {
+        for (int p0 = 0; p0 < P; p0 += PT) {
+          uint32_t acc[32];  // tile p0 + pp, row h, token q at DL_TSTRIDE * pp + 4 h + q
+          if (!base_only) {
+            tmem_ld32(t_lane + DL_TSTRIDE * (uint32_t)p0, acc);
+          } else {
+  #pragma unroll
+            for (int q = 0; q < 32; ++q) acc[q] = 0u;
+          }
+          float bsum[PT][DL_RPL][4];
+  #pragma unroll
           for (int pp = 0; pp < PT; ++pp)
-#pragma unroll
+  #pragma unroll
+            for (int h = 0; h < DL_RPL; ++h)
+  #pragma unroll
+              for (int q = 0; q < 4; ++q) bsum[pp][h][q] = 0.f;
+          for (int kz = 0; kz < ksplit; ++kz) {
+            const float* part = y_part + (int64_t)kz * batch * d_out;
+  #pragma unroll
+            for (int pp = 0; pp < PT; ++pp)
+  #pragma unroll
+              for (int h = 0; h < DL_RPL; ++h) {
+                const int64_t row = (int64_t)(tile0 + p0 + pp) * DL_ROWS + r_lo + 32 * DL_CWARPS * h;
+                if (p0 + pp < P && row < d_out) {
+  #pragma unroll
+                  for (int q = 0; q < 4; ++q)
+                    if (q < nt) bsum[pp][h][q] += part[(int64_t)D.tok[q] * d_out + row];
+                }
+              }
+          }
+  #pragma unroll
+          for (int pp = 0; pp < PT; ++pp)
+  #pragma unroll
             for (int h = 0; h < DL_RPL; ++h) {
               const int64_t row = (int64_t)(tile0 + p0 + pp) * DL_ROWS + r_lo + 32 * DL_CWARPS * h;
-              if (p0 + pp < P && row < d_out) {
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                  if (q < nt) bsum[pp][h][q] += part[(int64_t)D.tok[q] * d_out + row];
+              if (p0 + pp >= P || row >= d_out) continue;
+              float s_row = rs;
+              if (!base_only && mode == BD_SCALE_ROW) s_row = ldg_scale(scales, scale_f16, row);
+  #pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                if (q < nt) {
+                  const float v =
+                      bsum[pp][h][q] + (base_only ? 0.f : s_row * __uint_as_float(acc[DL_TSTRIDE * pp + 4 * h + q]));
+                  const int64_t t = D.tok[q];
+                  if (y_bf16)
+                    reinterpret_cast<uint16_t*>(y)[t * d_out + row] = (uint16_t)f2bf_bits(v);
+                  else
+                    reinterpret_cast<float*>(y)[t * d_out + row] = v;
+                }
               }
             }
         }
-#pragma unroll
-        for (int pp = 0; pp < PT; ++pp)
-#pragma unroll
-          for (int h = 0; h < DL_RPL; ++h) {
-            const int64_t row = (int64_t)(tile0 + p0 + pp) * DL_ROWS + r_lo + 32 * DL_CWARPS * h;
-            if (p0 + pp >= P || row >= d_out) continue;
-            float s_row = rs;
-            if (!base_only && mode == BD_SCALE_ROW) s_row = ldg_scale(scales, scale_f16, row);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              if (q < nt) {
-                const float v =
-                    bsum[pp][h][q] + (base_only ? 0.f : s_row * __uint_as_float(acc[DL_TSTRIDE * pp + 4 * h + q]));
-                const int64_t t = D.tok[q];
-                if (y_bf16)
-                  reinterpret_cast<uint16_t*>(y)[t * d_out + row] = (uint16_t)f2bf_bits(v);
-                else
-                  reinterpret_cast<float*>(y)[t * d_out + row] = v;
-              }
-            }
-          }
       }
       // the descriptor is no longer read
       __syncwarp();
@@ -890,16 +1043,16 @@ __global__ void __launch_bounds__(DL_THREADS, 1) k_delta_lut(
 // The kernel's layout needs its dynamic window to start low enough that the tables (on a
 // 64 KB boundary) and at least two ring stages fit: checked once per device from the
 // kernel's static shared memory and the device's reserved shared memory per block.
-static bool dl_layout_fits(const void* fn, bool xbf16) {
-  static std::atomic<uint64_t> ok_bits[2], bad_bits[2];
+static bool dl_layout_fits(const void* fn, bool xbf16, int v) {
+  static std::atomic<uint64_t> ok_bits[4], bad_bits[4];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) {
     (void)cudaGetLastError();
     return false;
   }
   const uint64_t bit = dev < 64 ? (1ull << dev) : 0ull;
-  if (bit && (ok_bits[xbf16].load() & bit)) return true;
-  if (bit && (bad_bits[xbf16].load() & bit)) return false;
+  if (bit && (ok_bits[v].load() & bit)) return true;
+  if (bit && (bad_bits[v].load() & bit)) return false;
   cudaFuncAttributes fa;
   int reserved = 0;
   if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess ||
@@ -909,22 +1062,29 @@ static bool dl_layout_fits(const void* fn, bool xbf16) {
   }
   const uint32_t start = (uint32_t)reserved + (uint32_t)fa.sharedSizeBytes;
   const bool fits = dl_layout(start, DL_SMEM, xbf16).stages >= 2;
-  if (bit) (fits ? ok_bits[xbf16] : bad_bits[xbf16]).fetch_or(bit);
+  if (bit) (fits ? ok_bits[v] : bad_bits[v]).fetch_or(bit);
   return fits;
 }
 
 bd_status launch_delta_lut(bool xbf16, const bd_tenant* tenants, bool scale_f16, const int32_t* seg,
                            int max_groups, int max_tc, const void* x, const float* y_part, int ksplit,
                            int64_t d_out, int64_t d_in, int64_t batch, void* y, bool y_bf16,
-                           uint32_t* status, cudaStream_t s) {
-  auto kfn = xbf16 ? k_delta_lut<true> : k_delta_lut<false>;
-  static std::atomic<uint64_t> attr[2];
-  if (!ensure_dyn_smem(kfn, DL_SMEM, attr[xbf16 ? 1 : 0])) return BD_ERR_CUDA;
-  if (!dl_layout_fits(reinterpret_cast<const void*>(kfn), xbf16)) return BD_ERR_INTERNAL;
+                           float* lut_part, int32_t* lut_cnt, int split_cap, uint32_t* status,
+                           cudaStream_t s) {
+  // the K-chunk variant only when the planner can choose kc >= 2: at most max_groups tenant
+  // groups of ceil(d_out / 512) tiles, cut in two, within the partial-sum budget
+  const int64_t tiles = (d_out + DL_ROWS - 1) / DL_ROWS, nwin = (d_in + DL_W - 1) / DL_W;
+  const bool split = nwin >= 4 && (int64_t)max_groups * tiles * 2 <= (int64_t)split_cap;
+  auto kfn = xbf16 ? (split ? k_delta_lut<true, true> : k_delta_lut<true, false>)
+                   : (split ? k_delta_lut<false, true> : k_delta_lut<false, false>);
+  const int v = (xbf16 ? 1 : 0) + (split ? 2 : 0);
+  static std::atomic<uint64_t> attr[4];
+  if (!ensure_dyn_smem(kfn, DL_SMEM, attr[v])) return BD_ERR_CUDA;
+  if (!dl_layout_fits(reinterpret_cast<const void*>(kfn), xbf16, v)) return BD_ERR_INTERNAL;
   launch_begin(K_DELTA_LUT, s);
   kfn<<<(unsigned)sm_count(), DL_THREADS, DL_SMEM, s>>>(tenants, scale_f16, seg, max_groups, max_tc, x,
                                                        y_part, ksplit, d_out, d_in, (int)batch, y, y_bf16,
-                                                       status);
+                                                       lut_part, lut_cnt, split_cap, status);
   launch_end(K_DELTA_LUT, s);
   BD_LAUNCH_CHECK();
   return BD_OK;

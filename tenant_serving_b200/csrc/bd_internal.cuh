@@ -21,10 +21,18 @@ constexpr int kTcSegTokens = 64;
 
 // Plan written by the tenant-bucket kernel into the apply workspace (int32 words):
 // [0] lookup groups, [1] tensor-core segments, [2..6] lookup groups per class (NT = 4, 3,
-// 2, 1 tokens of a tenant, then base-only groups), [7] unused; then the arrays.
+// 2, 1 tokens of a tenant, then base-only groups), [7] K chunks of the lookup kernel's
+// tenant units (1: every unit covers all of d_in); then the arrays.
 constexpr int kSegHeader = 8;
 constexpr int kLutTokens = 4;   // tokens of one tenant served by one pass of the lookup kernel
 constexpr int kLutClasses = 5;
+constexpr int kLutTileRows = 512;   // rows of one lookup-kernel tile (and of the serving layout)
+constexpr int kLutWindow = 256;     // columns of one lookup-kernel window
+constexpr int kLutMaxChunks = 8;    // most K chunks a lookup unit is cut into
+// Split budget: the planner cuts the lookup kernel's tenant units into K chunks only while
+// (units x chunks) stays within this many per SM; each such chunk keeps a 512-row x
+// 4-token fp32 partial sum in the workspace.
+constexpr int kLutSplitPerSm = 16;
 
 enum KernelKind : int32_t {
   K_DELTA_STATS = 0,     // fused delta + whole-matrix shifted sums for the clip
