@@ -197,6 +197,8 @@ __global__ void __launch_bounds__(256) k_delta_stats(const uint4* __restrict__ w
                                                      unsigned int* __restrict__ counter,
                                                      ClipParams* __restrict__ clip_out,
                                                      double* __restrict__ stats_out) {
+  pdl_wait();  // inputs may come from the previous kernel on the stream
+  pdl_trigger();
   using V = Vec<BF16>;
   // shift: delta of element 0 (every thread computes the same value); sums of the
   // shifted deltas are accumulated in fp64 per element
@@ -252,6 +254,8 @@ __global__ void __launch_bounds__(256, 4) k_scale_signpack(
     const uint8_t* __restrict__ wb, const uint8_t* __restrict__ wf, int64_t d_out, int d_in,
     int lg, int seg_chunks, int nseg, const ClipParams* __restrict__ clipp,
     uint32_t* __restrict__ signs, float* __restrict__ scales, double* __restrict__ partials) {
+  pdl_wait();  // inputs may come from the previous kernel on the stream
+  pdl_trigger();
   using V = Vec<BF16>;
   constexpr int VEC = V::N;
   constexpr int CHUNK = 32 * VEC;             // columns per chunk
@@ -345,6 +349,8 @@ __global__ void __launch_bounds__(256) k_col_scale_signpack(
     const uint8_t* __restrict__ wb, const uint8_t* __restrict__ wf, int64_t d_out, int64_t d_in,
     int tile_rows, int64_t nchunks, const ClipParams* __restrict__ clipp,
     uint32_t* __restrict__ signs, double* __restrict__ colpart) {
+  pdl_wait();  // inputs may come from the previous kernel on the stream
+  pdl_trigger();
   using V = Vec<BF16>;
   constexpr int VEC = V::N;
   constexpr int CHUNK = 32 * VEC;
@@ -412,6 +418,8 @@ __global__ void __launch_bounds__(256) k_col_scale_signpack(
 // ROW: scales[r] = sum_s partials[r][s] / d_in (one thread per row)
 __global__ void k_row_final(const double* __restrict__ partials, int nseg, int64_t d_out,
                             int64_t d_in, float* __restrict__ scales) {
+  pdl_wait();  // inputs may come from the previous kernel on the stream
+  pdl_trigger();
   const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (r >= d_out) return;
   double s = 0.0;
@@ -422,6 +430,8 @@ __global__ void k_row_final(const double* __restrict__ partials, int nseg, int64
 // COL: scales[i] = sum_t colpart[t][i] / d_out (one thread per column)
 __global__ void k_col_final(const double* __restrict__ colpart, int64_t ntile, int64_t d_out,
                             int64_t d_in, float* __restrict__ scales) {
+  pdl_wait();  // inputs may come from the previous kernel on the stream
+  pdl_trigger();
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= d_in) return;
   double s = 0.0;
@@ -433,6 +443,8 @@ __global__ void k_col_final(const double* __restrict__ colpart, int64_t ntile, i
 // is over G entries, so this is the mean over the block's entries); fp64, row order
 __global__ void k_block_final(const float* __restrict__ rowmean, int64_t d_out, int64_t ngc, int G,
                               float* __restrict__ scales) {
+  pdl_wait();  // inputs may come from the previous kernel on the stream
+  pdl_trigger();
   const int64_t nrb = (d_out + G - 1) / G;
   const int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (k >= nrb * ngc) return;
@@ -446,6 +458,8 @@ __global__ void k_block_final(const float* __restrict__ rowmean, int64_t d_out, 
 // TENSOR: one block; strided per-thread sums then a fixed tree
 __global__ void k_tensor_final(const double* __restrict__ partials, int64_t n, double count,
                                float* __restrict__ scales) {
+  pdl_wait();  // inputs may come from the previous kernel on the stream
+  pdl_trigger();
   __shared__ double sh[256];
   double s = 0.0;
   for (int64_t k = threadIdx.x; k < n; k += blockDim.x) s += partials[k];
@@ -545,9 +559,9 @@ bd_status launch_compress(const CompressPlan& p, const void* w_base, const void*
   }
   if (clip) {
     launch_begin(K_DELTA_STATS, s);
-    k_delta_stats<BF16><<<p.stats_blocks, 256, 0, s>>>((const uint4*)w_base, (const uint4*)w_fine,
-                                                       nvec, d_out * d_in, (double)cfg->clip_k,
-                                                       stat_parts, counter, clipp, stats_out);
+    BD_CUDA_TRY(launch_pdl(k_delta_stats<BF16>, dim3(p.stats_blocks), dim3(256), 0, s, (const uint4*)w_base,
+                           (const uint4*)w_fine, nvec, d_out * d_in, (double)cfg->clip_k, stat_parts, counter,
+                           clipp, stats_out));
     launch_end(K_DELTA_STATS, s);
     BD_LAUNCH_CHECK();
   }
@@ -556,13 +570,14 @@ bd_status launch_compress(const CompressPlan& p, const void* w_base, const void*
     const int64_t tasks = p.ntile * p.nchunks;
     const int64_t blocks = (tasks + 7) / 8;
     launch_begin(K_COL_SCALE_SIGNPACK, s);
-    k_col_scale_signpack<BF16><<<(unsigned)blocks, 256, 0, s>>>(
-        (const uint8_t*)w_base, (const uint8_t*)w_fine, d_out, d_in, p.col_tile, p.nchunks,
-        clipp, signs, part);
+    BD_CUDA_TRY(launch_pdl(k_col_scale_signpack<BF16>, dim3((unsigned)blocks), dim3(256), 0, s,
+                           (const uint8_t*)w_base, (const uint8_t*)w_fine, d_out, d_in, p.col_tile, p.nchunks,
+                           (const ClipParams*)clipp, signs, part));
     launch_end(K_COL_SCALE_SIGNPACK, s);
     BD_LAUNCH_CHECK();
     launch_begin(K_SCALE_FINAL, s);
-    k_col_final<<<(unsigned)((d_in + 255) / 256), 256, 0, s>>>(part, p.ntile, d_out, d_in, scales);
+    BD_CUDA_TRY(launch_pdl(k_col_final, dim3((unsigned)((d_in + 255) / 256)), dim3(256), 0, s, (const double*)part,
+                           p.ntile, d_out, d_in, scales));
     launch_end(K_SCALE_FINAL, s);
     BD_LAUNCH_CHECK();
     return BD_OK;
@@ -575,10 +590,10 @@ bd_status launch_compress(const CompressPlan& p, const void* w_base, const void*
   const int din = (int)d_in;
   // BLOCK: the per-row group means go to the workspace, the block means follow
   float* group_out = cfg->mode == BD_SCALE_BLOCK ? reinterpret_cast<float*>(part) : scales;
-#define BD_SIGNPACK(SEGC, CLIP, GRP)                                                           \
-  k_scale_signpack<BF16, SEGC, CLIP, GRP><<<blocks, 256, 0, s>>>(                              \
-      (const uint8_t*)w_base, (const uint8_t*)w_fine, d_out, din, lg, p.seg_chunks, p.nseg,    \
-      clipp, signs, group_out, part)
+#define BD_SIGNPACK(SEGC, CLIP, GRP)                                                                    \
+  BD_CUDA_TRY(launch_pdl(k_scale_signpack<BF16, SEGC, CLIP, GRP>, dim3(blocks), dim3(256), 0, s,           \
+                         (const uint8_t*)w_base, (const uint8_t*)w_fine, d_out, din, lg, p.seg_chunks,     \
+                         p.nseg, (const ClipParams*)clipp, signs, group_out, part))
   launch_begin(K_SCALE_SIGNPACK, s);
   if (p.seg_chunks >= 4) {
     if (clip) { if (group) BD_SIGNPACK(4, true, true); else BD_SIGNPACK(4, true, false); }
@@ -592,20 +607,21 @@ bd_status launch_compress(const CompressPlan& p, const void* w_base, const void*
   BD_LAUNCH_CHECK();
   if (cfg->mode == BD_SCALE_ROW) {
     launch_begin(K_SCALE_FINAL, s);
-    k_row_final<<<(unsigned)((d_out + 255) / 256), 256, 0, s>>>(part, p.nseg, d_out, d_in, scales);
+    BD_CUDA_TRY(launch_pdl(k_row_final, dim3((unsigned)((d_out + 255) / 256)), dim3(256), 0, s, (const double*)part,
+                           p.nseg, d_out, d_in, scales));
     launch_end(K_SCALE_FINAL, s);
     BD_LAUNCH_CHECK();
   } else if (cfg->mode == BD_SCALE_BLOCK) {
     const int64_t ngc = d_in >> lg, n = ((d_out + cfg->group_size - 1) / cfg->group_size) * ngc;
     launch_begin(K_SCALE_FINAL, s);
-    k_block_final<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(reinterpret_cast<const float*>(part), d_out, ngc,
-                                                              cfg->group_size, scales);
+    BD_CUDA_TRY(launch_pdl(k_block_final, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s,
+                           reinterpret_cast<const float*>(part), d_out, ngc, (int)cfg->group_size, scales));
     launch_end(K_SCALE_FINAL, s);
     BD_LAUNCH_CHECK();
   } else if (cfg->mode == BD_SCALE_TENSOR) {
     launch_begin(K_SCALE_FINAL, s);
-    k_tensor_final<<<1, 256, 0, s>>>(part, d_out * (int64_t)p.nseg, (double)d_out * (double)d_in,
-                                     scales);
+    BD_CUDA_TRY(launch_pdl(k_tensor_final, dim3(1), dim3(256), 0, s, (const double*)part, d_out * (int64_t)p.nseg,
+                           (double)d_out * (double)d_in, scales));
     launch_end(K_SCALE_FINAL, s);
     BD_LAUNCH_CHECK();
   }

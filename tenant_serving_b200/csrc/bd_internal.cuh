@@ -141,6 +141,25 @@ inline bool is_pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
     }                                               \
   } while (0)
 
+// Launch `kernel` on `s` with programmatic stream serialization allowed: its blocks may be
+// scheduled while the previous kernel on the stream drains (the kernel calls pdl_wait()
+// before reading anything).
+template <typename... Params, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Params>(args)...);
+}
+
 #define BD_LAUNCH_CHECK()                           \
   do {                                              \
     cudaError_t _e = cudaGetLastError();            \
@@ -168,6 +187,15 @@ __device__ __forceinline__ double warp_sum_d(double v) {
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
+
+// Programmatic dependent launch (sm_90+). A kernel launched with launch_pdl may start while
+// the previous kernel on its stream is still running; pdl_wait() blocks until that kernel
+// has completed and its writes are visible, so it comes before any read of data another
+// kernel may have produced. pdl_trigger() lets the next kernel on the stream start
+// launching (it still waits for this one in its own pdl_wait). Both are no-ops for a
+// kernel launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   // 16-byte global load that is not kept in L1 (each byte is read once)
