@@ -66,6 +66,8 @@ __global__ void __launch_bounds__(1024) k_tenant_bucket(const int32_t* __restric
                                                         int32_t* __restrict__ seg_base,
                                                         bd_tenant* __restrict__ tc_rec,
                                                         uint32_t* __restrict__ status) {
+  pdl_wait();  // inputs may come from the previous kernel on the stream
+  pdl_trigger();
   extern __shared__ int32_t cnt[];  // n_tenants + 1 counters (last = base only)
   __shared__ int32_t wsum[kPlanQ][32];
   __shared__ int32_t bad;
@@ -236,6 +238,8 @@ __global__ void __launch_bounds__(256) k_base_gemv_f32(const float* __restrict__
                                                        const float* __restrict__ X, int64_t d_out,
                                                        int64_t d_in, int batch,
                                                        float* __restrict__ y_part) {
+  pdl_wait();  // inputs may come from the previous kernel on the stream
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (row >= d_out) return;
@@ -403,11 +407,11 @@ bd_status apply_impl(const void* w_base, int32_t w_dtype, int64_t d_out, int64_t
   if (!ensure_dyn_smem(k_tenant_bucket, (kMaxTenants + 1) * (int)sizeof(int32_t), bucket_attr))
     return BD_ERR_CUDA;
   launch_begin(K_TENANT_BUCKET, s);
-  k_tenant_bucket<<<1, 1024, bucket_smem, s>>>(tenant_ids, (int)batch, n_tenants, L.max_groups,
-                                               L.max_tc, tenants, kTcMinTokens, d_in,
-                                               (d_out + kLutTileRows - 1) / kLutTileRows, L.split_cap,
-                                               reinterpret_cast<int32_t*>(ws + L.off_lcnt), seg,
-                                               reinterpret_cast<bd_tenant*>(ws + L.off_tcrec), status);
+  BD_CUDA_TRY(launch_pdl(k_tenant_bucket, dim3(1), dim3(1024), bucket_smem, s, tenant_ids, (int)batch, n_tenants,
+                         L.max_groups, L.max_tc, tenants, (int)kTcMinTokens, d_in,
+                         (int64_t)((d_out + kLutTileRows - 1) / kLutTileRows), L.split_cap,
+                         reinterpret_cast<int32_t*>(ws + L.off_lcnt), seg,
+                         reinterpret_cast<bd_tenant*>(ws + L.off_tcrec), status));
   launch_end(K_TENANT_BUCKET, s);
   BD_LAUNCH_CHECK();
 
@@ -422,8 +426,8 @@ bd_status apply_impl(const void* w_base, int32_t w_dtype, int64_t d_out, int64_t
   } else {
     const int64_t blocks = (d_out * 32 + 255) / 256;
     launch_begin(K_BASE_GEMV, s);
-    k_base_gemv_f32<<<(unsigned)blocks, 256, 0, s>>>((const float*)w_base, (const float*)x, d_out,
-                                                     d_in, (int)batch, y_part);
+    BD_CUDA_TRY(launch_pdl(k_base_gemv_f32, dim3((unsigned)blocks), dim3(256), 0, s, (const float*)w_base,
+                           (const float*)x, d_out, d_in, (int)batch, y_part));
     launch_end(K_BASE_GEMV, s);
     BD_LAUNCH_CHECK();
   }

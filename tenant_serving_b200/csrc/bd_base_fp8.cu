@@ -79,6 +79,8 @@ __device__ __forceinline__ uint2 pack8(const uint32_t* c) {
 template <bool BF16>
 __global__ void __launch_bounds__(256) k_quantize_fp8(const void* __restrict__ w, int64_t d_out, int64_t d_in,
                                                       uint8_t* __restrict__ codes, float* __restrict__ scales) {
+  pdl_wait();  // inputs may come from the previous kernel on the stream
+  pdl_trigger();
   __shared__ float red[8];
   for (int64_t row = blockIdx.x; row < d_out; row += gridDim.x) {
     const uint8_t* wr = reinterpret_cast<const uint8_t*>(w) + row * d_in * (BF16 ? 2 : 4);
@@ -112,6 +114,8 @@ __global__ void __launch_bounds__(256) k_quantize_fp8(const void* __restrict__ w
 // ------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(128) k_x_limbs(const uint16_t* __restrict__ x, int64_t d_in, int batch, int h,
                                                  int n_tile, uint8_t* __restrict__ x8, float* __restrict__ xmul) {
+  pdl_wait();  // inputs may come from the previous kernel on the stream
+  pdl_trigger();
   __shared__ float red[4];
   const int t = blockIdx.x;
   const int j = t / h, c = t % h;
@@ -207,6 +211,8 @@ __global__ void __launch_bounds__(128, 1) k_base_fp8(const __grid_constant__ CUt
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
+  pdl_wait();  // the set-up above overlaps the previous kernel on the stream
+  pdl_trigger();
 
   bool timed_out = false;
   if (warp == 0) {
@@ -350,8 +356,8 @@ bd_status launch_base_fp8(const Fp8Plan& p, const uint8_t* codes, const float* w
                           int64_t d_out, int64_t d_in, int64_t batch, uint8_t* x8, float* xmul, float* y_part,
                           uint32_t* status, cudaStream_t s) {
   launch_begin(K_X_LIMBS, s);
-  k_x_limbs<<<(unsigned)(p.tiles_n * p.h), 128, 0, s>>>(static_cast<const uint16_t*>(x), d_in, (int)batch, p.h,
-                                                         p.n_tile, x8, xmul);
+  BD_CUDA_TRY(launch_pdl(k_x_limbs, dim3((unsigned)(p.tiles_n * p.h)), dim3(128), 0, s,
+                         static_cast<const uint16_t*>(x), d_in, (int)batch, p.h, p.n_tile, x8, xmul));
   launch_end(K_X_LIMBS, s);
   BD_LAUNCH_CHECK();
   CUtensorMap tw, tx;
@@ -362,8 +368,8 @@ bd_status launch_base_fp8(const Fp8Plan& p, const uint8_t* codes, const float* w
   if (p.tiles_m > 65535) return BD_ERR_SHAPE;
   dim3 grid(p.tiles_n, p.tiles_m, p.ksplit);
   launch_begin(K_BASE_FP8, s);
-  k_base_fp8<<<grid, 128, p.smem, s>>>(tw, tx, w_scales, xmul, d_out, (int)batch, p.h, p.n_tile, p.stages,
-                                       p.kblocks, p.kb_per_split, y_part, status);
+  BD_CUDA_TRY(launch_pdl(k_base_fp8, grid, dim3(128), p.smem, s, tw, tx, w_scales, (const float*)xmul, d_out,
+                         (int)batch, p.h, p.n_tile, p.stages, p.kblocks, p.kb_per_split, y_part, status));
   launch_end(K_BASE_FP8, s);
   BD_LAUNCH_CHECK();
   return BD_OK;
@@ -384,9 +390,11 @@ extern "C" bd_status bd_quantize_base_fp8(const void* w, int32_t w_dtype, int64_
   if (blocks > cap) blocks = cap;
   launch_begin(K_QUANT_FP8, s);
   if (w_dtype == BD_BF16)
-    k_quantize_fp8<true><<<(unsigned)blocks, 256, 0, s>>>(w, d_out, d_in, codes, scales);
+    BD_CUDA_TRY(launch_pdl(k_quantize_fp8<true>, dim3((unsigned)blocks), dim3(256), 0, s, w, d_out, d_in, codes,
+                           scales));
   else
-    k_quantize_fp8<false><<<(unsigned)blocks, 256, 0, s>>>(w, d_out, d_in, codes, scales);
+    BD_CUDA_TRY(launch_pdl(k_quantize_fp8<false>, dim3((unsigned)blocks), dim3(256), 0, s, w, d_out, d_in, codes,
+                           scales));
   launch_end(K_QUANT_FP8, s);
   BD_LAUNCH_CHECK();
   return BD_OK;

@@ -65,6 +65,8 @@ __global__ void __launch_bounds__(128, 1) k_base_tc(const __grid_constant__ CUte
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
+  pdl_wait();  // the set-up above overlaps the previous kernel on the stream
+  pdl_trigger();
 
   bool timed_out = false;
   if (warp == 0) {
@@ -223,8 +225,8 @@ bd_status launch_base_tc(const TcPlan& p, const void* w_base, const void* x, int
   if (p.tiles_m > 65535) return BD_ERR_SHAPE;  // row blocks run along grid y
   dim3 grid(p.tiles_n, p.tiles_m, p.ksplit);
   launch_begin(K_BASE_TC, s);
-  k_base_tc<<<grid, 128, p.smem, s>>>(tw, tx, d_out, (int)batch, p.n_tile, p.stages, p.kblocks,
-                                      p.kb_per_split, y_part, status);
+  BD_CUDA_TRY(launch_pdl(k_base_tc, grid, dim3(128), p.smem, s, tw, tx, d_out, (int)batch, p.n_tile, p.stages,
+                         p.kblocks, p.kb_per_split, y_part, status));
   launch_end(K_BASE_TC, s);
   BD_LAUNCH_CHECK();
   return BD_OK;

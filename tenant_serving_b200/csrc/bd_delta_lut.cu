@@ -714,6 +714,10 @@ __global__ void __launch_bounds__(DL_THREADS, 1) k_delta_lut(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // the set-up above overlaps the previous kernel on the stream; its outputs (the plan, the
+  // base partial sums) are read only after this
+  pdl_wait();
+  pdl_trigger();
 
   const int nwin = (int)((d_in + DL_W - 1) / DL_W);
   const int tiles = (int)((d_out + DL_ROWS - 1) / DL_ROWS);
@@ -1082,9 +1086,9 @@ bd_status launch_delta_lut(bool xbf16, const bd_tenant* tenants, bool scale_f16,
   if (!ensure_dyn_smem(kfn, DL_SMEM, attr[v])) return BD_ERR_CUDA;
   if (!dl_layout_fits(reinterpret_cast<const void*>(kfn), xbf16, v)) return BD_ERR_INTERNAL;
   launch_begin(K_DELTA_LUT, s);
-  kfn<<<(unsigned)sm_count(), DL_THREADS, DL_SMEM, s>>>(tenants, scale_f16, seg, max_groups, max_tc, x,
-                                                       y_part, ksplit, d_out, d_in, (int)batch, y, y_bf16,
-                                                       lut_part, lut_cnt, split_cap, status);
+  BD_CUDA_TRY(launch_pdl(kfn, dim3((unsigned)sm_count()), dim3(DL_THREADS), DL_SMEM, s, tenants, scale_f16, seg,
+                         max_groups, max_tc, x, y_part, ksplit, d_out, d_in, (int)batch, y, y_bf16, lut_part, lut_cnt,
+                         split_cap, status));
   launch_end(K_DELTA_LUT, s);
   BD_LAUNCH_CHECK();
   return BD_OK;

@@ -54,6 +54,8 @@ __global__ void __launch_bounds__(256) k_tc_gather(const int32_t* __restrict__ s
                                                    int max_groups, int max_tc,
                                                    const uint16_t* __restrict__ x, int64_t d_in,
                                                    __half* __restrict__ xg, float* __restrict__ xinv) {
+  pdl_wait();  // inputs may come from the previous kernel on the stream
+  pdl_trigger();
   const int n_tc = seg_base[1];
   const int sidx = blockIdx.y;
   if (sidx >= n_tc) return;
@@ -234,6 +236,8 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_delta_tc(
     const float* __restrict__ xinv, const float* __restrict__ y_part, int ksplit, int64_t d_out,
     int64_t d_in, int batch, void* __restrict__ y, bool y_bf16, int nmax, int xwin,
     uint32_t* __restrict__ status) {
+  pdl_wait();  // inputs may come from the previous kernel on the stream
+  pdl_trigger();
   const int n_tc = seg_base[1];
   const int mtiles = (int)((d_out + DT_BM - 1) / DT_BM);
   const int items = n_tc * mtiles;
@@ -611,8 +615,8 @@ bd_status launch_delta_tc(const bd_tenant* tc_rec, const int32_t* seg, int max_g
   // 1. gather X of the tensor-core segments
   dim3 gg(DT_NMAX / 8, (unsigned)max_tc);  // 8 rows per CTA
   launch_begin(K_TC_GATHER, s);
-  k_tc_gather<<<gg, 256, 0, s>>>(seg, max_groups, max_tc, static_cast<const uint16_t*>(x), d_in,
-                                 xg, xinv);
+  BD_CUDA_TRY(launch_pdl(k_tc_gather, gg, dim3(256), 0, s, seg, max_groups, max_tc,
+                         static_cast<const uint16_t*>(x), d_in, xg, xinv));
   launch_end(K_TC_GATHER, s);
   BD_LAUNCH_CHECK();
   // 2. tensor-core delta + combine
@@ -638,9 +642,9 @@ bd_status launch_delta_tc(const bd_tenant* tc_rec, const int32_t* seg, int max_g
   int64_t grid = (int64_t)sm_count();
   if (grid > mtiles * max_tc) grid = mtiles * max_tc;
   launch_begin(K_DELTA_TC, s);
-  k_delta_tc<<<(unsigned)grid, DT_THREADS, smem, s>>>(tm, tc_rec, seg, max_groups, max_tc, xinv,
-                                                      y_part, ksplit, d_out, d_in, (int)batch, y,
-                                                      y_bf16, nmax, xwin, status);
+  BD_CUDA_TRY(launch_pdl(k_delta_tc, dim3((unsigned)grid), dim3(DT_THREADS), smem, s, tm, tc_rec, seg, max_groups,
+                         max_tc, (const float*)xinv, y_part, ksplit, d_out, d_in, (int)batch, y, y_bf16, nmax, xwin,
+                         status));
   launch_end(K_DELTA_TC, s);
   BD_LAUNCH_CHECK();
   return BD_OK;
