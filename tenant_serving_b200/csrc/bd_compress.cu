@@ -440,19 +440,28 @@ __global__ void k_col_final(const double* __restrict__ colpart, int64_t ntile, i
 }
 
 // BLOCK: scales[rb][g] = mean over rows r of row block rb of rowmean[r][g] (each row mean
-// is over G entries, so this is the mean over the block's entries); fp64, row order
-__global__ void k_block_final(const float* __restrict__ rowmean, int64_t d_out, int64_t ngc, int G,
-                              float* __restrict__ scales) {
+// is over G entries, so this is the mean over the block's entries). Block (32 x 8
+// threads) per (row block, 32 groups): thread (x, y) sums rows y, y + 8, ... of group x in
+// fp64, then the 8 partial sums are added in y order (deterministic).
+__global__ void __launch_bounds__(256) k_block_final(const float* __restrict__ rowmean, int64_t d_out, int64_t ngc,
+                                                     int G, float* __restrict__ scales) {
   pdl_wait();  // inputs may come from the previous kernel on the stream
   pdl_trigger();
-  const int64_t nrb = (d_out + G - 1) / G;
-  const int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (k >= nrb * ngc) return;
-  const int64_t rb = k / ngc, g = k - rb * ngc;
+  __shared__ double part[8][33];
+  const int64_t rb = blockIdx.x;
+  const int64_t g = (int64_t)blockIdx.y * 32 + threadIdx.x;
   const int64_t r0 = rb * G, r1 = r0 + G < d_out ? r0 + G : d_out;
-  double s = 0.0;
-  for (int64_t r = r0; r < r1; ++r) s += (double)rowmean[r * ngc + g];
-  scales[k] = (float)(s / (double)(r1 - r0));
+  double sum = 0.0;
+  if (g < ngc)
+    for (int64_t r = r0 + threadIdx.y; r < r1; r += 8) sum += (double)rowmean[r * ngc + g];
+  part[threadIdx.y][threadIdx.x] = sum;
+  __syncthreads();
+  if (threadIdx.y == 0 && g < ngc) {
+    double t = 0.0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) t += part[k][threadIdx.x];
+    scales[rb * ngc + g] = (float)(t / (double)(r1 - r0));
+  }
 }
 
 // TENSOR: one block; strided per-thread sums then a fixed tree
@@ -502,6 +511,9 @@ bd_status plan_compress(int32_t dtype, int64_t d_out, int64_t d_in, const bd_com
   const int64_t G = cfg->group_size;
   const bool grouped = cfg->mode == BD_SCALE_GROUP || cfg->mode == BD_SCALE_BLOCK;
   if (!scale_mode_ok(cfg->mode, cfg->group_size, d_in)) return BD_ERR_CONFIG;
+  if (cfg->mode == BD_SCALE_BLOCK &&
+      ((d_out + G - 1) / G > 0x7FFFFFFF || (d_in / G + 31) / 32 > 65535))  // the block reduction's grid
+    return BD_ERR_SHAPE;
   p->bf16 = dtype == BD_BF16;
   p->chunk = p->bf16 ? 256 : 128;
   p->nchunks = (d_in + p->chunk - 1) / p->chunk;
@@ -612,9 +624,10 @@ bd_status launch_compress(const CompressPlan& p, const void* w_base, const void*
     launch_end(K_SCALE_FINAL, s);
     BD_LAUNCH_CHECK();
   } else if (cfg->mode == BD_SCALE_BLOCK) {
-    const int64_t ngc = d_in >> lg, n = ((d_out + cfg->group_size - 1) / cfg->group_size) * ngc;
+    const int64_t ngc = d_in >> lg;
     launch_begin(K_SCALE_FINAL, s);
-    BD_CUDA_TRY(launch_pdl(k_block_final, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s,
+    const int64_t nrb = (d_out + cfg->group_size - 1) / cfg->group_size;  // grid limits checked in the plan
+    BD_CUDA_TRY(launch_pdl(k_block_final, dim3((unsigned)nrb, (unsigned)((ngc + 31) / 32)), dim3(32, 8), 0, s,
                            reinterpret_cast<const float*>(part), d_out, ngc, (int)cfg->group_size, scales));
     launch_end(K_SCALE_FINAL, s);
     BD_LAUNCH_CHECK();
