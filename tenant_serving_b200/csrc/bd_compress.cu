@@ -427,16 +427,26 @@ __global__ void k_row_final(const double* __restrict__ partials, int nseg, int64
   scales[r] = (float)(s / (double)d_in);
 }
 
-// COL: scales[i] = sum_t colpart[t][i] / d_out (one thread per column)
-__global__ void k_col_final(const double* __restrict__ colpart, int64_t ntile, int64_t d_out,
-                            int64_t d_in, float* __restrict__ scales) {
+// COL: scales[i] = sum_t colpart[t][i] / d_out. Block (32 x 8 threads) per 32 columns:
+// thread (x, y) sums tiles y, y + 8, ... of column x, then the 8 partial sums are added in
+// y order (deterministic).
+__global__ void __launch_bounds__(256) k_col_final(const double* __restrict__ colpart, int64_t ntile, int64_t d_out,
+                                                   int64_t d_in, float* __restrict__ scales) {
   pdl_wait();  // inputs may come from the previous kernel on the stream
   pdl_trigger();
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= d_in) return;
-  double s = 0.0;
-  for (int64_t t = 0; t < ntile; ++t) s += colpart[t * d_in + i];
-  scales[i] = (float)(s / (double)d_out);
+  __shared__ double part[8][33];
+  const int64_t i = (int64_t)blockIdx.x * 32 + threadIdx.x;
+  double sum = 0.0;
+  if (i < d_in)
+    for (int64_t t = threadIdx.y; t < ntile; t += 8) sum += colpart[t * d_in + i];
+  part[threadIdx.y][threadIdx.x] = sum;
+  __syncthreads();
+  if (threadIdx.y == 0 && i < d_in) {
+    double tot = 0.0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) tot += part[k][threadIdx.x];
+    scales[i] = (float)(tot / (double)d_out);
+  }
 }
 
 // BLOCK: scales[rb][g] = mean over rows r of row block rb of rowmean[r][g] (each row mean
@@ -588,7 +598,7 @@ bd_status launch_compress(const CompressPlan& p, const void* w_base, const void*
     launch_end(K_COL_SCALE_SIGNPACK, s);
     BD_LAUNCH_CHECK();
     launch_begin(K_SCALE_FINAL, s);
-    BD_CUDA_TRY(launch_pdl(k_col_final, dim3((unsigned)((d_in + 255) / 256)), dim3(256), 0, s, (const double*)part,
+    BD_CUDA_TRY(launch_pdl(k_col_final, dim3((unsigned)((d_in + 31) / 32)), dim3(32, 8), 0, s, (const double*)part,
                            p.ntile, d_out, d_in, scales));
     launch_end(K_SCALE_FINAL, s);
     BD_LAUNCH_CHECK();
