@@ -138,9 +138,12 @@ bd_status bd_compress(const void* w_base, const void* w_fine, int32_t dtype, int
  *     BD_NOALLOC_SCRATCH_BYTES are rejected with BD_ERR_WORKSPACE before any launch.
  *     GROUP mode needs about 10 KB at any size; ROW / TENSOR need 8 bytes per row per
  *     column segment (every Llama-3-8B projection fits); COL needs 8 bytes per column
- *     per tile of rows, so large COL problems do not fit.
+ *     per tile of rows and BLOCK 4 bytes per (row, group), so large COL and BLOCK
+ *     problems do not fit.
  *   - The first call on each device looks up the array's device address (with that
  *     device current) and caches it; make that first call before any stream capture.
+ *     The cached address does not survive cudaDeviceReset: after a reset, use
+ *     bd_compress (or a process that loads the library afresh).
  *   - Every call shares the one array and it keeps the last call's contents; nothing in
  *     it has to start at zero. Calls whose execution overlaps on the GPU (other streams,
  *     other host threads) race on it: serialise them.
