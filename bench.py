@@ -89,7 +89,9 @@ def parse():
     p.add_argument("--compress-layers", type=int, default=N_LAYERS)
     p.add_argument("--no-compress", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--no-extra", action="store_true", help="skip the decode and mixed workloads")
+    p.add_argument("--no-extra", action="store_true", help="skip the decode, mixed and cold-start workloads")
+    p.add_argument("--extra", default="decode,decode_fp8,mixed,cold_start",
+                   help="comma-separated extra workloads to run after the serving step (N = 1)")
     p.add_argument("--cpu-seconds", type=float, default=15.0)
     return p.parse_args()
 
@@ -878,10 +880,11 @@ def main():
     dec = dec8 = mix = None
     cold = None
     if rank == 0 and world == 1 and not args.no_extra:
-        dec = bench_decode(args, log, peaks)
-        dec8 = bench_decode(args, log, peaks, fp8=True)
-        mix = bench_mixed(args, log, peaks)
-        cold = bench_cold_start(args, log, peaks)
+        extra = set(e for e in args.extra.split(",") if e)
+        dec = bench_decode(args, log, peaks) if "decode" in extra else None
+        dec8 = bench_decode(args, log, peaks, fp8=True) if "decode_fp8" in extra else None
+        mix = bench_mixed(args, log, peaks) if "mixed" in extra else None
+        cold = bench_cold_start(args, log, peaks) if "cold_start" in extra else None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(args.cpu_seconds)
     if rank == 0:
