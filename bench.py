@@ -60,8 +60,10 @@ def tc_min_tokens() -> int:
 # was built from: once they change, the number no longer describes the kernel and the
 # roofline reports traffic = null.
 NCU_TRAFFIC = {
+    # profiles/delta_lut_serving_layer.md: mean over the qkv, o, gate_up and down calls
+    # (each a quarter of a step's launches) of dram__bytes_read.sum + dram__bytes_write.sum
     "delta_lut": {"sources": ["bd_delta_lut.cu", "bd_internal.cuh", "bd_tc.cuh"],
-                  "sha256_16": "0000000000000000", "bytes_per_launch": None},
+                  "sha256_16": "26e40ca3b865e33c", "bytes_per_launch": 562501740.0},
 }
 
 
@@ -213,12 +215,14 @@ def whole_job_rate(pg, units: float, ms: float):
 
 
 def serving_config(args, world: int) -> dict:
-    return {"workload": "serving: 32-layer Llama-3-8B-shaped projection stack "
-                        "(q, k, v, o, gate, up, down; applied as fused qkv / o / gate_up / down, "
-                        "128 calls), bf16 base + 100 resident tenants (sign words + fp16 "
-                        "group-128 scales), batch 512, Zipf(1.1) tenant ids, one decode step per step",
+    return {"workload": f"serving: {args.layers}-layer Llama-3-8B-shaped projection stack "
+                        f"(q, k, v, o, gate, up, down; applied as fused qkv / o / gate_up / down, "
+                        f"{4 * args.layers} calls), bf16 base + {args.tenants} resident tenants (sign words + "
+                        f"fp16 group-128 scales), batch {args.batch}, Zipf(1.1) tenant ids, one decode step "
+                        f"per step",
             "layers": args.layers, "tenants": args.tenants, "batch": args.batch,
-            "group_size": GROUP, "l2": "inputs larger than L2 (~112 GB resident)",
+            "group_size": GROUP,
+            "l2": f"inputs larger than L2 (~{3.5 * args.layers * args.tenants / 100:.0f} GB resident)",
             "parallelism": f"replicas x{world}"}
 
 
