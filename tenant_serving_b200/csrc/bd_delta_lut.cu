@@ -198,6 +198,28 @@ __device__ __forceinline__ void tmem_ld8_wait(uint32_t taddr, float* v) {
   for (int q = 0; q < 8; ++q) v[q] = __uint_as_float(r[q]);
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// 32 lanes x 8 (or 4) columns of tensor memory -> registers, without waiting: the registers
+// hold the values only after tmem_ld_tile_wait on them (the wait takes them as operands,
+// so no use can be scheduled before it). Lets a tile's table reads overlap the load.
+__device__ __forceinline__ void tmem_ld_tile_async(uint32_t taddr, uint32_t* r) {
+  if (DL_RPL == 2)
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+  else
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_tile_wait(uint32_t* r) {
+  if (DL_RPL == 2)
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7])
+                 :
+                 : "memory");
+  else
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]) : : "memory");
+}
 // the running sums of one tile (DL_TSTRIDE columns)
 __device__ __forceinline__ void tmem_st_tile(uint32_t taddr, const float* v) {
   if (DL_RPL == 2) tmem_st8(taddr, v);
@@ -920,6 +942,9 @@ __global__ void __launch_bounds__(DL_THREADS, 1) k_delta_lut(
             dead = true;
             break;
           }
+          // the previous window's stores of the running sums are complete before they are
+          // read back below
+          if (win > wbeg) tmem_wait_st();
           for (int p = 0; p < P; ++p) {
             if (!__all_sync(0xffffffffu, mbar_wait(&full[S.slot], S.phase, abort_flag))) {
               dead = true;
@@ -930,15 +955,20 @@ __global__ void __launch_bounds__(DL_THREADS, 1) k_delta_lut(
 #pragma unroll
             for (int q = 0; q < 4 * DL_RPL; ++q) part[q] = 0.f;
             const uint32_t tcol = t_lane + DL_TSTRIDE * (uint32_t)p;
-            if (win > wbeg) {
-              // running sums of this tile from the previous windows
-              tmem_wait_st();
-              tmem_ld_tile(tcol, part);
-            }
+            // the running sums of this tile from the previous windows load while the
+            // window's table reads run; they are added at the end
+            uint32_t prev[4 * DL_RPL];
+            const bool carry = win > wbeg;
+            if (carry) tmem_ld_tile_async(tcol, prev);
 #pragma unroll
             for (int h = 0; h < DL_RPL; ++h)
               dl_row_window(D, st, r_lo + 32 * DL_CWARPS * h, tile0 + p, win, nt, sig, hi_slots, scale_f16, d_out,
                             d_in, wpr, K, sel, part + 4 * h);
+            if (carry) {
+              tmem_ld_tile_wait(prev);
+#pragma unroll
+              for (int q = 0; q < 4 * DL_RPL; ++q) part[q] += __uint_as_float(prev[q]);
+            }
             tmem_st_tile(tcol, part);
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[S.slot]);
