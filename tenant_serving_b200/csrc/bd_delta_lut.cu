@@ -369,28 +369,23 @@ __device__ __forceinline__ void lut_row(const uint32_t (&wd)[8], const float (&s
                                         const uint32_t (&sel)[4], float* part) {
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    // the word's four table reads per token, added as a tree (two dependent adds, not four)
+    float2 e[4], f[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const uint32_t addr = prmt(wd[i], K[i][j >> 1], sel[j]);
       if (NT == 1) {
-        a0 += lds_off<0>(addr);
+        e[j].x = lds_off<0>(addr);
       } else {
-        const float2 e = lds2_off<0>(addr);
-        a0 += e.x;
-        a1 += e.y;
-        if (NT == 3) a2 += lds_off<(int)DL_PAGE>(addr);
-        if (NT == 4) {
-          const float2 f = lds2_off<(int)DL_PAGE>(addr);
-          a2 += f.x;
-          a3 += f.y;
-        }
+        e[j] = lds2_off<0>(addr);
+        if (NT == 3) f[j].x = lds_off<(int)DL_PAGE>(addr);
+        if (NT == 4) f[j] = lds2_off<(int)DL_PAGE>(addr);
       }
     }
-    part[0] = fmaf(sc[i], a0, part[0]);
-    if (NT > 1) part[1] = fmaf(sc[i], a1, part[1]);
-    if (NT > 2) part[2] = fmaf(sc[i], a2, part[2]);
-    if (NT > 3) part[3] = fmaf(sc[i], a3, part[3]);
+    part[0] = fmaf(sc[i], (e[0].x + e[1].x) + (e[2].x + e[3].x), part[0]);
+    if (NT > 1) part[1] = fmaf(sc[i], (e[0].y + e[1].y) + (e[2].y + e[3].y), part[1]);
+    if (NT > 2) part[2] = fmaf(sc[i], (f[0].x + f[1].x) + (f[2].x + f[3].x), part[2]);
+    if (NT > 3) part[3] = fmaf(sc[i], (f[0].y + f[1].y) + (f[2].y + f[3].y), part[3]);
   }
 }
 
