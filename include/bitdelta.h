@@ -338,10 +338,12 @@ size_t bd_apply_workspace_size(int64_t d_out, int64_t d_in, int64_t batch, int32
  * work, chosen per tenant on the device:
  *   - a tenant with at least bd_tc_min_tokens() tokens in the batch (9 as built),
  *     stored in the TILED layout with
- *     fp16 scales in GROUP (group_size >= 64), ROW or TENSOR mode (bf16 w_base and
- *     d_in % 64 == 0), is a dense product on the tensor cores, in segments of <= 64 of
- *     its tokens; its activations are scaled per token by a power of two into fp16 for
- *     that product (exact for bf16 values in fp16's normal range);
+ *     fp16 scales in GROUP or BLOCK (group_size >= 64), ROW, COL or TENSOR mode (bf16
+ *     activations and d_in % 64 == 0), is a dense product on the tensor cores, in
+ *     segments of <= 64 of its tokens; its activations are scaled per token by a power of
+ *     two into fp16 for that product (exact for bf16 values in fp16's normal range; for
+ *     COL scales the activations are multiplied by the column scales first, and that
+ *     product is rounded to fp16, a relative error of at most 2^-11 per element);
  *   - every other tenant goes through the sign lookup-table kernel, its packed signs and
  *     scales streamed once per group of <= 4 of its tokens (once in all when it has at
  *     most 4 tokens in the batch).

@@ -49,7 +49,7 @@ inline int max_groups_for(int64_t batch, int32_t n_tenants) {
 __device__ __forceinline__ bool tc_eligible(const bd_tenant& T, int64_t d_in) {
   const bool mode_ok = ((T.mode == BD_SCALE_GROUP || T.mode == BD_SCALE_BLOCK) && T.group_size >= 64 &&
                         scale_mode_ok(T.mode, T.group_size, d_in)) ||
-                       T.mode == BD_SCALE_ROW || T.mode == BD_SCALE_TENSOR;
+                       T.mode == BD_SCALE_ROW || T.mode == BD_SCALE_COL || T.mode == BD_SCALE_TENSOR;
   const bool ptr_ok = T.signs != nullptr && T.scales != nullptr &&
                       ((reinterpret_cast<uintptr_t>(T.signs) | reinterpret_cast<uintptr_t>(T.scales)) & 15u) == 0;
   // the tensor-core kernel streams whole tiles of the serving layout

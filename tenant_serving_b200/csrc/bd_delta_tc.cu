@@ -14,15 +14,18 @@
 //     each 32-bit register of two halves is one shift and one LOP3 of the word;
 //   - X is gathered once per call in the same column order (k_tc_gather) as fp16 of
 //     x * 2^e_t, with 2^e_t per token chosen so the largest |x| stays below 2^15: bf16
-//     values are then exact in fp16 (tiny ones lose only sub-2^-24 bits);
+//     values are then exact in fp16 (tiny ones lose only sub-2^-24 bits). For a tenant
+//     with column scales the gather multiplies each x_i by s_i first (A is then +/-1):
+//     Delta_hat x = sign . (s * x); the fp16 rounding of s_i x_i is the one inexact step
+//     (relative 2^-11 per product);
 //   - one thread issues tcgen05.mma with A from tensor memory and B from shared memory
 //     (M=128, N = n_u rounded to 16, K=16, fp32 accumulation in tensor memory); four
 //     more warps read the accumulator, multiply by 2^-e_t (exact), add the base product
 //     and write y. The accumulator is double buffered so that this epilogue overlaps
 //     the next tile's MMAs.
 // Tenants qualify when they are stored in the tiled serving layout, their scales are
-// fp16 and in GROUP (group >= 64), ROW or TENSOR mode, and d_in % 64 == 0; the planner
-// sends the rest to the lookup-table kernel.
+// fp16 and in GROUP or BLOCK (group >= 64), ROW, COL or TENSOR mode, and d_in % 64 == 0;
+// the planner sends the rest to the lookup-table kernel.
 #include "bd_internal.cuh"
 #include "bd_tc.cuh"
 
@@ -52,6 +55,7 @@ constexpr uint32_t DT_WIN_SCALE_BYTES = 512;  // 128 rows x 2 fp16 (tiled group-
 // seg arrays: tc_tenant, tc_start, tc_count, tc_xrow (Xg row of the segment's first token)
 __global__ void __launch_bounds__(256) k_tc_gather(const int32_t* __restrict__ seg_base,
                                                    int max_groups, int max_tc,
+                                                   const bd_tenant* __restrict__ tc_rec,
                                                    const uint16_t* __restrict__ x, int64_t d_in,
                                                    __half* __restrict__ xg, float* __restrict__ xinv) {
   pdl_wait();  // inputs may come from the previous kernel on the stream
@@ -82,18 +86,45 @@ __global__ void __launch_bounds__(256) k_tc_gather(const int32_t* __restrict__ s
   }
   const int t = permv[tc_start[sidx] + r];
   const uint16_t* xt = x + (int64_t)t * d_in;
-  // largest |x| of the token (unrolled so that a lane's loads are in flight together)
-  float m = 0.f;
-#pragma unroll 4
-  for (int b = lane; b < nblk; b += 32) {
+  // column scales of the segment's tenant (fp16), folded into its activations
+  const bool col = tc_rec[sidx].mode == BD_SCALE_COL;
+  const uint16_t* cs = static_cast<const uint16_t*>(tc_rec[sidx].scales);
+  // 32 values of column block b: x, times the column scale for a COL tenant
+  auto load32 = [&](int b, float* v) {
     const uint4* p = reinterpret_cast<const uint4*>(xt + 32 * b);
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const uint4 v = p[k];
-      const uint32_t a[4] = {v.x, v.y, v.z, v.w};
+      const uint4 w = p[k];
+      const uint32_t a[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-      for (int j = 0; j < 4; ++j) m = fmaxf(m, fmaxf(fabsf(bf16lo(a[j])), fabsf(bf16hi(a[j]))));
+      for (int j = 0; j < 4; ++j) {
+        v[8 * k + 2 * j] = bf16lo(a[j]);
+        v[8 * k + 2 * j + 1] = bf16hi(a[j]);
+      }
     }
+    if (col) {
+      const uint4* q = reinterpret_cast<const uint4*>(cs + 32 * b);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint4 w = q[k];
+        const uint32_t a[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const __half2 h = *reinterpret_cast<const __half2*>(&a[j]);
+          v[8 * k + 2 * j] *= __low2float(h);
+          v[8 * k + 2 * j + 1] *= __high2float(h);
+        }
+      }
+    }
+  };
+  // largest |x| (|s x| for a COL tenant) of the token
+  float m = 0.f;
+#pragma unroll 2
+  for (int b = lane; b < nblk; b += 32) {
+    float v[32];
+    load32(b, v);
+#pragma unroll
+    for (int k = 0; k < 32; ++k) m = fmaxf(m, fabsf(v[k]));
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -107,18 +138,10 @@ __global__ void __launch_bounds__(256) k_tc_gather(const int32_t* __restrict__ s
   const float sc = ldexpf(1.f, e);
 #pragma unroll 2
   for (int b = lane; b < nblk; b += 32) {
-    const uint4* p = reinterpret_cast<const uint4*>(xt + 32 * b);
     float v[32];
+    load32(b, v);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const uint4 w = p[k];
-      const uint32_t a[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        v[8 * k + 2 * j] = bf16lo(a[j]) * sc;
-        v[8 * k + 2 * j + 1] = bf16hi(a[j]) * sc;
-      }
-    }
+    for (int k = 0; k < 32; ++k) v[k] *= sc;
     // K position 2q <- column q, 2q + 1 <- column q + 16
     uint32_t o[16];
 #pragma unroll
@@ -317,7 +340,8 @@ __global__ void __launch_bounds__(DT_THREADS, 1) k_delta_tc(
       const int gshift = (T.mode == BD_SCALE_GROUP || blockwise) ? __ffs(T.group_size) - 1 : 0;
       const int64_t srow = blockwise ? (row >> gshift) : row;  // BLOCK: G x G blocks
       uint32_t s_item = 0;
-      if (kind == 2 && live) s_item = sc16[T.mode == BD_SCALE_ROW ? row : 0];
+      // (a COL tenant's scales are in its gathered activations: A = +/-1)
+      if (kind == 2 && live) s_item = T.mode == BD_SCALE_COL ? 0x3C00u : sc16[T.mode == BD_SCALE_ROW ? row : 0];
       auto stage_scale = [&](int kb) -> uint32_t {
         if (!live || kb >= nkb) return 0u;
         return sc16[srow * (d_in >> gshift) + (((int64_t)kb * DT_BK) >> gshift)];
@@ -615,7 +639,7 @@ bd_status launch_delta_tc(const bd_tenant* tc_rec, const int32_t* seg, int max_g
   // 1. gather X of the tensor-core segments
   dim3 gg(DT_NMAX / 8, (unsigned)max_tc);  // 8 rows per CTA
   launch_begin(K_TC_GATHER, s);
-  BD_CUDA_TRY(launch_pdl(k_tc_gather, gg, dim3(256), 0, s, seg, max_groups, max_tc,
+  BD_CUDA_TRY(launch_pdl(k_tc_gather, gg, dim3(256), 0, s, seg, max_groups, max_tc, tc_rec,
                          static_cast<const uint16_t*>(x), d_in, xg, xinv));
   launch_end(K_TC_GATHER, s);
   BD_LAUNCH_CHECK();

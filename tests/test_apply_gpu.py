@@ -333,7 +333,9 @@ def test_many_token_tenants_delta_only(bd, mode, G, layout):
     """300 tokens (five tensor-core segments), 9 (the smallest many-token tenant), 8 (two
     passes of the lookup-table kernel), 20 and 1 token; 200 rows (a partial 128-row tile),
     384 columns (a partial 256-column tile of the serving layout; 768 for groups of 256).
-    Column scales (mode 2) stay on the lookup-table path."""
+    Column scales (mode 2) in the tiled layout take the tensor-core path with the scales
+    folded into the fp16 activations: that product rounds once per element (relative
+    2^-11), so its fp32 check is 1e-3 per token instead of 1e-5."""
     d_out, d_in = 200, (768 if G == 256 else 384)
     wb, tenants, ids, x = _many_token_problem(mode * 7 + G + layout, d_out, d_in,
                                               [300, 9, 8, 20, 1], mode, G, zero_base=True)
@@ -341,7 +343,8 @@ def test_many_token_tenants_delta_only(bd, mode, G, layout):
     y, rc, flags = _run(bd, wb, tenants, ids, x, y_dtype="f32", layout=layout)
     assert rc == bd.BD_OK and flags == 0
     assert_apply_close(y, y_ref)
-    assert_apply_close(y, y_ref, tol=1e-5, per_token=True, what="delta only (fp32 out)")
+    tight = 1e-3 if (mode == 2 and layout == 1) else 1e-5
+    assert_apply_close(y, y_ref, tol=tight, per_token=True, what="delta only (fp32 out)")
 
 
 @pytest.mark.parametrize("layout", [0, 1])
