@@ -434,8 +434,10 @@ def bench_serving(args, rank, pg, log, peaks):
                      "unit": unit, "frac": (achieved / peak) if achieved else None,
                      "traffic": ncu_traffic(dname),
                      "algorithmic_per_launch": (work / dl) if (work and dl) else None,
-                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json "
-                                    f"{'bf16_tflops_sustained' if unit == 'TFLOP/s' else 'hbm_gbs'})",
+                     "peak_source": (f"measured (MEASURED_PEAKS.json "
+                                     f"{'bf16_tflops_sustained' if unit == 'TFLOP/s' else 'hbm_gbs'})"
+                                     if peak_src == "measured" else
+                                     "fallback: the pool's earlier measurement (no MEASURED_PEAKS.json)"),
                      "avg_launch_us": dms / dl * 1e3 if dl else None},
         "kernel_rates": {k: {"achieved": kernel_work[k][0] / (prof[k][1] / 1e3) /
                                          (1e12 if kernel_work[k][1] == "TFLOP/s" else 1e9),

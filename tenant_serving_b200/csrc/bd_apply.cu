@@ -62,7 +62,8 @@ __global__ void __launch_bounds__(1024) k_tenant_bucket(const int32_t* __restric
                                                         int n_tenants, int max_groups, int max_tc,
                                                         const bd_tenant* __restrict__ tenants,
                                                         int tc_min, int64_t d_in, int64_t lut_tiles,
-                                                        int split_cap, int32_t* __restrict__ lut_cnt,
+                                                        int split_cap, int lut_ctas,
+                                                        int32_t* __restrict__ lut_cnt,
                                                         int32_t* __restrict__ seg_base,
                                                         bd_tenant* __restrict__ tc_rec,
                                                         uint32_t* __restrict__ status) {
@@ -201,16 +202,17 @@ __global__ void __launch_bounds__(1024) k_tenant_bucket(const int32_t* __restric
     seg_base[1] = tidx;
 #pragma unroll
     for (int k = 0; k < kLutClasses; ++k) seg_base[2 + k] = wsum[3 + k][last];
-    // K chunks of the lookup kernel's tenant units: when there are too few (group, tile)
-    // units to keep every SM busy, each is cut into kc chunks of d_in (kc divides the
-    // windows, >= 2 windows per chunk), as many as the partial-sum budget allows
+    // K chunks of the lookup kernel's tenant units: when there are fewer (group, tile)
+    // units than kLutMinUnitsPerCta per CTA of the lookup kernel, whole units would split
+    // unevenly over the SMs, so each is cut into kc chunks of d_in (kc divides the windows,
+    // >= 2 windows per chunk), as many as the partial-sum budget allows
     int64_t units = 0;
 #pragma unroll
     for (int k = 0; k < kLutClasses - 1; ++k) units += wsum[3 + k][last];
     units *= lut_tiles;
     const int64_t nwin = (d_in + kLutWindow - 1) / kLutWindow;
     int kc = 1;
-    if (units > 0)
+    if (units > 0 && units < (int64_t)kLutMinUnitsPerCta * lut_ctas)
       for (int c = kLutMaxChunks; c >= 2; --c)
         if (nwin % c == 0 && nwin / c >= 2 && units * c <= (int64_t)split_cap) {
           kc = c;
@@ -409,7 +411,7 @@ bd_status apply_impl(const void* w_base, int32_t w_dtype, int64_t d_out, int64_t
   launch_begin(K_TENANT_BUCKET, s);
   BD_CUDA_TRY(launch_pdl(k_tenant_bucket, dim3(1), dim3(1024), bucket_smem, s, tenant_ids, (int)batch, n_tenants,
                          L.max_groups, L.max_tc, tenants, (int)kTcMinTokens, d_in,
-                         (int64_t)((d_out + kLutTileRows - 1) / kLutTileRows), L.split_cap,
+                         (int64_t)((d_out + kLutTileRows - 1) / kLutTileRows), L.split_cap, sm_count(),
                          reinterpret_cast<int32_t*>(ws + L.off_lcnt), seg,
                          reinterpret_cast<bd_tenant*>(ws + L.off_tcrec), status));
   launch_end(K_TENANT_BUCKET, s);

@@ -1100,10 +1100,13 @@ bd_status launch_delta_lut(bool xbf16, const bd_tenant* tenants, bool scale_f16,
                            int64_t d_out, int64_t d_in, int64_t batch, void* y, bool y_bf16,
                            float* lut_part, int32_t* lut_cnt, int split_cap, uint32_t* status,
                            cudaStream_t s) {
-  // the K-chunk variant only when the planner can choose kc >= 2: at most max_groups tenant
-  // groups of ceil(d_out / 512) tiles, cut in two, within the partial-sum budget
+  // the K-chunk variant when the planner cuts units for any plan of this shape (at most
+  // max_groups tenant groups of ceil(d_out / 512) tiles, fewer than kLutMinUnitsPerCta per
+  // CTA), and for long rows (>= 32 windows), where a plan with few units is worth cutting
+  // even if most plans of the shape are not
   const int64_t tiles = (d_out + DL_ROWS - 1) / DL_ROWS, nwin = (d_in + DL_W - 1) / DL_W;
-  const bool split = nwin >= 4 && (int64_t)max_groups * tiles * 2 <= (int64_t)split_cap;
+  const bool split = split_cap >= 2 && nwin >= 4 &&
+                     ((int64_t)max_groups * tiles < (int64_t)kLutMinUnitsPerCta * sm_count() || nwin >= 32);
   auto kfn = xbf16 ? (split ? k_delta_lut<true, true> : k_delta_lut<true, false>)
                    : (split ? k_delta_lut<false, true> : k_delta_lut<false, false>);
   const int v = (xbf16 ? 1 : 0) + (split ? 2 : 0);

@@ -115,6 +115,26 @@ def test_delta_only_tight(bd, mode, d_out, d_in, layout):
 
 
 @pytest.mark.parametrize("layout", [0, 1])
+@pytest.mark.parametrize("d_out,d_in", [(600, 8224), (1100, 14336), (520, 4096)])
+def test_k_chunks(bd, d_out, d_in, layout):
+    """Few (tenant group, 512-row tile) units: the lookup-table kernel cuts each unit
+    into K chunks of whole 256-column windows (33 ragged windows into 3 chunks, 56 into 8,
+    16 into 8), and the CTA that completes a tile adds the chunks' partial sums. Every
+    scale mode, groups of 1-4 tokens and a 6-token tenant (two passes); W_base = 0 and
+    fp32 outputs, held to 1e-5 per token as well."""
+    G = 32 if d_in % 128 else 128
+    ids = np.array([0] * 4 + [1] * 3 + [2] * 2 + [3] + [4] * 6 + [-1] * 2, dtype=np.int32)
+    np.random.default_rng(d_in).shuffle(ids)
+    wb, tenants, ids, x = _problem(d_out * 3 + d_in, d_out, d_in, len(ids), 5, (0, 1, 2, 3, 4), G=G,
+                                   zero_base=True, ids=ids)
+    y_ref = O.apply_multi(wb, "bf16", tenants, ids, x, "bf16")
+    y, rc, flags = _run(bd, wb, tenants, ids, x, y_dtype="f32", layout=layout)
+    assert rc == bd.BD_OK and flags == 0
+    assert_apply_close(y, y_ref)
+    assert_apply_close(y, y_ref, tol=1e-5, per_token=True, what="delta only (fp32 out)")
+
+
+@pytest.mark.parametrize("layout", [0, 1])
 def test_mixed_modes_and_group_sizes(bd, layout):
     rng = np.random.default_rng(12)
     d_out, d_in = 520, 2048
