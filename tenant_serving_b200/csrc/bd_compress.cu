@@ -15,8 +15,10 @@
 //                      one row, 16 bytes per lane per input; signs are packed with two
 //                      (bf16) or three (fp32) xor-shuffles of per-lane bit masks; group
 //                      sums are xor-shuffle trees; row / tensor sums go to fp64 partials.
-//   k_col_scale_signpack  COL mode: a warp walks a tile of rows of one column chunk,
-//                      keeping fp64 column sums in registers; fp64 partials per tile.
+//   k_col_scale_signpack  COL mode: a CTA of 8 warps walks a tile of rows of one column
+//                      chunk, each warp its own rows with 8 rows in flight (fp32 sums over
+//                      those 8, fp64 across them); the warps' column sums are added in
+//                      shared memory into one fp64 partial per column and CTA.
 //   k_scale_final      fixed-order reduction of the partials into row / column / tensor
 //                      scales (deterministic, no atomics).
 //   k_block_final      BLOCK mode: the main pass writes each row's group means; the
@@ -344,8 +346,13 @@ __global__ void __launch_bounds__(256, 4) k_scale_signpack(
 // ------------------------------------------------------------------------------------
 // COL mode: per-column sums over row tiles
 // ------------------------------------------------------------------------------------
-template <bool BF16>
-__global__ void __launch_bounds__(256) k_col_scale_signpack(
+// A CTA of 8 warps takes 8 x tile_rows consecutive rows of one column chunk (CHUNK
+// columns, VEC per lane). Warp w walks rows w * tile_rows .. of them with UR rows of both
+// inputs in flight; the |delta| of a column over those UR rows is summed in fp32 and added
+// to the lane's fp64 sums. The CTA then adds its 8 warps' sums in warp order into one fp64
+// partial per column: colpart[cta tile][column].
+template <bool BF16, bool CLIP>
+__global__ void __launch_bounds__(256, 2) k_col_scale_signpack(
     const uint8_t* __restrict__ wb, const uint8_t* __restrict__ wf, int64_t d_out, int64_t d_in,
     int tile_rows, int64_t nchunks, const ClipParams* __restrict__ clipp,
     uint32_t* __restrict__ signs, double* __restrict__ colpart) {
@@ -356,22 +363,19 @@ __global__ void __launch_bounds__(256) k_col_scale_signpack(
   constexpr int CHUNK = 32 * VEC;
   constexpr int LPW = 32 / VEC;
   constexpr int ESZ = BF16 ? 2 : 4;
-  constexpr int UR = 4;  // rows in flight per warp
-  const int lane = threadIdx.x & 31;
-  const int64_t task = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int64_t ntile = (d_out + tile_rows - 1) / tile_rows;
-  if (task >= ntile * nchunks) return;
-  const int64_t tile = task / nchunks;
-  const int64_t chunk = task % nchunks;
+  constexpr int UR = 8;  // rows in flight per warp
+  __shared__ double red[8][CHUNK];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t tile = blockIdx.x / nchunks;
+  const int64_t chunk = blockIdx.x % nchunks;
   const int64_t col = chunk * CHUNK + lane * VEC;
   const bool valid = col < d_in;
   ClipF cp{0.f, 0.f, 0.f, 0.f};
-  const bool do_clip = clipp != nullptr;
-  if (do_clip) cp = load_clip(clipp);
+  if (CLIP) cp = load_clip(clipp);
   double acc[VEC];
 #pragma unroll
   for (int k = 0; k < VEC; ++k) acc[k] = 0.0;
-  const int64_t r0 = tile * tile_rows;
+  const int64_t r0 = (tile * 8 + warp) * (int64_t)tile_rows;
   const int64_t r1 = min(d_out, r0 + tile_rows);
   const int64_t words_per_row = d_in >> 5;
   const int64_t rstride = d_in * ESZ;
@@ -386,6 +390,9 @@ __global__ void __launch_bounds__(256) k_col_scale_signpack(
         f[u] = ldg_stream(pf + u * rstride);
       }
     }
+    float sum[VEC];
+#pragma unroll
+    for (int k = 0; k < VEC; ++k) sum[k] = 0.f;
 #pragma unroll
     for (int u = 0; u < UR; ++u) {
       if (r + u >= r1) break;  // warp-uniform
@@ -395,9 +402,9 @@ __global__ void __launch_bounds__(256) k_col_scale_signpack(
         V::delta(b[u], f[u], d);
 #pragma unroll
         for (int k = 0; k < VEC; ++k) {
-          float dc = do_clip ? clamp_delta(d[k], cp) : d[k];
+          const float dc = CLIP ? clamp_delta(d[k], cp) : d[k];
           m |= (dc < 0.f ? 0u : 1u) << k;
-          acc[k] += (double)fabsf(dc);
+          sum[k] += fabsf(dc);
         }
       }
       uint32_t v = m << (VEC * (lane % LPW));
@@ -405,10 +412,20 @@ __global__ void __launch_bounds__(256) k_col_scale_signpack(
       for (int o = 1; o < LPW; o <<= 1) v |= __shfl_xor_sync(0xffffffffu, v, o);
       if (valid && (lane % LPW) == 0) signs[(r + u) * words_per_row + (col >> 5)] = v;
     }
-  }
-  if (valid) {
 #pragma unroll
-    for (int k = 0; k < VEC; ++k) colpart[tile * d_in + col + k] = acc[k];
+    for (int k = 0; k < VEC; ++k) acc[k] += (double)sum[k];
+  }
+#pragma unroll
+  for (int k = 0; k < VEC; ++k) red[warp][lane * VEC + k] = acc[k];
+  __syncthreads();
+  for (int c = threadIdx.x; c < CHUNK; c += blockDim.x) {
+    const int64_t cc = chunk * CHUNK + c;
+    if (cc < d_in) {
+      double t = 0.0;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) t += red[w][c];
+      colpart[tile * d_in + cc] = t;
+    }
   }
 }
 
@@ -539,11 +556,14 @@ bd_status plan_compress(int32_t dtype, int64_t d_out, int64_t d_in, const bd_com
   p->nseg = (int)((p->nchunks + segc - 1) / segc);
   p->stats_blocks = sms * 4;
   p->main_blocks = (int)((d_out * (int64_t)p->nseg + 7) / 8);
-  // COL tiles: enough tasks for the GPU, tiles of 32..256 rows
-  int tile = 256;
-  while (tile > 32 && ((d_out + tile - 1) / tile) * p->nchunks < target_tasks) tile >>= 1;
+  // COL: CTAs of 8 warps x tile rows, tile 8..64 rows: the longest that still gives
+  // every SM 8 CTAs (else 8)
+  int tile = 64;
+  while (tile > 8 && ((d_out + 8 * tile - 1) / (8 * tile)) * p->nchunks < (int64_t)sms * 8) tile >>= 1;
   p->col_tile = tile;
-  p->ntile = (d_out + tile - 1) / tile;
+  p->ntile = (d_out + 8 * tile - 1) / (8 * tile);
+  // one-dimensional grids of the main passes
+  if ((d_out * (int64_t)p->nseg + 7) / 8 > 0x7FFFFFFF || p->ntile * p->nchunks > 0x7FFFFFFF) return BD_ERR_SHAPE;
   size_t off = kStatusBytes;
   p->off_clip = off;
   off = align_up(off + sizeof(ClipParams), 256);
@@ -589,12 +609,12 @@ bd_status launch_compress(const CompressPlan& p, const void* w_base, const void*
   }
   double* part = reinterpret_cast<double*>(ws + p.off_part);
   if (cfg->mode == BD_SCALE_COL) {
-    const int64_t tasks = p.ntile * p.nchunks;
-    const int64_t blocks = (tasks + 7) / 8;
+    const int64_t blocks = p.ntile * p.nchunks;  // grid limit checked in the plan
     launch_begin(K_COL_SCALE_SIGNPACK, s);
-    BD_CUDA_TRY(launch_pdl(k_col_scale_signpack<BF16>, dim3((unsigned)blocks), dim3(256), 0, s,
-                           (const uint8_t*)w_base, (const uint8_t*)w_fine, d_out, d_in, p.col_tile, p.nchunks,
-                           (const ClipParams*)clipp, signs, part));
+    auto kcol = clip ? k_col_scale_signpack<BF16, true> : k_col_scale_signpack<BF16, false>;
+    BD_CUDA_TRY(launch_pdl(kcol, dim3((unsigned)blocks), dim3(256), 0, s, (const uint8_t*)w_base,
+                           (const uint8_t*)w_fine, d_out, d_in, p.col_tile, p.nchunks, (const ClipParams*)clipp,
+                           signs, part));
     launch_end(K_COL_SCALE_SIGNPACK, s);
     BD_LAUNCH_CHECK();
     launch_begin(K_SCALE_FINAL, s);
