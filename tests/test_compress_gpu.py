@@ -125,6 +125,30 @@ def test_clip_flips_signs_when_bound_positive(bd):
     assert int(signs[0, 0]) == 0xFFFFFFFF
 
 
+@pytest.mark.parametrize("mode", [O.MODE_GROUP, O.MODE_BLOCK])
+@pytest.mark.parametrize("side", [1.0, -1.0])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_clip_bound_past_zero_rewrites_signs(bd, mode, side, dtype):
+    """A delta shifted so far that lo > 0 (side +1) or hi < 0 (side -1): the clamp moves
+    the far tail across zero, so the signs of every group with a clamped entry change;
+    G = 64 and 512 column groups (G x G blocks) over 130 rows."""
+    rng = np.random.default_rng(19 + int(side > 0) + 2 * mode)
+    for G in (64, 512):
+        d_out, d_in = 130, 1024
+        wb = rng.normal(0, 0.02, size=(d_out, d_in))
+        d = side * (5.0 + rng.normal(0, 1.0, size=(d_out, d_in)))
+        d[7, 3:40] = -side * 4.0  # far on the other side of zero
+        wf = wb + d
+        if dtype == "bf16":
+            wb, wf = bf16_bits(wb), bf16_bits(wf)
+        else:
+            wb, wf = wb.astype(np.float32), wf.astype(np.float32)
+        ref, signs, _ = _check(bd, wb, wf, dtype, mode, G, True, 3.0)
+        lo, hi = ref["stats"][2], ref["stats"][3]
+        assert (lo > 0) if side > 0 else (hi < 0)
+        assert int(signs[7, 1]) == (0xFFFFFFFF if side > 0 else 0)
+
+
 def test_bf16_llama_k_proj_full(bd):
     """Full k_proj shape (1024 x 4096, bf16), delta ~ N(0, 0.001), 0.05% outliers x30,
     group 128 with the 3-sigma clip; compared element by element."""
