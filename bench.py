@@ -60,10 +60,11 @@ def tc_min_tokens() -> int:
 # was built from: once they change, the number no longer describes the kernel and the
 # roofline reports traffic = null.
 NCU_TRAFFIC = {
-    # profiles/delta_lut_serving_layer.md: mean over the qkv, o, gate_up and down calls
-    # (each a quarter of a step's launches) of dram__bytes_read.sum + dram__bytes_write.sum
+    # ncu capture of the serving workload's 1-layer stack: mean over the qkv, o, gate_up and
+    # down calls (each a quarter of a step's launches) of dram__bytes_read.sum +
+    # dram__bytes_write.sum
     "delta_lut": {"sources": ["bd_delta_lut.cu", "bd_internal.cuh", "bd_tc.cuh"],
-                  "sha256_16": "26e40ca3b865e33c", "bytes_per_launch": 562501740.0},
+                  "sha256_16": "d61e003ad34c34dd", "bytes_per_launch": 586390980.0},
 }
 
 
