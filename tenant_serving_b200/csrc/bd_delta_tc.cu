@@ -52,12 +52,17 @@ constexpr uint32_t DT_WIN_SCALE_BYTES = 512;  // 128 rows x 2 fp16 (tiled group-
 // ------------------------------------------------------------------------------------
 // gather: X_u rows for every tensor-core segment, permuted and scaled into fp16 range
 // ------------------------------------------------------------------------------------
-// seg arrays: tc_tenant, tc_start, tc_count, tc_xrow (Xg row of the segment's first token)
-__global__ void __launch_bounds__(256) k_tc_gather(const int32_t* __restrict__ seg_base,
-                                                   int max_groups, int max_tc,
-                                                   const bd_tenant* __restrict__ tc_rec,
-                                                   const uint16_t* __restrict__ x, int64_t d_in,
-                                                   __half* __restrict__ xg, float* __restrict__ xinv) {
+// seg arrays: tc_tenant, tc_start, tc_count, tc_xrow (Xg row of the segment's first token).
+// One CTA of DT_GATHER_THREADS per Xg row (blockIdx.x: the row within its segment,
+// blockIdx.y: the segment): every thread takes 32-column blocks tid, tid + 128, ... of
+// the token, so the row's largest |value| is one pass of short per-thread loops and a CTA
+// reduction; the second pass re-reads the row (from L1 / L2) to scale and write it.
+constexpr int DT_GATHER_THREADS = 128;
+__global__ void __launch_bounds__(DT_GATHER_THREADS) k_tc_gather(const int32_t* __restrict__ seg_base,
+                                                                 int max_groups, int max_tc,
+                                                                 const bd_tenant* __restrict__ tc_rec,
+                                                                 const uint16_t* __restrict__ x, int64_t d_in,
+                                                                 __half* __restrict__ xg, float* __restrict__ xinv) {
   pdl_wait();  // inputs may come from the previous kernel on the stream
   pdl_trigger();
   const int n_tc = seg_base[1];
@@ -70,18 +75,18 @@ __global__ void __launch_bounds__(256) k_tc_gather(const int32_t* __restrict__ s
   const int32_t* permv = tc_xrow + max_tc;
   const int count = tc_count[sidx];
   const int npad = (count + 15) & ~15;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = blockIdx.x * 8 + warp;
-  if (r >= npad) return;
+  const int r = blockIdx.x;
+  if (r >= npad) return;  // CTA-uniform
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t xr = tc_xrow[sidx] + r;
   __half* out = xg + xr * d_in;
   const int nblk = (int)(d_in >> 5);
   if (r >= count) {
-    for (int b = lane; b < nblk; b += 32) {
+    for (int b = tid; b < nblk; b += DT_GATHER_THREADS) {
       uint4* o = reinterpret_cast<uint4*>(out + 32 * b);
       o[0] = o[1] = o[2] = o[3] = make_uint4(0, 0, 0, 0);
     }
-    if (lane == 0) xinv[xr] = 0.f;
+    if (tid == 0) xinv[xr] = 0.f;
     return;
   }
   const int t = permv[tc_start[sidx] + r];
@@ -118,9 +123,10 @@ __global__ void __launch_bounds__(256) k_tc_gather(const int32_t* __restrict__ s
     }
   };
   // largest |x| (|s x| for a COL tenant) of the token
+  __shared__ float wmax[DT_GATHER_THREADS / 32];
   float m = 0.f;
 #pragma unroll 2
-  for (int b = lane; b < nblk; b += 32) {
+  for (int b = tid; b < nblk; b += DT_GATHER_THREADS) {
     float v[32];
     load32(b, v);
 #pragma unroll
@@ -128,6 +134,10 @@ __global__ void __launch_bounds__(256) k_tc_gather(const int32_t* __restrict__ s
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) wmax[warp] = m;
+  __syncthreads();
+#pragma unroll
+  for (int w = 0; w < DT_GATHER_THREADS / 32; ++w) m = fmaxf(m, wmax[w]);
   int e = 0;
   if (m > 0.f) {
     int E;
@@ -137,7 +147,7 @@ __global__ void __launch_bounds__(256) k_tc_gather(const int32_t* __restrict__ s
   }
   const float sc = ldexpf(1.f, e);
 #pragma unroll 2
-  for (int b = lane; b < nblk; b += 32) {
+  for (int b = tid; b < nblk; b += DT_GATHER_THREADS) {
     float v[32];
     load32(b, v);
 #pragma unroll
@@ -155,7 +165,7 @@ __global__ void __launch_bounds__(256) k_tc_gather(const int32_t* __restrict__ s
     dst[2] = make_uint4(o[8], o[9], o[10], o[11]);
     dst[3] = make_uint4(o[12], o[13], o[14], o[15]);
   }
-  if (lane == 0) xinv[xr] = ldexpf(1.f, -e);
+  if (tid == 0) xinv[xr] = ldexpf(1.f, -e);
 }
 
 // ------------------------------------------------------------------------------------
@@ -637,9 +647,9 @@ bd_status launch_delta_tc(const bd_tenant* tc_rec, const int32_t* seg, int max_g
                           bool y_bf16, uint32_t* status, cudaStream_t s) {
   if (max_tc <= 0) return BD_OK;
   // 1. gather X of the tensor-core segments
-  dim3 gg(DT_NMAX / 8, (unsigned)max_tc);  // 8 rows per CTA
+  dim3 gg(DT_NMAX, (unsigned)max_tc);  // one CTA per Xg row
   launch_begin(K_TC_GATHER, s);
-  BD_CUDA_TRY(launch_pdl(k_tc_gather, gg, dim3(256), 0, s, seg, max_groups, max_tc, tc_rec,
+  BD_CUDA_TRY(launch_pdl(k_tc_gather, gg, dim3(DT_GATHER_THREADS), 0, s, seg, max_groups, max_tc, tc_rec,
                          static_cast<const uint16_t*>(x), d_in, xg, xinv));
   launch_end(K_TC_GATHER, s);
   BD_LAUNCH_CHECK();
