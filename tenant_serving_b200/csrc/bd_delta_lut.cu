@@ -363,10 +363,12 @@ __host__ __device__ __forceinline__ uint32_t dl_chunk_off(int c, bool single) {
 }
 
 // The lookups of one row-window: wd[i] = sign word (i + sigma) % 8 of the row, sc[i] its
-// scale. part[t] += sum over the window of sc * (table entry), token t.
+// scale. part[t] += sum over the window of sc * (table entry), token t; the even and odd
+// words accumulate in two independent chains (shorter dependency chains per lane).
 template <int NT>
 __device__ __forceinline__ void lut_row(const uint32_t (&wd)[8], const float (&sc)[8], const uint32_t (&K)[8][2],
                                         const uint32_t (&sel)[4], float* part) {
+  float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     // the word's four table reads per token, added as a tree (two dependent adds, not four)
@@ -382,11 +384,15 @@ __device__ __forceinline__ void lut_row(const uint32_t (&wd)[8], const float (&s
         if (NT == 4) f[j] = lds2_off<(int)DL_PAGE>(addr);
       }
     }
-    part[0] = fmaf(sc[i], (e[0].x + e[1].x) + (e[2].x + e[3].x), part[0]);
-    if (NT > 1) part[1] = fmaf(sc[i], (e[0].y + e[1].y) + (e[2].y + e[3].y), part[1]);
-    if (NT > 2) part[2] = fmaf(sc[i], (f[0].x + f[1].x) + (f[2].x + f[3].x), part[2]);
-    if (NT > 3) part[3] = fmaf(sc[i], (f[0].y + f[1].y) + (f[2].y + f[3].y), part[3]);
+    // even and odd words in two chains of running sums, added at the end
+    float* a = acc[i & 1];
+    a[0] = fmaf(sc[i], (e[0].x + e[1].x) + (e[2].x + e[3].x), a[0]);
+    if (NT > 1) a[1] = fmaf(sc[i], (e[0].y + e[1].y) + (e[2].y + e[3].y), a[1]);
+    if (NT > 2) a[2] = fmaf(sc[i], (f[0].x + f[1].x) + (f[2].x + f[3].x), a[2]);
+    if (NT > 3) a[3] = fmaf(sc[i], (f[0].y + f[1].y) + (f[2].y + f[3].y), a[3]);
   }
+#pragma unroll
+  for (int t = 0; t < NT; ++t) part[t] += acc[0][t] + acc[1][t];
 }
 
 // Tables of one window for the group's tokens, from the x slice (and column scales) in
