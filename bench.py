@@ -64,7 +64,7 @@ NCU_TRAFFIC = {
     # down calls (each a quarter of a step's launches) of dram__bytes_read.sum +
     # dram__bytes_write.sum
     "delta_lut": {"sources": ["bd_delta_lut.cu", "bd_internal.cuh", "bd_tc.cuh"],
-                  "sha256_16": "d61e003ad34c34dd", "bytes_per_launch": 586390980.0},
+                  "sha256_16": "706ffd8085fd8fc3", "bytes_per_launch": 586094528.0},
 }
 
 
